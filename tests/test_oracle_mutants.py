@@ -1,0 +1,55 @@
+"""Mutation check of the oracle's pins (CPU only).
+
+Each case plants one plausible mistake in a private copy of the oracle's C
+source (a flipped sign, a transposed or dropped index, a wrong tie rule, a
+missing gate, an unstable sort, the wrong rounding), builds it with gcc, and
+runs the pin tests against that build.  The pins must fail for every mutant;
+the product code is never involved.
+"""
+import os
+import re
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "adafuse_oracle.c")
+
+MUTANTS = {
+    "merge_gate_sign": (r"acc \+= g\[s\] \* d;", "acc -= g[s] * d;"),
+    "merge_A_transposed": (r"A\[e \* a_es \+ \(int64_t\)j \* d_in \+ i\]\);\n                acc \+= g",
+                           "A[e * a_es + (int64_t)i * r + j]);\n                acc += g"),
+    "merge_drop_last_rank_term": (r"for \(int32_t j = 0; j < r; \+\+j\)\n                    d \+= orc_bf16_to_double\(B\[e \* b_es \+ o \* r \+ j\]\) \*\n                         orc_bf16_to_double\(A",
+                                  "for (int32_t j = 0; j < r - 1; ++j)\n                    d += orc_bf16_to_double(B[e * b_es + o * r + j]) *\n                         orc_bf16_to_double(A"),
+    "topk_tie_to_higher_index": (r"    return a < b;\n}", "    return a > b;\n}"),
+    "router_bias_dropped": (r"            if \(br\) acc = acc \+ br\[e\];\n            z\[t \* E \+ e\] = acc;",
+                            "            z[t * E + e] = acc;"),
+    "softmax_always_renormalised": (r"if \(renorm\) for", "if (1) for"),
+    "apply_gate_missing": (r"acc \+= gate\[t \* k \+ s\] \* d;", "acc += d;"),
+    "apply_uses_W_transposed": (r"orc_bf16_to_double\(W\[o \* d_in \+ i\]\);",
+                                "orc_bf16_to_double(W[(i % d_out) * d_in + (o % d_in)]);"),
+    "segments_unstable": (r"    for \(int64_t p = 0; p < P; \+\+p\) \{\n        int32_t e = idx\[p\];\n        if \(e < 0 \|\| e >= E\) continue;",
+                          "    for (int64_t p = P - 1; p >= 0; --p) {\n        int32_t e = idx[p];\n        if (e < 0 || e >= E) continue;"),
+    "bf16_ties_away_from_zero": (r"double n = nearbyint\(a / q\);", "double n = round(a / q);"),
+    "router_fused_multiply_add": (r"                float p = xj \* Wr\[\(int64_t\)e \* H \+ j\];\n                acc = acc \+ p;",
+                                  "                acc = fmaf(xj, Wr[(int64_t)e * H + j], acc);"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_planted_mistake(name, tmp_path):
+    pat, rep = MUTANTS[name]
+    src = open(SRC).read()
+    mutated, n = re.subn(pat, lambda m: rep, src, count=1)
+    assert n == 1, f"mutation {name} did not apply"
+    csrc = tmp_path / "mutant.c"
+    csrc.write_text(mutated)
+    lib = tmp_path / "libmutant.so"
+    subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp",
+                           "-ffp-contract=off", "-o", str(lib), str(csrc), "-lm"])
+    env = dict(os.environ, ADAFUSE_ORACLE_LIB=str(lib))
+    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
+                        os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode != 0, f"pins did not catch mutant {name}:\n{r.stdout[-2000:]}"
