@@ -1,0 +1,495 @@
+// Segmented-gather apply for mixed-adapter batches (unmerged form):
+//   y_l = x_l W_l^T + sum_s g_s (x_l A_{e_s}^T) B_{e_s}^T     for every linear l.
+//
+// AdaFuse names the kernel "Segmented Gather Matrix Multiplication" (page pt
+// section 2.B); the pages print no formula for the unmerged form, so it is the
+// plain mixed-batch LoRA product above, per token with that token's top-k.
+//
+// Three launches per call, independent of the number of layers:
+//   1. segments  stable sort of the (token, slot) pairs by expert (segments.cu);
+//   2. shrink    for every (linear, used expert): the expert's segment of tokens
+//                times A_e^T, gate-scaled, rounded to bf16 into
+//                S_l[T, U*r] (column block q = the q-th used expert);
+//   3. apply     one persistent tcgen05 kernel over all (linear, 128-row) units:
+//                D[128 x Npad] = W_tile x^T (d_in/64 swizzled K chunks) then
+//                + Bcat_tile S^T (the used experts' B rows, gathered by TMA),
+//                all into one fp32 TMEM accumulator, then y = bf16(D^T).
+// W is streamed exactly once per token tile; the x and S tiles come from L2.
+#include <algorithm>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace af {
+
+namespace {
+
+// ------------------------------------------------------------------ workspace
+
+struct WsLayout {
+    size_t off_offsets, off_used, off_perm, off_S, total;
+    int32_t Umax, Kext;
+};
+
+WsLayout ws_layout(const Plan* p, int64_t T, int32_t k)
+{
+    WsLayout w{};
+    const int64_t P = T * k;
+    w.Umax = (int32_t)std::min<int64_t>(p->E, P);
+    w.Kext = ((w.Umax * p->r + 63) / 64) * 64;
+    w.off_offsets = 0;
+    w.off_used = 256;
+    w.off_perm = 512;
+    w.off_S = 512 + (((size_t)P * 4 + 255) / 256) * 256;
+    w.total = w.off_S + (((size_t)p->n_lin * (size_t)T * (size_t)w.Kext * 2 + 255) / 256) * 256;
+    return w;
+}
+
+// ------------------------------------------------------------------ shrink
+
+constexpr int kShrinkThreads = 256;
+constexpr int kShrinkChunk = 128;               // d_in columns per smem stage
+constexpr int kShrinkWords = kShrinkChunk / 2 + 1;   // padded row (bf16 pairs)
+
+__global__ void __launch_bounds__(kShrinkThreads) shrink_kernel(const LinDesc* lins, const uint16_t* const* x_ptrs,
+                                                                 int64_t T, int32_t k, int32_t r,
+                                                                 const int32_t* offsets, const int32_t* perm,
+                                                                 const int32_t* used, const float* gate, uint16_t* S,
+                                                                 int32_t Kext, int32_t Umax)
+{
+    extern __shared__ uint32_t sm_shrink[];
+    const int NB = max(1, kShrinkThreads / r);           // tokens per batch
+    uint32_t* As = sm_shrink;                            // [r][kShrinkWords]
+    uint32_t* Xs = As + r * kShrinkWords;                // [NB][kShrinkWords]
+    int* tok = reinterpret_cast<int*>(Xs + NB * kShrinkWords);   // [NB]
+    float* coef = reinterpret_cast<float*>(tok + NB);            // [NB]
+    __shared__ int s_nb, s_cursor;
+
+    const int l = blockIdx.x, q = blockIdx.y, tid = threadIdx.x;
+    const LinDesc L = lins[l];
+    const uint16_t* x = x_ptrs[l];
+    uint16_t* Sl = S + (int64_t)l * T * Kext;
+    const int U = used[0];
+
+    // Zero this block's columns for every token (and the padding columns).
+    {
+        const int c0 = q * r, c1 = (q == Umax - 1) ? Kext : (q + 1) * r;
+        const int per_row = (c1 - c0) / 8;
+        for (int64_t id = tid; id < T * per_row; id += kShrinkThreads) {
+            const int64_t t = id / per_row;
+            const int cc = (int)(id - t * per_row);
+            *reinterpret_cast<uint4*>(Sl + t * Kext + c0 + cc * 8) = make_uint4(0, 0, 0, 0);
+        }
+    }
+    if (q >= U) return;
+    const int e = used[1 + q];
+    const int seg0 = offsets[e], seg1 = offsets[e + 1];
+    const uint16_t* Ae = L.A + (int64_t)e * L.a_es;
+    if (tid == 0) s_cursor = seg0;
+    __syncthreads();
+
+    const int j = tid % r, bi = tid / r;
+    while (true) {
+        if (tid == 0) {
+            // Next batch of distinct tokens of this segment; pairs of one token
+            // are adjacent (ascending pair id), their gates add up.
+            int nb = 0, c = s_cursor;
+            while (c < seg1) {
+                const int pr = perm[c];
+                const int t = pr / k;
+                if (nb > 0 && tok[nb - 1] == t) { coef[nb - 1] += gate[pr]; ++c; continue; }
+                if (nb == NB) break;
+                tok[nb] = t;
+                coef[nb] = gate[pr];
+                ++nb;
+                ++c;
+            }
+            s_cursor = c;
+            s_nb = nb;
+        }
+        __syncthreads();
+        const int nb = s_nb;
+        if (nb == 0) break;
+        float acc = 0.f;
+        for (int c0 = 0; c0 < L.d_in; c0 += kShrinkChunk) {
+            // stage A_e rows and the batch's x rows (bf16 pairs, padded rows)
+            for (int id = tid; id < (r + nb) * (kShrinkChunk / 8); id += kShrinkThreads) {
+                const int row = id / (kShrinkChunk / 8), cc = id % (kShrinkChunk / 8);
+                const int col = c0 + cc * 8;
+                uint4 v = make_uint4(0, 0, 0, 0);
+                uint32_t* dst;
+                if (row < r) {
+                    if (col < L.d_in) v = ld_global_nc_v4(Ae + (int64_t)row * L.d_in + col);
+                    dst = As + row * kShrinkWords + cc * 4;
+                } else {
+                    const int bt = row - r;
+                    if (col < L.d_in) v = ld_global_nc_v4(x + (int64_t)tok[bt] * L.d_in + col);
+                    dst = Xs + bt * kShrinkWords + cc * 4;
+                }
+                dst[0] = v.x; dst[1] = v.y; dst[2] = v.z; dst[3] = v.w;
+            }
+            __syncthreads();
+            if (bi < nb) {
+                const uint32_t* ar = As + j * kShrinkWords;
+                const uint32_t* xr = Xs + bi * kShrinkWords;
+#pragma unroll 8
+                for (int w = 0; w < kShrinkChunk / 2; ++w) {
+                    const uint32_t aw = ar[w], xw = xr[w];
+                    acc = fmaf(bf16lo(xw), bf16lo(aw), acc);
+                    acc = fmaf(bf16hi(xw), bf16hi(aw), acc);
+                }
+            }
+            __syncthreads();
+        }
+        if (bi < nb) {
+            const float v = coef[bi] * acc;
+            Sl[(int64_t)tok[bi] * Kext + q * r + j] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+        }
+        __syncthreads();
+    }
+}
+
+// ------------------------------------------------------------------ apply
+
+struct ApplyArgs {
+    const LinDesc* lins;
+    const CUtensorMap* maps;
+    const uint16_t* const* x_ptrs;
+    uint16_t* const* y_ptrs;
+    const int32_t* used;
+    const uint16_t* S;
+    const int32_t* cta_start;
+    int32_t* status;
+    int64_t T;
+    int32_t n_lin, r, Kext, Npad, n_tt;
+    int32_t ST;
+    uint32_t stage_bytes, off_bar, acc_stride, tmem_cols;
+};
+
+constexpr int kApplyThreads = 256;
+constexpr uint32_t kAChunkBytes = kTileM * kChunkK * 2;     // 16 KB
+
+struct UnitIt {
+    int l, mt, n_rt;
+    __device__ void init(const LinDesc* lins, int n_lin, int64_t u)
+    {
+        int lo = 0, hi = n_lin - 1;
+        while (lo < hi) {
+            int mid = (lo + hi + 1) >> 1;
+            if (lins[mid].unit_base <= u) lo = mid; else hi = mid - 1;
+        }
+        l = lo;
+        n_rt = lins[l].n_rt;
+        mt = (int)(u - lins[l].unit_base);
+    }
+    __device__ void next(const LinDesc* lins, int n_lin)
+    {
+        if (++mt == n_rt) {
+            mt = 0;
+            if (++l < n_lin) n_rt = lins[l].n_rt;
+        }
+    }
+};
+
+__device__ __forceinline__ bool mbar_wait_drain2(uint64_t* bar, uint32_t parity)
+{
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+    }
+    return true;
+}
+
+__global__ void __launch_bounds__(kApplyThreads, 1) apply_fused_kernel(const __grid_constant__ ApplyArgs a)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(base + a.off_bar);
+    uint64_t* empty = full + a.ST;
+    uint64_t* accfull = empty + a.ST;
+    uint64_t* accempty = accfull + 2;
+    uint64_t* donebar = accempty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(donebar + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    int* s_used = reinterpret_cast<int*>(tmem_slot + 4);     // [1 + kMaxE]
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < a.ST; ++i) { mbar_init(&full[i], 1 + 64); mbar_init(&empty[i], 1); }
+        for (int i = 0; i < 2; ++i) { mbar_init(&accfull[i], 1); mbar_init(&accempty[i], 4); }
+        mbar_init(donebar, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (threadIdx.x <= kMaxE) s_used[threadIdx.x] = a.used[threadIdx.x];
+    // Zero the A regions: expert chunks load only the groups they use.
+    for (int s = 0; s < a.ST; ++s)
+        for (uint32_t o = threadIdx.x * 16; o < kAChunkBytes; o += kApplyThreads * 16)
+            st_shared_v4(smem_u32(base + (size_t)s * a.stage_bytes + o), make_uint4(0, 0, 0, 0));
+    fence_proxy_async_smem();
+    __syncthreads();
+    const int U = s_used[0];
+    const int nKe = (U * a.r + kChunkK - 1) / kChunkK;
+
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, a.tmem_cols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    const int u_begin = a.cta_start[blockIdx.x], u_end = a.cta_start[blockIdx.x + 1];
+    const int nunits = u_end - u_begin;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0 && nunits > 0) {
+            int64_t gc = 0, issued = 0;
+            bool stop = false;
+            for (int tt = 0; tt < a.n_tt && !stop; ++tt) {
+                UnitIt it;
+                it.init(a.lins, a.n_lin, u_begin);
+                for (int ui = 0; ui < nunits && !stop; ++ui) {
+                    const LinDesc& L = a.lins[it.l];
+                    const int nKb = (L.d_in + kChunkK - 1) / kChunkK;
+                    const int m0 = it.mt * kTileM;
+                    const CUtensorMap* mW = a.maps + (size_t)it.l * kMapsPerLinear + kMapW;
+                    const CUtensorMap* mB = a.maps + (size_t)it.l * kMapsPerLinear + kMapB;
+                    for (int kc = 0; kc < nKb + nKe; ++kc, ++gc) {
+                        const int s = (int)(gc % a.ST);
+                        if (!mbar_wait(&empty[s], (uint32_t)((gc / a.ST) & 1) ^ 1u, abort_flag)) { stop = true; break; }
+                        uint8_t* dst = base + (size_t)s * a.stage_bytes;
+                        if (kc < nKb) {
+                            mbar_arrive_expect_tx(&full[s], kAChunkBytes);
+                            tma_load_2d(dst, mW, &full[s], kc * kChunkK, m0);
+                        } else {
+                            const int col0 = (kc - nKb) * kChunkK;
+                            int ng = 0;
+                            for (int g = 0; g < 8; ++g) if (col0 + g * 8 < U * a.r) ++ng;
+                            mbar_arrive_expect_tx(&full[s], (uint32_t)ng * 2048u);
+                            for (int g = 0; g < 8; ++g) {
+                                const int c = col0 + g * 8;
+                                if (c >= U * a.r) break;
+                                const int qq = c / a.r, j0 = c - qq * a.r;
+                                tma_load_3d(dst + (size_t)g * 2048u, mB, &full[s], j0, m0, s_used[1 + qq]);
+                            }
+                        }
+                        issued = gc + 1;
+                    }
+                    if (ui + 1 < nunits) it.next(a.lins, a.n_lin);
+                }
+            }
+            // Drain the TMA loads still in flight (the last ST stages).  The
+            // loaders' cp.async arrivals complete the same phases.
+            for (int64_t g = std::max<int64_t>(0, issued - a.ST); g < issued; ++g)
+                mbar_wait_drain2(&full[g % a.ST], (uint32_t)((g / a.ST) & 1));
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0 && nunits > 0) {
+            const uint32_t idesc = make_idesc_bf16(kTileM, (uint32_t)a.Npad, 0u, 0u);
+            int64_t gc = 0;
+            int64_t uc = 0;
+            bool stop = false;
+            for (int tt = 0; tt < a.n_tt && !stop; ++tt) {
+                UnitIt it;
+                it.init(a.lins, a.n_lin, u_begin);
+                for (int ui = 0; ui < nunits && !stop; ++ui, ++uc) {
+                    const LinDesc& L = a.lins[it.l];
+                    const int nKb = (L.d_in + kChunkK - 1) / kChunkK;
+                    const int acc = (int)(uc & 1);
+                    if (!mbar_wait(&accempty[acc], (uint32_t)((uc >> 1) & 1) ^ 1u, abort_flag)) { stop = true; break; }
+                    tc_fence_after();
+                    const uint32_t d = tmem_base + (uint32_t)acc * a.acc_stride;
+                    for (int kc = 0; kc < nKb + nKe; ++kc, ++gc) {
+                        const int s = (int)(gc % a.ST);
+                        if (!mbar_wait(&full[s], (uint32_t)((gc / a.ST) & 1), abort_flag)) { stop = true; break; }
+                        tc_fence_after();
+                        fence_proxy_async_smem();
+                        const uint32_t aaddr = smem_u32(base + (size_t)s * a.stage_bytes);
+                        const uint32_t baddr = aaddr + kAChunkBytes;
+#pragma unroll
+                        for (int kk = 0; kk < kChunkK / 16; ++kk) {
+                            const uint64_t adesc = (kc < nKb)
+                                ? make_sdesc(aaddr + (uint32_t)kk * 32u, 16u, 1024u, kLayoutSw128)
+                                : make_sdesc(aaddr + (uint32_t)kk * 4096u, 2048u, 128u, kLayoutNone);
+                            const uint64_t bdesc = make_sdesc(baddr + (uint32_t)kk * 32u, 16u, 1024u, kLayoutSw128);
+                            tc_mma_bf16(d, adesc, bdesc, idesc, (kc | kk) ? 1u : 0u);
+                        }
+                        tc_commit(&empty[s]);
+                    }
+                    if (stop) break;
+                    tc_commit(&accfull[acc]);
+                    if (ui + 1 < nunits) it.next(a.lins, a.n_lin);
+                }
+            }
+            tc_commit(donebar);
+            mbar_wait_drain2(donebar, 0);
+        }
+        __syncwarp();
+    } else if (warp == 2 || warp == 3) {
+        // ------------------------------------------------------------ x / S loaders
+        if (nunits > 0) {
+            const int tl = (warp - 2) * 32 + lane;
+            int64_t gc = 0;
+            bool stop = false;
+            for (int tt = 0; tt < a.n_tt && !stop; ++tt) {
+                UnitIt it;
+                it.init(a.lins, a.n_lin, u_begin);
+                for (int ui = 0; ui < nunits && !stop; ++ui) {
+                    const LinDesc& L = a.lins[it.l];
+                    const int nKb = (L.d_in + kChunkK - 1) / kChunkK;
+                    const uint16_t* x = a.x_ptrs[it.l];
+                    const uint16_t* Sl = a.S + (int64_t)it.l * a.T * a.Kext;
+                    for (int kc = 0; kc < nKb + nKe; ++kc, ++gc) {
+                        const int s = (int)(gc % a.ST);
+                        bool ok = mbar_wait(&empty[s], (uint32_t)((gc / a.ST) & 1) ^ 1u, abort_flag);
+                        if (!__all_sync(0xffffffffu, ok)) { stop = true; break; }
+                        const uint32_t bdst = smem_u32(base + (size_t)s * a.stage_bytes + kAChunkBytes);
+                        for (int id = tl; id < a.Npad * 8; id += 64) {
+                            const int t = id >> 3, c = id & 7;
+                            const int64_t tabs = (int64_t)tt * kApplyMaxN + t;
+                            const uint32_t dst = bdst + (uint32_t)(t >> 3) * 1024u + (uint32_t)(t & 7) * 128u
+                                               + ((uint32_t)(c ^ (t & 7)) << 4);
+                            const uint16_t* src = x;
+                            uint32_t nbytes = 0;
+                            if (kc < nKb) {
+                                const int col = kc * kChunkK + c * 8;
+                                if (tabs < a.T && col < L.d_in) { src = x + tabs * L.d_in + col; nbytes = 16; }
+                            } else {
+                                const int col = (kc - nKb) * kChunkK + c * 8;
+                                if (tabs < a.T) { src = Sl + tabs * a.Kext + col; nbytes = 16; }
+                            }
+                            cp_async_16(dst, src, nbytes);
+                        }
+                        cp_async_mbar_arrive_noinc(&full[s]);
+                    }
+                    if (ui + 1 < nunits) it.next(a.lins, a.n_lin);
+                }
+            }
+            asm volatile("cp.async.wait_all;" ::: "memory");
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int q = warp & 3;
+        if (nunits > 0) {
+            int64_t uc = 0;
+            bool stop = false;
+            for (int tt = 0; tt < a.n_tt && !stop; ++tt) {
+                UnitIt it;
+                it.init(a.lins, a.n_lin, u_begin);
+                for (int ui = 0; ui < nunits; ++ui, ++uc) {
+                    const int acc = (int)(uc & 1);
+                    bool ok = mbar_wait(&accfull[acc], (uint32_t)((uc >> 1) & 1), abort_flag);
+                    if (!__all_sync(0xffffffffu, ok)) { stop = true; break; }
+                    tc_fence_after();
+                    const LinDesc& L = a.lins[it.l];
+                    uint16_t* y = a.y_ptrs[it.l];
+                    const int row = it.mt * kTileM + q * 32 + lane;
+                    const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)acc * a.acc_stride;
+                    for (int c0 = 0; c0 < a.Npad; c0 += 32) {
+                        uint32_t v[32];
+                        if (a.Npad - c0 >= 32) {
+                            tc_ld_x32(tbase + (uint32_t)c0, v);
+                        } else {
+                            uint32_t h[16];
+                            tc_ld_x16(tbase + (uint32_t)c0, h);
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) { v[i] = h[i]; v[16 + i] = 0; }
+                        }
+                        tc_wait_ld();
+                        if (row < L.d_out) {
+                            const int ncol = min(32, a.Npad - c0);
+                            for (int i = 0; i < ncol; ++i) {
+                                const int64_t t = (int64_t)tt * kApplyMaxN + c0 + i;
+                                if (t < a.T)
+                                    y[t * L.d_out + row] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[i])));
+                            }
+                        }
+                    }
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&accempty[acc]);
+                    if (ui + 1 < nunits) it.next(a.lins, a.n_lin);
+                }
+            }
+        }
+    }
+
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, a.tmem_cols);
+    }
+    if (threadIdx.x == 0 && *abort_flag) atomicOr(a.status, ADAFUSE_STATUS_TIMEOUT);
+}
+
+}  // namespace
+
+size_t apply_workspace_bytes(const Plan* p, int64_t T, int32_t k)
+{
+    return ws_layout(p, T, k).total;
+}
+
+int launch_apply(Plan* p, const void* const* x_ptrs, void* const* y_ptrs, int64_t T, const int32_t* idx,
+                 const float* gate, int32_t k, void* ws, size_t ws_bytes, cudaStream_t s)
+{
+    const WsLayout w = ws_layout(p, T, k);
+    if (ws_bytes < w.total) return ADAFUSE_ERR_WORKSPACE_TOO_SMALL;
+    uint8_t* wsb = static_cast<uint8_t*>(ws);
+    int32_t* offsets = reinterpret_cast<int32_t*>(wsb + w.off_offsets);
+    int32_t* used = reinterpret_cast<int32_t*>(wsb + w.off_used);
+    int32_t* perm = reinterpret_cast<int32_t*>(wsb + w.off_perm);
+    uint16_t* S = reinterpret_cast<uint16_t*>(wsb + w.off_S);
+
+    int rc = launch_segments(idx, T, k, p->E, offsets, perm, used, p->d_status, s);
+    if (rc != ADAFUSE_OK) return rc;
+
+    const int NB = std::max(1, kShrinkThreads / p->r);
+    const size_t shrink_smem = (size_t)(p->r + NB) * kShrinkWords * 4 + (size_t)NB * 8;
+    if (shrink_smem > 48 * 1024) {
+        if (cudaFuncSetAttribute(shrink_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)shrink_smem) != cudaSuccess)
+            return ADAFUSE_ERR_CUDA;
+    }
+    shrink_kernel<<<dim3((unsigned)p->n_lin, (unsigned)w.Umax), kShrinkThreads, shrink_smem, s>>>(
+        p->d_desc, reinterpret_cast<const uint16_t* const*>(x_ptrs), T, k, p->r, offsets, perm, used, gate, S, w.Kext,
+        w.Umax);
+    if (cudaGetLastError() != cudaSuccess) return ADAFUSE_ERR_CUDA;
+
+    ApplyArgs a{};
+    a.lins = p->d_desc;
+    a.maps = p->d_maps;
+    a.x_ptrs = reinterpret_cast<const uint16_t* const*>(x_ptrs);
+    a.y_ptrs = reinterpret_cast<uint16_t* const*>(y_ptrs);
+    a.used = used;
+    a.S = S;
+    a.cta_start = p->d_apply_start;
+    a.status = p->d_status;
+    a.T = T;
+    a.n_lin = p->n_lin;
+    a.r = p->r;
+    a.Kext = w.Kext;
+    a.n_tt = (int32_t)((T + kApplyMaxN - 1) / kApplyMaxN);
+    a.Npad = (int32_t)std::min<int64_t>(kApplyMaxN, ((T + 15) / 16) * 16);
+    a.stage_bytes = kAChunkBytes + (uint32_t)a.Npad * 128u;
+    uint32_t accs = 32;
+    while (accs < (uint32_t)a.Npad) accs <<= 1;
+    a.acc_stride = accs;
+    a.tmem_cols = 2 * accs;
+    const uint32_t kSmemMax = 232448u;
+    int ST = (int)((kSmemMax - 2048u) / a.stage_bytes);
+    ST = std::min(ST, 8);
+    if (ST < 2) return ADAFUSE_ERR_UNSUPPORTED;
+    a.ST = ST;
+    a.off_bar = (uint32_t)ST * a.stage_bytes;
+    const uint32_t smem = a.off_bar + 1024u + 1024u;
+    if (cudaFuncSetAttribute(apply_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+        return ADAFUSE_ERR_CUDA;
+    apply_fused_kernel<<<p->apply_grid, kApplyThreads, smem, s>>>(a);
+    p->last_launches = 3;
+    return cuda_err(cudaGetLastError());
+}
+
+}  // namespace af

@@ -1,0 +1,76 @@
+// Internal declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <vector>
+
+#include "../../include/adafuse.h"
+
+namespace af {
+
+// One targeted linear as the kernels see it (device table, built once).
+struct LinDesc {
+    const uint16_t* W;
+    uint16_t* W_out;
+    const uint16_t* A;
+    const uint16_t* B;
+    int64_t a_es;          // expert stride of A, elements
+    int64_t b_es;          // expert stride of B, elements
+    int64_t tile_base;     // first merge tile (128 x 128) of this linear
+    int64_t unit_base;     // first apply unit (128 output rows) of this linear
+    int32_t d_out, d_in;
+    int32_t n_rt;          // ceil(d_out / 128)
+    int32_t n_strips;      // ceil(d_in / 128)
+};
+
+// Tensor maps kept per linear: W (load), W_out (load/store), B (3-D stack).
+constexpr int kMapsPerLinear = 3;
+constexpr int kMapW = 0, kMapWout = 1, kMapB = 2;
+
+constexpr int kTileM = 128;      // output rows per tile (MMA M, TMEM lanes)
+constexpr int kTileN = 128;      // merge: d_in columns per tile (MMA N)
+constexpr int kChunkK = 64;      // apply: d_in per pipeline stage (one 128-byte swizzle row)
+constexpr int kMaxSlots = ADAFUSE_MAX_SLOTS;
+constexpr int kMaxKr = ADAFUSE_MAX_KR;
+constexpr int kMaxE = ADAFUSE_MAX_E;
+constexpr int kApplyMaxN = 256;  // tokens per apply tile (MMA N)
+
+struct Plan {
+    int device = 0;
+    int num_sms = 0;
+    int n_lin = 0, E = 0, r = 0;
+    uint32_t flags = 0;
+    std::vector<adafuse_linear> lins;
+    std::vector<LinDesc> h_desc;
+    LinDesc* d_desc = nullptr;
+    CUtensorMap* d_maps = nullptr;
+    int32_t* d_status = nullptr;
+    int64_t merge_tiles = 0;
+    int64_t apply_units = 0;
+    int32_t apply_grid = 0;
+    int32_t* d_apply_start = nullptr;   // [apply_grid + 1] first unit per CTA
+    int32_t last_launches = 0;
+};
+
+}  // namespace af
+
+struct adafuse_plan : public af::Plan {};
+
+namespace af {
+
+// Launchers (defined in the .cu files).  All return ADAFUSE_* codes.
+int launch_merge_fused(Plan* p, const int32_t* idx0, const float* gate0, const int32_t* idx1,
+                       const float* gate1, int32_t k, int mode, cudaStream_t s);
+int launch_merge_per_linear(Plan* p, const int32_t* idx, const float* gate, int32_t k, cudaStream_t s);
+int launch_segments(const int32_t* idx, int64_t T, int32_t k, int32_t E, int32_t* offsets, int32_t* perm,
+                    int32_t* used, int32_t* status, cudaStream_t s);
+size_t apply_workspace_bytes(const Plan* p, int64_t T, int32_t k);
+int launch_apply(Plan* p, const void* const* x_ptrs, void* const* y_ptrs, int64_t T, const int32_t* idx,
+                 const float* gate, int32_t k, void* ws, size_t ws_bytes, cudaStream_t s);
+
+inline int cuda_err(cudaError_t e) { return e == cudaSuccess ? ADAFUSE_OK : ADAFUSE_ERR_CUDA; }
+
+}  // namespace af

@@ -1,0 +1,500 @@
+// Fused all-layer LoRA merge (SGMM), its in-place switch variant, and the
+// per-linear baseline.
+//
+// AdaFuse, page pt section 2.B ("Fusao de Adaptadores e Kernel SGMM") and page
+// ja section 2.2: the activated adapters' down (A) and up (B) projections are
+// concatenated and fused into the backbone weight of every targeted linear,
+// W' = W + sum_s g_s B_{e_s} A_{e_s}, in a single kernel launch across layers,
+// with the large product split into GEMM tiles assigned to thread blocks and a
+// prefetch buffer hiding global->shared latency.
+//
+// B200 design (one persistent CTA per SM, warp-specialised):
+//   warp 0      TMA producer: W tile (128 rows x 128 cols, two 64-column boxes,
+//               128-byte swizzle) into a W ring; the selected experts' B rows
+//               (128 x k*r, no swizzle) into a B ring.
+//   warp 1      allocates TMEM (2 x 128 fp32 columns) and issues tcgen05.mma:
+//               dW tile = Bcat[128 x Kp] * Acat[Kp x 128] into TMEM, K = k*r.
+//   warps 2-3   build Acat for a 128-column strip once per strip: gate-scaled
+//               A rows (fp32 multiply, bf16 round) in the MN-major core-matrix
+//               layout; double-buffered, reused by every row tile of the strip.
+//   warps 4-11  epilogue: dW from TMEM (tcgen05.ld), W from the swizzled smem
+//               tile, W + dW rounded to bf16 in place, then one thread stores
+//               the tile with TMA.  The stage is released once the store has
+//               read it.
+// HBM traffic is W read + W' write (4 bytes per element) plus the selected
+// adapters; the tensor cores carry the rank-(k*r) contraction (16*k*r/4 FLOP/B).
+#include <algorithm>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace af {
+
+namespace {
+
+struct MergeArgs {
+    const LinDesc* lins;
+    const CUtensorMap* maps;
+    const int32_t* idx0;
+    const float* gate0;
+    const int32_t* idx1;
+    const float* gate1;
+    int32_t* status;
+    int64_t total_tiles;
+    int32_t n_lin;
+    int32_t E, r;
+    int32_t k;          // slots per selection
+    int32_t ns;         // slots in this pass: k (merge) or 2k (switch)
+    int32_t Kp;         // ns*r rounded up to 16
+    int32_t mode;       // 0: merge W -> W_out; 1: switch, W_out in place
+    int32_t SW, SB, NA; // W stages, B stages, A buffers
+    uint32_t off_B, off_A, off_bar;
+};
+
+constexpr int kMergeThreads = 384;
+constexpr uint32_t kWTileBytes = kTileM * kTileN * 2;       // 32 KB
+constexpr uint32_t kWBoxBytes = kWTileBytes / 2;            // 16 KB: 64 cols x 128 rows
+constexpr int kEpiWarps = 8;
+
+struct TileIt {
+    int l, strip, rt, n_rt, n_strips;
+    __device__ void init(const LinDesc* lins, int n_lin, int64_t g)
+    {
+        int lo = 0, hi = n_lin - 1;
+        while (lo < hi) {
+            int mid = (lo + hi + 1) >> 1;
+            if (lins[mid].tile_base <= g) lo = mid; else hi = mid - 1;
+        }
+        l = lo;
+        n_rt = lins[l].n_rt;
+        n_strips = lins[l].n_strips;
+        int64_t local = g - lins[l].tile_base;
+        strip = (int)(local / n_rt);
+        rt = (int)(local - (int64_t)strip * n_rt);
+    }
+    __device__ void next(const LinDesc* lins, int n_lin)
+    {
+        if (++rt == n_rt) {
+            rt = 0;
+            if (++strip == n_strips) {
+                strip = 0;
+                if (++l < n_lin) {
+                    n_rt = lins[l].n_rt;
+                    n_strips = lins[l].n_strips;
+                }
+            }
+        }
+    }
+};
+
+// Wait that ignores the abort flag (used to drain in-flight async work).
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity)
+{
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+    }
+    return true;
+}
+
+__device__ __forceinline__ uint4 scale_bf16x8(uint4 raw, float g)
+{
+    uint4 o;
+    o.x = pack_bf16x2(bf16lo(raw.x) * g, bf16hi(raw.x) * g);
+    o.y = pack_bf16x2(bf16lo(raw.y) * g, bf16hi(raw.y) * g);
+    o.z = pack_bf16x2(bf16lo(raw.z) * g, bf16hi(raw.z) * g);
+    o.w = pack_bf16x2(bf16lo(raw.w) * g, bf16hi(raw.w) * g);
+    return o;
+}
+
+__device__ __forceinline__ uint32_t add_bf16x2(uint32_t w, uint32_t d0, uint32_t d1)
+{
+    return pack_bf16x2(bf16lo(w) + __uint_as_float(d0), bf16hi(w) + __uint_as_float(d1));
+}
+
+__global__ void __launch_bounds__(kMergeThreads, 1) merge_fused_kernel(const __grid_constant__ MergeArgs a)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sW = base;
+    uint8_t* sB = base + a.off_B;
+    uint8_t* sA = base + a.off_A;
+    uint64_t* wfull = reinterpret_cast<uint64_t*>(base + a.off_bar);
+    uint64_t* wempty = wfull + a.SW;
+    uint64_t* bfull = wempty + a.SW;
+    uint64_t* bempty = bfull + a.SB;
+    uint64_t* afull = bempty + a.SB;
+    uint64_t* aempty = afull + a.NA;
+    uint64_t* accfull = aempty + a.NA;
+    uint64_t* accempty = accfull + 2;
+    uint64_t* donebar = accempty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(donebar + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    int* s_skip = reinterpret_cast<int*>(tmem_slot + 2);
+    int* s_e = reinterpret_cast<int*>(tmem_slot + 4);
+    float* s_g = reinterpret_cast<float*>(s_e + kMaxSlots);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t BBytes = (uint32_t)a.Kp * 256u;     // 128 rows x Kp bf16
+    const uint32_t ABytes = (uint32_t)a.Kp * 256u;     // Kp rows x 128 cols bf16
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < a.SW; ++i) { mbar_init(&wfull[i], 1); mbar_init(&wempty[i], 1); }
+        for (int i = 0; i < a.SB; ++i) { mbar_init(&bfull[i], 1); mbar_init(&bempty[i], 1); }
+        for (int i = 0; i < a.NA; ++i) { mbar_init(&afull[i], 2); mbar_init(&aempty[i], 1); }
+        for (int i = 0; i < 2; ++i) { mbar_init(&accfull[i], 1); mbar_init(&accempty[i], kEpiWarps); }
+        mbar_init(donebar, 1);
+        *abort_flag = 0;
+        int bad = 0;
+        int same = 1;
+        for (int s = 0; s < a.ns; ++s) {
+            int e;
+            float g;
+            if (s < a.k) { e = a.idx0[s]; g = a.gate0[s]; }
+            else { e = a.idx1[s - a.k]; g = -a.gate1[s - a.k]; }
+            if (e < 0 || e >= a.E) { bad = 1; e = -1; g = 0.f; }
+            s_e[s] = e;
+            s_g[s] = g;
+        }
+        if (a.mode == 1) {
+            for (int s = 0; s < a.k; ++s)
+                if (a.idx0[s] != a.idx1[s] || __float_as_uint(a.gate0[s]) != __float_as_uint(a.gate1[s])) same = 0;
+        } else {
+            same = 0;
+        }
+        *s_skip = same;
+        if (bad && blockIdx.x == 0) atomicOr(a.status, ADAFUSE_STATUS_BAD_INDEX);
+        fence_mbar_init();
+    }
+    // Zero the B ring: stages of skipped slots and the K padding stay zero.
+    for (uint32_t o = threadIdx.x * 16; o < (uint32_t)a.SB * BBytes; o += kMergeThreads * 16)
+        st_shared_v4(smem_u32(sB + o), make_uint4(0, 0, 0, 0));
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (*s_skip) return;       // switch between identical selections: nothing to do
+
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, 256);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    const int64_t G = gridDim.x;
+    const int64_t t_begin = (int64_t)blockIdx.x * a.total_tiles / G;
+    const int64_t t_end = ((int64_t)blockIdx.x + 1) * a.total_tiles / G;
+    const int64_t count = t_end - t_begin;
+    const int kmap_in = a.mode == 1 ? kMapWout : kMapW;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0 && count > 0) {
+            TileIt it;
+            it.init(a.lins, a.n_lin, t_begin);
+            int nbox = 0;
+            for (int s = 0; s < a.ns; ++s) if (s_e[s] >= 0) nbox += a.r / 8;
+            const uint32_t bbytes = (uint32_t)nbox * 2048u;
+            int64_t issued_w = 0, issued_b = 0;
+            for (int64_t i = 0; i < count; ++i) {
+                const int sw = (int)(i % a.SW);
+                if (!mbar_wait(&wempty[sw], (uint32_t)((i / a.SW) & 1) ^ 1u, abort_flag)) break;
+                const CUtensorMap* mW = a.maps + (size_t)it.l * kMapsPerLinear + kmap_in;
+                const int n0 = it.strip * kTileN, m0 = it.rt * kTileM;
+                uint8_t* dstW = sW + (size_t)sw * kWTileBytes;
+                mbar_arrive_expect_tx(&wfull[sw], kWTileBytes);
+                tma_load_2d(dstW, mW, &wfull[sw], n0, m0);
+                tma_load_2d(dstW + kWBoxBytes, mW, &wfull[sw], n0 + 64, m0);
+                issued_w = i + 1;
+
+                const int sb = (int)(i % a.SB);
+                if (!mbar_wait(&bempty[sb], (uint32_t)((i / a.SB) & 1) ^ 1u, abort_flag)) break;
+                const CUtensorMap* mB = a.maps + (size_t)it.l * kMapsPerLinear + kMapB;
+                uint8_t* dstB = sB + (size_t)sb * BBytes;
+                mbar_arrive_expect_tx(&bfull[sb], bbytes);
+                for (int s = 0; s < a.ns; ++s) {
+                    const int e = s_e[s];
+                    if (e < 0) continue;
+                    for (int jg = 0; jg < a.r / 8; ++jg)
+                        tma_load_3d(dstB + (size_t)((s * a.r) / 8 + jg) * 2048u, mB, &bfull[sb], jg * 8, m0, e);
+                }
+                issued_b = i + 1;
+                if (i + 1 < count) it.next(a.lins, a.n_lin);
+            }
+            // Drain: the loads this thread issued must land before the CTA exits.
+            for (int64_t j = std::max<int64_t>(0, issued_w - a.SW); j < issued_w; ++j)
+                mbar_wait_drain(&wfull[j % a.SW], (uint32_t)((j / a.SW) & 1));
+            for (int64_t j = std::max<int64_t>(0, issued_b - a.SB); j < issued_b; ++j)
+                mbar_wait_drain(&bfull[j % a.SB], (uint32_t)((j / a.SB) & 1));
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0 && count > 0) {
+            TileIt it;
+            it.init(a.lins, a.n_lin, t_begin);
+            const uint32_t idesc = make_idesc_bf16(kTileM, kTileN, 0u, 1u);
+            const uint32_t sbo_a = (uint32_t)a.Kp * 16u;     // n-group stride of Acat
+            int64_t strip_seq = -1;
+            for (int64_t i = 0; i < count; ++i) {
+                const bool first = (i == 0) || (it.rt == 0);
+                const bool last = (i + 1 == count) || (it.rt == it.n_rt - 1);
+                if (first) ++strip_seq;
+                const int ab = (int)(strip_seq % a.NA);
+                const int sb = (int)(i % a.SB);
+                const int acc = (int)(i & 1);
+                if (!mbar_wait(&bfull[sb], (uint32_t)((i / a.SB) & 1), abort_flag)) break;
+                if (first && !mbar_wait(&afull[ab], (uint32_t)((strip_seq / a.NA) & 1), abort_flag)) break;
+                if (!mbar_wait(&accempty[acc], (uint32_t)((i >> 1) & 1) ^ 1u, abort_flag)) break;
+                tc_fence_after();
+                const uint32_t d = tmem_base + (uint32_t)acc * kTileN;
+                const uint32_t baddr = smem_u32(sB + (size_t)sb * BBytes);
+                const uint32_t aaddr = smem_u32(sA + (size_t)ab * ABytes);
+                for (int kk = 0; kk < a.Kp / 16; ++kk) {
+                    const uint64_t adesc = make_sdesc(baddr + (uint32_t)kk * 4096u, 2048u, 128u, kLayoutNone);
+                    const uint64_t bdesc = make_sdesc(aaddr + (uint32_t)kk * 256u, 128u, sbo_a, kLayoutNone);
+                    tc_mma_bf16(d, adesc, bdesc, idesc, kk > 0 ? 1u : 0u);
+                }
+                tc_commit(&accfull[acc]);
+                tc_commit(&bempty[sb]);
+                if (last) tc_commit(&aempty[ab]);
+                if (i + 1 < count) it.next(a.lins, a.n_lin);
+            }
+            tc_commit(donebar);
+            mbar_wait_drain(donebar, 0);
+        }
+        __syncwarp();
+    } else if (warp == 2 || warp == 3) {
+        // ------------------------------------------------------------ Acat builder
+        if (count > 0) {
+            const int tb = (warp - 2) * 32 + lane;
+            const uint32_t sbo_a = (uint32_t)a.Kp * 16u;
+            TileIt it;
+            it.init(a.lins, a.n_lin, t_begin);
+            int64_t strip_seq = -1;
+            for (int64_t i = 0; i < count; ++i) {
+                if (i == 0 || it.rt == 0) {
+                    ++strip_seq;
+                    const int ab = (int)(strip_seq % a.NA);
+                    bool ok = mbar_wait(&aempty[ab], (uint32_t)((strip_seq / a.NA) & 1) ^ 1u, abort_flag);
+                    ok = __all_sync(0xffffffffu, ok);
+                    if (!ok) break;
+                    const LinDesc L = a.lins[it.l];
+                    const int n0 = it.strip * kTileN;
+                    const uint32_t abase = smem_u32(sA + (size_t)ab * ABytes);
+                    const int total = a.Kp * 16;         // (row c, 8-column group) pairs
+                    for (int id0 = 0; id0 < total; id0 += 64 * 8) {
+                        uint4 v[8];
+                        float gs[8];
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) {
+                            const int id = id0 + u * 64 + tb;
+                            v[u] = make_uint4(0, 0, 0, 0);
+                            gs[u] = 0.f;
+                            if (id < total) {
+                                const int c = id >> 4, ng = id & 15;
+                                const int s = c / a.r, j = c - s * a.r;
+                                const int col = n0 + ng * 8;
+                                if (s < a.ns && s_e[s] >= 0 && col < L.d_in) {
+                                    v[u] = ld_global_nc_v4(L.A + (int64_t)s_e[s] * L.a_es + (int64_t)j * L.d_in + col);
+                                    gs[u] = s_g[s];
+                                }
+                            }
+                        }
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) {
+                            const int id = id0 + u * 64 + tb;
+                            if (id < total) {
+                                const int c = id >> 4, ng = id & 15;
+                                st_shared_v4(abase + (uint32_t)ng * sbo_a + (uint32_t)(c >> 3) * 128u + (uint32_t)(c & 7) * 16u,
+                                             scale_bf16x8(v[u], gs[u]));
+                            }
+                        }
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&afull[ab]);
+                }
+                if (i + 1 < count) it.next(a.lins, a.n_lin);
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int ew = warp - 4;            // 0..7
+        const int q = warp & 3;             // TMEM lane quarter this warp may access
+        const int h = ew >> 2;              // column half (64 columns)
+        const int row = q * 32 + lane;
+        const bool leader = (ew == 0 && lane == 0);
+        bool aborted = false;
+        TileIt it;
+        if (count > 0) it.init(a.lins, a.n_lin, t_begin);
+        for (int64_t i = 0; i < count; ++i) {
+            const int acc = (int)(i & 1);
+            const int sw = (int)(i % a.SW);
+            bool ok = mbar_wait(&accfull[acc], (uint32_t)((i >> 1) & 1), abort_flag);
+            ok = ok && mbar_wait(&wfull[sw], (uint32_t)((i / a.SW) & 1), abort_flag);
+            ok = __all_sync(0xffffffffu, ok);
+            if (ok) {
+                tc_fence_after();
+                uint32_t va[32], vb[32];
+                const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)acc * kTileN + (uint32_t)h * 64u;
+                tc_ld_x32(taddr, va);
+                tc_ld_x32(taddr + 32u, vb);
+                tc_wait_ld();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&accempty[acc]);
+                const uint32_t wrow = smem_u32(sW + (size_t)sw * kWTileBytes + (size_t)h * kWBoxBytes) + (uint32_t)row * 128u;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const uint32_t addr = wrow + ((uint32_t)(c ^ (row & 7)) << 4);
+                    const uint4 w = ld_shared_v4(addr);
+                    const uint32_t* d = (c < 4) ? &va[c * 8] : &vb[(c - 4) * 8];
+                    uint4 o;
+                    o.x = add_bf16x2(w.x, d[0], d[1]);
+                    o.y = add_bf16x2(w.y, d[2], d[3]);
+                    o.z = add_bf16x2(w.z, d[4], d[5]);
+                    o.w = add_bf16x2(w.w, d[6], d[7]);
+                    st_shared_v4(addr, o);
+                }
+                fence_proxy_async_smem();
+            }
+            if (named_bar_red_or(1, kEpiWarps * 32, !ok || *abort_flag != 0)) { aborted = true; break; }
+            if (leader) {
+                const CUtensorMap* mO = a.maps + (size_t)it.l * kMapsPerLinear + kMapWout;
+                const int n0 = it.strip * kTileN, m0 = it.rt * kTileM;
+                uint8_t* src = sW + (size_t)sw * kWTileBytes;
+                tma_store_2d(mO, src, n0, m0);
+                tma_store_2d(mO, src + kWBoxBytes, n0 + 64, m0);
+                bulk_commit_group();
+                bulk_wait_group_read<1>();
+                if (i > 0) mbar_arrive(&wempty[(i - 1) % a.SW]);
+            }
+            if (i + 1 < count) it.next(a.lins, a.n_lin);
+        }
+        if (leader) {
+            bulk_wait_group<0>();
+            if (count > 0 && !aborted) mbar_arrive(&wempty[(count - 1) % a.SW]);
+        }
+    }
+
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, 256);
+    }
+    if (threadIdx.x == 0 && *abort_flag) atomicOr(a.status, ADAFUSE_STATUS_TIMEOUT);
+}
+
+// ------------------------------------------------------------------ baseline
+
+// One launch per linear; each thread produces 8 consecutive outputs of a row
+// with CUDA-core FMAs straight from global memory.
+__global__ void __launch_bounds__(128) merge_per_linear_kernel(LinDesc L, const int32_t* idx, const float* gate,
+                                                                int32_t k, int32_t E, int32_t r, int32_t* status)
+{
+    __shared__ int s_e[kMaxSlots];
+    __shared__ float s_g[kMaxSlots];
+    if (threadIdx.x < k) {
+        int e = idx[threadIdx.x];
+        float g = gate[threadIdx.x];
+        if (e < 0 || e >= E) {
+            if (blockIdx.x == 0 && blockIdx.y == 0) atomicOr(status, ADAFUSE_STATUS_BAD_INDEX);
+            e = -1;
+            g = 0.f;
+        }
+        s_e[threadIdx.x] = e;
+        s_g[threadIdx.x] = g;
+    }
+    __syncthreads();
+    const int o = blockIdx.y;
+    const int i0 = (blockIdx.x * blockDim.x + threadIdx.x) * 8;
+    if (i0 >= L.d_in) return;
+    const uint4 w = ld_global_nc_v4(L.W + (int64_t)o * L.d_in + i0);
+    float acc[8] = {bf16lo(w.x), bf16hi(w.x), bf16lo(w.y), bf16hi(w.y),
+                    bf16lo(w.z), bf16hi(w.z), bf16lo(w.w), bf16hi(w.w)};
+    for (int s = 0; s < k; ++s) {
+        const int e = s_e[s];
+        if (e < 0) continue;
+        const float g = s_g[s];
+        const uint16_t* Bo = L.B + (int64_t)e * L.b_es + (int64_t)o * r;
+        const uint16_t* Ae = L.A + (int64_t)e * L.a_es + i0;
+        for (int j = 0; j < r; ++j) {
+            const float b = g * __uint_as_float((uint32_t)Bo[j] << 16);
+            const uint4 av = ld_global_nc_v4(Ae + (int64_t)j * L.d_in);
+            acc[0] += b * bf16lo(av.x); acc[1] += b * bf16hi(av.x);
+            acc[2] += b * bf16lo(av.y); acc[3] += b * bf16hi(av.y);
+            acc[4] += b * bf16lo(av.z); acc[5] += b * bf16hi(av.z);
+            acc[6] += b * bf16lo(av.w); acc[7] += b * bf16hi(av.w);
+        }
+    }
+    uint4 out;
+    out.x = pack_bf16x2(acc[0], acc[1]);
+    out.y = pack_bf16x2(acc[2], acc[3]);
+    out.z = pack_bf16x2(acc[4], acc[5]);
+    out.w = pack_bf16x2(acc[6], acc[7]);
+    *reinterpret_cast<uint4*>(L.W_out + (int64_t)o * L.d_in + i0) = out;
+}
+
+}  // namespace
+
+int launch_merge_fused(Plan* p, const int32_t* idx0, const float* gate0, const int32_t* idx1,
+                       const float* gate1, int32_t k, int mode, cudaStream_t s)
+{
+    MergeArgs a{};
+    a.lins = p->d_desc;
+    a.maps = p->d_maps;
+    a.idx0 = idx0; a.gate0 = gate0;
+    a.idx1 = idx1 ? idx1 : idx0; a.gate1 = gate1 ? gate1 : gate0;
+    a.status = p->d_status;
+    a.total_tiles = p->merge_tiles;
+    a.n_lin = p->n_lin;
+    a.E = p->E; a.r = p->r; a.k = k;
+    a.ns = mode == 1 ? 2 * k : k;
+    a.Kp = ((a.ns * p->r + 15) / 16) * 16;
+    a.mode = mode;
+    if (a.ns > kMaxSlots || a.Kp > kMaxKr) return ADAFUSE_ERR_UNSUPPORTED;
+
+    const uint32_t BBytes = (uint32_t)a.Kp * 256u;
+    const uint32_t ABytes = BBytes;
+    const uint32_t kSmemMax = 232448u;                  // 227 KB opt-in per block
+    const uint32_t extra = 1024u /*alignment*/ + 1024u /*barriers, slots*/;
+    int NA = 2, SB = 2, SW = 0;
+    auto fits = [&](int sw, int sb, int na) {
+        return (uint64_t)sw * kWTileBytes + (uint64_t)sb * BBytes + (uint64_t)na * ABytes + extra <= kSmemMax;
+    };
+    // The epilogue releases a W stage one tile late (after the next tile's
+    // store has been issued), so the W ring needs at least two stages.
+    for (int sw = 6; sw >= 2 && SW == 0; --sw) if (fits(sw, SB, NA)) SW = sw;
+    if (SW == 0) { NA = 1; SB = 2; for (int sw = 6; sw >= 2 && SW == 0; --sw) if (fits(sw, SB, NA)) SW = sw; }
+    if (SW == 0) { NA = 1; SB = 1; for (int sw = 6; sw >= 2 && SW == 0; --sw) if (fits(sw, SB, NA)) SW = sw; }
+    if (SW == 0) return ADAFUSE_ERR_UNSUPPORTED;
+    a.SW = SW; a.SB = SB; a.NA = NA;
+    a.off_B = (uint32_t)SW * kWTileBytes;
+    a.off_A = a.off_B + (uint32_t)SB * BBytes;
+    a.off_bar = a.off_A + (uint32_t)NA * ABytes;
+    const uint32_t smem = a.off_bar + 1024u + 1024u;
+
+    cudaError_t e = cudaFuncSetAttribute(merge_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return ADAFUSE_ERR_CUDA;
+    const int grid = (int)std::min<int64_t>(p->num_sms, p->merge_tiles);
+    merge_fused_kernel<<<grid, kMergeThreads, smem, s>>>(a);
+    p->last_launches = 1;
+    return cuda_err(cudaGetLastError());
+}
+
+int launch_merge_per_linear(Plan* p, const int32_t* idx, const float* gate, int32_t k, cudaStream_t s)
+{
+    int launches = 0;
+    for (int l = 0; l < p->n_lin; ++l) {
+        const LinDesc& L = p->h_desc[l];
+        dim3 grid((unsigned)((L.d_in + 8 * 128 - 1) / (8 * 128)), (unsigned)L.d_out);
+        merge_per_linear_kernel<<<grid, 128, 0, s>>>(L, idx, gate, k, p->E, p->r, p->d_status);
+        ++launches;
+    }
+    p->last_launches = launches;
+    return cuda_err(cudaGetLastError());
+}
+
+}  // namespace af

@@ -1,0 +1,143 @@
+// Token-level pre-gating router.
+//
+// AdaFuse, page pt section 2.A ("Arquitetura de Pre-Gating por Token") and
+// page ja section 2.1: a single lightweight top-2 router at the first expanded
+// layer decides, once per input token, which LoRA experts are active in every
+// later layer ("decide once, apply everywhere").  With ADAFUSE_POOL_MEAN the
+// decision is taken once for the mean of the rows (the "whole sentence" case of
+// the lay summary, section "A Solucao", item 1).
+//
+// One CTA per decision.  Warp 0 lane e owns expert e: its logit is the fp32 sum
+// of the products x_j * W_r[e, j] in ascending j (products rounded before the
+// add), so the decision is a fixed function of the inputs.  Warps 1-3 stage
+// the next 128-column chunk of x and W_r in shared memory while warp 0
+// consumes the current one.  Softmax and top-k are warp shuffles over the
+// lanes (ties to the lower index, NaN ranked last).
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace af {
+
+namespace {
+
+constexpr int kChunk = 128;      // keeps the double-buffered stage under 48 KB
+constexpr int kRouterThreads = 128;
+
+__device__ __forceinline__ float bf16_at(const uint16_t* p) { return __uint_as_float((uint32_t)(*p) << 16); }
+
+// Is (c1, z1, e1) ranked before (c0, z0, e0)?  Class 0 = finite or infinite
+// logit, 1 = NaN, 2 = no expert / already taken.
+__device__ __forceinline__ bool ranks_before(int c1, float z1, int e1, int c0, float z0, int e0)
+{
+    if (c1 != c0) return c1 < c0;
+    if (c1 == 0 && z1 != z0) return z1 > z0;
+    return e1 < e0;
+}
+
+__global__ void __launch_bounds__(kRouterThreads) pregate_kernel(const uint16_t* x, int64_t T, int32_t H,
+                                                                  int64_t ldx, const float* Wr, const float* br,
+                                                                  int32_t E, int32_t k, uint32_t flags,
+                                                                  int32_t* idx, float* gate)
+{
+    __shared__ float xs[2][kChunk];
+    __shared__ float ws[2][kMaxE][kChunk + 1];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const bool pool = (flags & ADAFUSE_POOL_MEAN) != 0;
+    const int64_t t = pool ? 0 : blockIdx.x;
+    const int nchunks = (H + kChunk - 1) / kChunk;
+
+    // Stage chunk c into buffer b: x row (or the column means) and W_r columns.
+    auto stage = [&](int c, int b, int t0, int nt) {
+        const int j0 = c * kChunk;
+        for (int jj = t0; jj < kChunk; jj += nt) {
+            const int j = j0 + jj;
+            float v = 0.f;
+            if (j < H) {
+                if (pool) {
+                    float acc = 0.f;
+                    for (int64_t tt = 0; tt < T; ++tt) acc = __fadd_rn(acc, bf16_at(x + tt * ldx + j));
+                    v = __fdiv_rn(acc, (float)T);
+                } else {
+                    v = bf16_at(x + t * ldx + j);
+                }
+            }
+            xs[b][jj] = v;
+        }
+        for (int id = t0; id < E * kChunk; id += nt) {
+            const int e = id / kChunk, jj = id - e * kChunk;
+            const int j = j0 + jj;
+            ws[b][e][jj] = (j < H) ? Wr[(int64_t)e * H + j] : 0.f;
+        }
+    };
+
+    stage(0, 0, tid, kRouterThreads);
+    __syncthreads();
+    float z = 0.f;
+    for (int c = 0; c < nchunks; ++c) {
+        const int b = c & 1;
+        if (warp == 0) {
+            if (lane < E) {
+                const int n = min(kChunk, H - c * kChunk);
+                for (int jj = 0; jj < n; ++jj) z = __fadd_rn(z, __fmul_rn(xs[b][jj], ws[b][lane][jj]));
+            }
+        } else if (c + 1 < nchunks) {
+            stage(c + 1, b ^ 1, tid - 32, kRouterThreads - 32);
+        }
+        __syncthreads();
+    }
+    if (warp != 0) return;
+
+    if (lane < E && br != nullptr) z = __fadd_rn(z, br[lane]);
+    const int cls = (lane >= E) ? 2 : (isnan(z) ? 1 : 0);
+
+    // softmax over the experts with a non-NaN logit
+    float m = (cls == 0) ? z : -INFINITY;
+    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    const float ex = (cls == 0) ? expf(z - m) : 0.f;
+    float sum = ex;
+    for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+    const float p = ex / sum;
+
+    // top-k by repeated warp argmax
+    bool taken = false;
+    int sel = 0;
+    float gsel = 0.f, gsum = 0.f;
+    for (int s = 0; s < k; ++s) {
+        int bc = taken ? 2 : cls, be = lane;
+        float bz = z;
+        for (int off = 16; off > 0; off >>= 1) {
+            const int oc = __shfl_xor_sync(0xffffffffu, bc, off);
+            const float oz = __shfl_xor_sync(0xffffffffu, bz, off);
+            const int oe = __shfl_xor_sync(0xffffffffu, be, off);
+            if (ranks_before(oc, oz, oe, bc, bz, be)) { bc = oc; bz = oz; be = oe; }
+        }
+        if (lane == be) taken = true;
+        const float pb = __shfl_sync(0xffffffffu, p, be);
+        if (lane == s) { sel = be; gsel = pb; }
+        gsum = __fadd_rn(gsum, pb);
+    }
+    if (lane < k) {
+        float g = gsel;
+        if (flags & ADAFUSE_RENORM) g = g / gsum;
+        idx[t * k + lane] = sel;
+        gate[t * k + lane] = g;
+    }
+}
+
+}  // namespace
+}  // namespace af
+
+extern "C" int adafuse_pregate(const void* x, int64_t T, int32_t H, int64_t x_row_stride, const float* W_r,
+                               const float* b_r, int32_t E, int32_t k, uint32_t flags, int32_t* idx, float* gate,
+                               adafuse_stream_t stream)
+{
+    if (!x || !W_r || !idx || !gate || T < 1 || H < 1 || x_row_stride < H) return ADAFUSE_ERR_INVALID_ARG;
+    if (E < 1 || E > af::kMaxE || k < 1 || k > E) return ADAFUSE_ERR_UNSUPPORTED;
+    if (flags & ~(ADAFUSE_RENORM | ADAFUSE_POOL_MEAN)) return ADAFUSE_ERR_INVALID_ARG;
+    const bool pool = (flags & ADAFUSE_POOL_MEAN) != 0;
+    if (!pool && T > 0x7fffffff) return ADAFUSE_ERR_UNSUPPORTED;
+    const unsigned grid = pool ? 1u : (unsigned)T;
+    af::pregate_kernel<<<grid, af::kRouterThreads, 0, (cudaStream_t)stream>>>(
+        static_cast<const uint16_t*>(x), T, H, x_row_stride, W_r, b_r, E, k, flags, idx, gate);
+    return af::cuda_err(cudaGetLastError());
+}

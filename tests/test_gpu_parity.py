@@ -1,0 +1,418 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle on
+the same seeded inputs.
+
+Acceptance: expert indices bit-exact; gates |d| <= 1e-6 + 1e-5 |g|; bf16
+outputs |d| <= 1e-2 |ref| + 1e-3 elementwise, and for the merge also the
+delta check in Frobenius norm (helpers.assert_delta_frobenius).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from helpers import ATOL, RTOL, Model, assert_close_bf16, assert_delta_frobenius, f64, u16
+
+pytestmark = pytest.mark.gpu
+
+GATE_ATOL, GATE_RTOL = 1e-6, 1e-5
+
+
+@pytest.fixture(scope="module")
+def am(cuda_device):
+    from adapter_merge_b200 import build
+    build.build()
+    import adapter_merge_b200
+    adapter_merge_b200.lib()
+    return adapter_merge_b200
+
+
+def to_dev(t, dev):
+    return t.to(dev)
+
+
+def check_gates(g_gpu, g_ref):
+    g_gpu = np.asarray(g_gpu, dtype=np.float64)
+    assert np.all(np.abs(g_gpu - g_ref) <= GATE_ATOL + GATE_RTOL * np.abs(g_ref))
+
+
+# ------------------------------------------------------------------ router
+
+@pytest.mark.parametrize("H,E,T,k,bias,renorm", [
+    (256, 4, 8, 2, False, False),       # tiny
+    (4096, 8, 64, 2, False, False),     # 7B decode: first token of 64 sequences
+    (4096, 8, 1, 2, False, True),       # 7B request start, renormalised gates
+    (5120, 16, 32, 2, True, False),     # 13B with a router bias
+    (300, 32, 17, 4, False, False),     # E = 32 lanes, ragged H
+    (100, 5, 3, 5, True, True),         # k = E
+    (8, 1, 2, 1, False, False),         # single expert
+])
+def test_pregate_matches_oracle(am, cuda_device, H, E, T, k, bias, renorm):
+    x = synth.normal((T, H), 1.0, torch.bfloat16, 1, f"px{H}{E}{T}")
+    W_r = synth.normal((E, H), H ** -0.5, torch.float32, 1, f"pw{H}{E}")
+    b_r = synth.normal((E,), 0.5, torch.float32, 1, f"pb{E}") if bias else None
+    idx_ref, gate_ref, z = oracle.pregate(u16(x), W_r.numpy(), k, None if b_r is None else b_r.numpy(), renorm)
+    idx, gate = am.pregate(x.to(cuda_device), W_r.to(cuda_device), k,
+                           None if b_r is None else b_r.to(cuda_device), renorm=renorm)
+    torch.cuda.synchronize()
+    assert np.array_equal(idx.cpu().numpy(), idx_ref)
+    check_gates(gate.cpu().numpy(), gate_ref)
+
+
+def test_pregate_ties_nan_and_strided_rows(am, cuda_device):
+    H, E, T, k = 64, 6, 5, 3
+    W_r = synth.normal((E, H), 0.125, torch.float32, 2, "tw")
+    W_r[3] = W_r[1]                  # experts 1 and 3 always tie: 1 must win
+    W_r[4, 7] = float("nan")         # expert 4's logit is NaN: ranked last, gate 0
+    big = synth.normal((T, 2 * H + 8), 1.0, torch.bfloat16, 2, "tx")
+    x = big[:, 8:8 + H]              # row stride 2H+8
+    idx_ref, gate_ref, _ = oracle.pregate(u16(x.contiguous()), W_r.numpy(), k)
+    dev = big.to(cuda_device)
+    idx, gate = am.pregate(dev[:, 8:8 + H], W_r.to(cuda_device), k)
+    torch.cuda.synchronize()
+    assert np.array_equal(idx.cpu().numpy(), idx_ref)
+    check_gates(gate.cpu().numpy(), gate_ref)
+    idx5, gate5 = am.pregate(dev[:, 8:8 + H], W_r.to(cuda_device), E)
+    i5 = idx5.cpu().numpy()
+    assert np.all(i5[:, -1] == 4)
+    assert np.all(gate5.cpu().numpy()[:, -1] == 0)
+
+
+@pytest.mark.parametrize("T", [1, 7, 64])
+def test_pregate_pooled_sequence_decision(am, cuda_device, T):
+    H, E, k = 4096, 8, 2
+    x = synth.normal((T, H), 1.0, torch.bfloat16, 3, f"pool{T}")
+    W_r = synth.normal((E, H), H ** -0.5, torch.float32, 3, "poolw")
+    idx_ref, gate_ref, _ = oracle.pregate(u16(x), W_r.numpy(), k, pool=True)
+    idx, gate = am.pregate(x.to(cuda_device), W_r.to(cuda_device), k, pool=True)
+    torch.cuda.synchronize()
+    assert idx.shape == (1, k)
+    assert np.array_equal(idx.cpu().numpy(), idx_ref)
+    check_gates(gate.cpu().numpy(), gate_ref)
+
+
+# ---------------------------------------------------------------- segments
+
+@pytest.mark.parametrize("T,k,E", [(1, 1, 1), (8, 2, 4), (64, 2, 8), (300, 4, 6), (2000, 2, 32)])
+def test_segments_match_oracle(am, cuda_device, T, k, E):
+    g = torch.Generator().manual_seed(T * 131 + E)
+    idx = torch.randint(0, E, (T, k), generator=g, dtype=torch.int32)
+    if T > 4:
+        idx[2, 0] = E + 5
+        idx[3, k - 1] = -1
+    off_ref, perm_ref, bad = oracle.segments(idx.numpy(), E)
+    status = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    off, perm, used = am.segments(idx.to(cuda_device), E, status=status)
+    torch.cuda.synchronize()
+    assert np.array_equal(off.cpu().numpy(), off_ref)
+    assert np.array_equal(perm.cpu().numpy()[: len(perm_ref)], perm_ref)
+    counts = np.diff(off_ref)
+    u = used.cpu().numpy()
+    assert u[0] == int((counts > 0).sum())
+    assert np.array_equal(u[1:1 + u[0]], np.nonzero(counts)[0])
+    assert int(status.item()) == (am.STATUS_BAD_INDEX if bad else 0)
+
+
+# ------------------------------------------------------------------- merge
+
+def run_merge(am, model, idx, gate, dev, per_linear=False):
+    i = torch.as_tensor(np.asarray(idx, dtype=np.int32)).to(dev)
+    g = torch.as_tensor(np.asarray(gate, dtype=np.float32)).to(dev)
+    if per_linear:
+        model.plan.merge_per_linear(i, g)
+    else:
+        model.plan.merge(i, g)
+    torch.cuda.synchronize()
+
+
+def check_merge(model, idx, gate, what, rows=None, delta=True):
+    for l, lin in enumerate(model.cfg.linears):
+        rr = (0, lin.d_out) if rows is None else rows(lin)
+        W = u16(model.w.W_views[l])
+        A, B = u16(model.w.A_views[l]), u16(model.w.B_views[l])
+        ref = oracle.merge_linear(W, A, B, idx, gate, rows=rr, nthreads=8)
+        got = u16(model.W_out[l][rr[0]:rr[1]])
+        assert_close_bf16(got, ref, f"{what} linear {l}")
+        if delta:
+            dz = oracle.merge_linear(np.zeros_like(W), A, B, idx, gate, rows=rr, nthreads=8)
+            assert_delta_frobenius(got, W[rr[0]:rr[1]], ref, dz, f"{what} linear {l}")
+
+
+def test_merge_tiny_chain_with_pregate(am, cuda_device):
+    """Tiny config end to end: the router's decision for token 0 drives the
+    merge of all four linears (decide once, apply everywhere)."""
+    cfg = synth.tiny()
+    m = Model(cfg, cuda_device, weights=None)
+    xr = synth.make_router_input(cfg, cfg.T_merge, 0)
+    idx_ref, gate_ref, _ = oracle.pregate(u16(xr), m.w.W_r.cpu().numpy(), cfg.k)
+    idx, gate = am.pregate(xr.to(cuda_device), m.w.W_r, cfg.k)
+    m.plan.merge(idx[0], gate[0])
+    torch.cuda.synchronize()
+    assert np.array_equal(idx.cpu().numpy(), idx_ref)
+    check_merge(m, idx_ref[0], gate_ref[0], "tiny")
+    rc, st = m.plan.status()
+    assert rc == 0 and st == 0
+    assert m.plan.last_launches == 1
+
+
+SHAPES = [(640, 392), (8, 8), (136, 1000), (256, 256), (1000, 72), (128, 136)]
+
+
+@pytest.mark.parametrize("E,r,k", [(5, 16, 2), (4, 8, 1), (8, 64, 4), (6, 32, 3), (32, 8, 2)])
+def test_merge_shapes_and_ranks(am, cuda_device, E, r, k):
+    cfg = synth.custom(SHAPES, E, r, k, 1, name=f"mshape{E}{r}{k}")
+    m = Model(cfg, cuda_device)
+    idx, gate = synth.random_selection(1, E, k, 7, f"msel{E}{r}{k}")
+    run_merge(am, m, idx[0], gate[0], cuda_device)
+    check_merge(m, idx[0].numpy(), gate[0].numpy().astype(np.float64), f"E{E} r{r} k{k}")
+
+
+def test_merge_zero_backbone_isolates_delta(am, cuda_device):
+    cfg = synth.custom([(384, 520), (200, 136)], 4, 16, 2, 1, name="mzero")
+    m = Model(cfg, cuda_device, zero_w=True)
+    idx, gate = np.array([2, 0]), np.array([0.6, 0.3], dtype=np.float32)
+    run_merge(am, m, idx, gate, cuda_device)
+    check_merge(m, idx, gate.astype(np.float64), "zero W", delta=False)
+
+
+def test_merge_poison_unselected_adapters(am, cuda_device):
+    cfg = synth.custom([(384, 264)], 6, 16, 2, 1, name="mpoison")
+    m = Model(cfg, cuda_device)
+    idx, gate = np.array([4, 1]), np.array([0.5, 0.25], dtype=np.float32)
+    run_merge(am, m, idx, gate, cuda_device)
+    clean = m.W_out[0].clone()
+    for e in (0, 2, 3, 5):
+        m.w.A_views[0][e].fill_(float("nan"))
+        m.w.B_views[0][e].fill_(float("nan"))
+    run_merge(am, m, idx, gate, cuda_device)
+    assert torch.equal(m.W_out[0].view(torch.int16), clean.view(torch.int16))
+
+
+def test_merge_in_place_and_deterministic(am, cuda_device):
+    cfg = synth.custom([(512, 384), (136, 264)], 4, 16, 2, 1, name="minpl")
+    m = Model(cfg, cuda_device)
+    idx, gate = np.array([3, 1]), np.array([0.4, 0.35], dtype=np.float32)
+    run_merge(am, m, idx, gate, cuda_device)
+    out1 = [t.clone() for t in m.W_out]
+    run_merge(am, m, idx, gate, cuda_device)
+    for a, b in zip(out1, m.W_out):
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+    mi = Model(cfg, cuda_device, in_place=True, weights=synth.make_weights(cfg, 0, device=cuda_device))
+    run_merge(am, mi, idx, gate, cuda_device)
+    for a, b in zip(out1, mi.W_out):
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+def test_merge_bad_index_skipped_and_flagged(am, cuda_device):
+    cfg = synth.custom([(256, 136)], 4, 8, 2, 1, name="mbad")
+    m = Model(cfg, cuda_device)
+    idx, gate = np.array([1, 9]), np.array([0.5, 0.5], dtype=np.float32)
+    run_merge(am, m, idx, gate, cuda_device)
+    rc, st = m.plan.status()
+    assert rc == 0 and st == am.STATUS_BAD_INDEX
+    check_merge(m, idx, gate.astype(np.float64), "bad index")
+    assert m.plan.status() == (0, 0)
+
+
+def test_merge_per_linear_baseline(am, cuda_device):
+    cfg = synth.custom(SHAPES, 5, 16, 2, 1, name="mpl")
+    m = Model(cfg, cuda_device)
+    idx, gate = np.array([0, 3]), np.array([0.45, 0.2], dtype=np.float32)
+    run_merge(am, m, idx, gate, cuda_device, per_linear=True)
+    assert m.plan.last_launches == len(SHAPES)
+    check_merge(m, idx, gate.astype(np.float64), "per-linear")
+
+
+def test_switch_in_place(am, cuda_device):
+    """Switch old -> new on the merged weights: matches the oracle's switch of
+    the oracle's own merged weights; identical selections leave W_out alone."""
+    cfg = synth.custom([(384, 264), (136, 520)], 5, 16, 2, 1, name="mswitch")
+    m = Model(cfg, cuda_device)
+    old_i, old_g = np.array([1, 4]), np.array([0.55, 0.3], dtype=np.float32)
+    new_i, new_g = np.array([2, 1]), np.array([0.4, 0.25], dtype=np.float32)
+    run_merge(am, m, old_i, old_g, cuda_device)
+    d = lambda a, t: torch.as_tensor(a.astype(t)).to(cuda_device)
+    m.plan.switch(d(new_i, np.int32), d(new_g, np.float32), d(old_i, np.int32), d(old_g, np.float32))
+    torch.cuda.synchronize()
+    for l in range(cfg.n_lin):
+        W, A, B = u16(m.w.W_views[l]), u16(m.w.A_views[l]), u16(m.w.B_views[l])
+        cur = oracle.merge_linear(W, A, B, old_i, old_g.astype(np.float64))
+        ref = oracle.merge_linear(cur, A, B, list(new_i) + list(old_i),
+                                  list(new_g.astype(np.float64)) + list(-old_g.astype(np.float64)))
+        assert_close_bf16(u16(m.W_out[l]), ref, f"switch linear {l}")
+    before = [t.clone() for t in m.W_out]
+    m.plan.switch(d(new_i, np.int32), d(new_g, np.float32), d(new_i, np.int32), d(new_g, np.float32))
+    torch.cuda.synchronize()
+    for a, b in zip(before, m.W_out):
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+# ------------------------------------------------------------------- apply
+
+def apply_setup(cfg, dev, T, seed=0, zero_w=False, sel=None):
+    m = Model(cfg, dev, seed=seed, zero_w=zero_w)
+    X, xs = synth.make_apply_inputs(cfg, T, seed)
+    xs_dev = [x.to(dev) for x in xs]
+    ys = [torch.empty((T, l.d_out), dtype=torch.bfloat16, device=dev) for l in cfg.linears]
+    import adapter_merge_b200 as am
+    xp, yp = am.pointer_table(xs_dev, dev), am.pointer_table(ys, dev)
+    if sel is None:
+        idx, gate = synth.random_selection(T, cfg.E, cfg.k, seed + 11, f"asel{cfg.name}{T}")
+    else:
+        idx, gate = sel
+    ws = torch.empty(m.plan.workspace_bytes(T, cfg.k), dtype=torch.uint8, device=dev)
+    return m, xs, xs_dev, ys, xp, yp, idx, gate, ws
+
+
+def check_apply(m, xs, ys, idx, gate, what, tokens=None, lins=None):
+    cfg = m.cfg
+    for l in (range(cfg.n_lin) if lins is None else lins):
+        W, A, B = u16(m.w.W_views[l]), u16(m.w.A_views[l]), u16(m.w.B_views[l])
+        tt = (0, xs[l].shape[0]) if tokens is None else tokens
+        ref = oracle.apply_linear(u16(xs[l]), W, A, B, np.asarray(idx, np.int32),
+                                  np.asarray(gate, np.float64), tokens=tt, nthreads=8)
+        assert_close_bf16(u16(ys[l][tt[0]:tt[1]]), ref, f"{what} linear {l}")
+
+
+def run_apply(m, xp, yp, T, idx, gate, ws, dev):
+    i = torch.as_tensor(np.asarray(idx, dtype=np.int32)).to(dev)
+    g = torch.as_tensor(np.asarray(gate, dtype=np.float32)).to(dev)
+    m.plan.apply(xp, yp, T, i, g, ws)
+    torch.cuda.synchronize()
+
+
+def test_apply_tiny_chain_with_pregate(am, cuda_device):
+    cfg = synth.tiny()
+    m, xs, xs_dev, ys, xp, yp, _, _, ws = apply_setup(cfg, cuda_device, cfg.T_apply)
+    xr = synth.make_router_input(cfg, cfg.T_apply, 0)
+    idx_ref, gate_ref, _ = oracle.pregate(u16(xr), m.w.W_r.cpu().numpy(), cfg.k)
+    idx, gate = am.pregate(xr.to(cuda_device), m.w.W_r, cfg.k)
+    m.plan.apply(xp, yp, cfg.T_apply, idx, gate, ws)
+    torch.cuda.synchronize()
+    assert np.array_equal(idx.cpu().numpy(), idx_ref)
+    check_apply(m, xs, ys, idx_ref, gate_ref, "tiny apply")
+    assert m.plan.status() == (0, 0)
+    assert m.plan.last_launches == 3
+
+
+@pytest.mark.parametrize("T", [1, 5, 16, 17, 64, 130, 256, 300])
+def test_apply_token_counts(am, cuda_device, T):
+    cfg = synth.custom([(384, 520), (136, 72)], 6, 16, 2, T, name=f"aT{T}")
+    m, xs, xs_dev, ys, xp, yp, idx, gate, ws = apply_setup(cfg, cuda_device, T)
+    run_apply(m, xp, yp, T, idx, gate, ws, cuda_device)
+    check_apply(m, xs, ys, idx.numpy(), gate.numpy().astype(np.float64), f"T={T}")
+
+
+@pytest.mark.parametrize("E,r,k,T", [(4, 8, 1, 16), (8, 16, 2, 64), (32, 64, 4, 128), (16, 32, 2, 32), (3, 24, 3, 9)])
+def test_apply_ranks(am, cuda_device, E, r, k, T):
+    cfg = synth.custom([(256, 392), (520, 136)], E, r, k, T, name=f"aR{E}{r}{k}{T}")
+    m, xs, xs_dev, ys, xp, yp, idx, gate, ws = apply_setup(cfg, cuda_device, T)
+    run_apply(m, xp, yp, T, idx, gate, ws, cuda_device)
+    check_apply(m, xs, ys, idx.numpy(), gate.numpy().astype(np.float64), f"E{E} r{r} k{k} T{T}")
+
+
+def test_apply_zero_gates_poison_bad_and_duplicate(am, cuda_device):
+    T = 24
+    cfg = synth.custom([(264, 392)], 6, 16, 2, T, name="aedge")
+    m, xs, xs_dev, ys, xp, yp, idx, gate, ws = apply_setup(cfg, cuda_device, T)
+    idx = idx.clone()
+    gate = gate.clone()
+    # a few rows use only experts {0, 1, 2}; then poison experts 3..5 below
+    # for a run where every row uses {0, 1, 2}
+    run_apply(m, xp, yp, T, idx, torch.zeros_like(gate), ws, cuda_device)
+    check_apply(m, xs, ys, idx.numpy(), np.zeros((T, 2)), "zero gates")
+    sel = torch.tensor([[0, 1], [2, 0], [1, 2]] * (T // 3), dtype=torch.int32)
+    run_apply(m, xp, yp, T, sel, gate, ws, cuda_device)
+    clean = ys[0].clone()
+    for e in (3, 4, 5):
+        m.w.A_views[0][e].fill_(float("nan"))
+        m.w.B_views[0][e].fill_(float("nan"))
+    run_apply(m, xp, yp, T, sel, gate, ws, cuda_device)
+    assert torch.equal(ys[0].view(torch.int16), clean.view(torch.int16))
+    # invalid index: slot skipped, flagged; duplicate experts in a row: gates add
+    bad = sel.clone()
+    bad[4, 1] = 17
+    bad[5, 1] = bad[5, 0]
+    run_apply(m, xp, yp, T, bad, gate, ws, cuda_device)
+    rc, st = m.plan.status()
+    assert rc == 0 and st == am.STATUS_BAD_INDEX
+    check_apply(m, xs, ys, bad.numpy(), gate.numpy().astype(np.float64), "bad/dup")
+
+
+def test_apply_equals_merged_weights(am, cuda_device):
+    """Merged form equals unmerged: with one shared selection, apply(x) agrees
+    with x W'^T for the GPU's own merged W' to within the bf16 rounding of W'."""
+    T = 32
+    cfg = synth.custom([(384, 520), (256, 136)], 5, 16, 2, T, name="aeq")
+    sel_i = torch.tensor([[3, 1]] * T, dtype=torch.int32)
+    sel_g = torch.tensor([[0.5, 0.3]] * T, dtype=torch.float32)
+    m, xs, xs_dev, ys, xp, yp, _, _, ws = apply_setup(cfg, cuda_device, T, sel=(sel_i, sel_g))
+    run_apply(m, xp, yp, T, sel_i, sel_g, ws, cuda_device)
+    run_merge(am, m, sel_i[0].numpy(), sel_g[0].numpy(), cuda_device)
+    for l in range(cfg.n_lin):
+        x = f64(xs[l]); Wm = f64(m.W_out[l]); y = f64(ys[l])
+        ym = x @ Wm.T
+        bound = 2.0 ** -8 * (np.abs(x) @ np.abs(Wm).T) + 2.0 ** -7 * np.abs(ym) + 1e-6
+        assert np.all(np.abs(y - ym) <= bound)
+
+
+# ------------------------------------------------------------- full sizes
+
+def sampled_rows(lin, n=3):
+    return [(0, 1), (lin.d_out // 2, lin.d_out // 2 + 1), (lin.d_out - 1, lin.d_out)][:n]
+
+
+@pytest.mark.parametrize("cfg_fn", [synth.llama7b, synth.llama13b])
+def test_full_size_merge_sampled(am, cuda_device, cfg_fn):
+    """Full model, in the benchmark's launch configuration: pregate on one
+    token, one merge launch over every linear; sampled rows of a spread of
+    linears against the oracle (rows are independent, so a row is exact)."""
+    cfg = cfg_fn()
+    m = Model(cfg, cuda_device)
+    xr = synth.make_router_input(cfg, 1, 0, device=cuda_device)
+    idx, gate = am.pregate(xr, m.w.W_r, cfg.k)
+    m.plan.merge(idx[0], gate[0])
+    torch.cuda.synchronize()
+    idx_ref, gate_ref, _ = oracle.pregate(u16(xr), m.w.W_r.cpu().numpy(), cfg.k)
+    assert np.array_equal(idx.cpu().numpy(), idx_ref)
+    g = gate.cpu().numpy()[0].astype(np.float64)
+    picks = sorted(set([0, 1, 4, 6, cfg.n_lin // 2, cfg.n_lin // 2 + 5, cfg.n_lin - 1]))
+    for l in picks:
+        lin = cfg.linears[l]
+        W, A, B = u16(m.w.W_views[l]), u16(m.w.A_views[l]), u16(m.w.B_views[l])
+        for rr in sampled_rows(lin):
+            ref = oracle.merge_linear(W, A, B, idx_ref[0], g, rows=rr)
+            got = u16(m.W_out[l][rr[0]:rr[1]])
+            assert_close_bf16(got, ref, f"{cfg.name} linear {l} rows {rr}")
+            dz = oracle.merge_linear(np.zeros_like(W), A, B, idx_ref[0], g, rows=rr)
+            assert_delta_frobenius(got, W[rr[0]:rr[1]], ref, dz, f"{cfg.name} linear {l} rows {rr}")
+    assert m.plan.status() == (0, 0)
+
+
+@pytest.mark.parametrize("cfg_fn", [synth.llama7b, synth.llama13b])
+def test_full_size_apply_sampled(am, cuda_device, cfg_fn):
+    """Batched decode at full size: per-sequence routing on each sequence's
+    first token, one apply over every linear; sampled (linear, token) rows
+    against the oracle."""
+    cfg = cfg_fn()
+    T = cfg.T_apply
+    m = Model(cfg, cuda_device)
+    X, xs_dev = synth.make_apply_inputs(cfg, T, 0, device=cuda_device)
+    ys = [torch.empty((T, l.d_out), dtype=torch.bfloat16, device=cuda_device) for l in cfg.linears]
+    xp, yp = am.pointer_table(xs_dev, cuda_device), am.pointer_table(ys, cuda_device)
+    xr = synth.make_router_input(cfg, T, 0, device=cuda_device, tag="xfirst")
+    idx, gate = am.pregate(xr, m.w.W_r, cfg.k)
+    ws = torch.empty(m.plan.workspace_bytes(T, cfg.k), dtype=torch.uint8, device=cuda_device)
+    m.plan.apply(xp, yp, T, idx, gate, ws)
+    torch.cuda.synchronize()
+    idx_ref, gate_ref, _ = oracle.pregate(u16(xr), m.w.W_r.cpu().numpy(), cfg.k)
+    assert np.array_equal(idx.cpu().numpy(), idx_ref)
+    g = gate.cpu().numpy().astype(np.float64)
+    picks = sorted(set([0, 3, 4, 6, cfg.n_lin // 2, cfg.n_lin - 1]))
+    for l in picks:
+        W, A, B = u16(m.w.W_views[l]), u16(m.w.A_views[l]), u16(m.w.B_views[l])
+        x = u16(xs_dev[l])
+        for t in (0, T // 2, T - 1):
+            ref = oracle.apply_linear(x, W, A, B, idx_ref, g, tokens=(t, t + 1), nthreads=8)
+            assert_close_bf16(u16(ys[l][t:t + 1]), ref, f"{cfg.name} apply linear {l} token {t}")
+    assert m.plan.status() == (0, 0)
