@@ -153,8 +153,14 @@ class Plan:
         arr = (Linear * len(linears))()
         for i, (W, W_out, A, B) in enumerate(linears):
             d_out, d_in = W.shape
+            for t, inner in ((W, (d_in, 1)), (W_out, (d_in, 1)), (A, (d_in, 1)), (B, (r, 1))):
+                if tuple(t.stride()[-2:]) != inner and t.shape[-2] > 1:
+                    raise ValueError(f"linear {i}: tensors must be row-major inside each expert "
+                                     f"(strides {tuple(t.stride())})")
+            a_es = A.stride(0) if A.shape[0] > 1 else r * d_in
+            b_es = B.stride(0) if B.shape[0] > 1 else d_out * r
             arr[i] = Linear(W.data_ptr(), W_out.data_ptr(), A.data_ptr(), B.data_ptr(),
-                            d_out, d_in, A.stride(0), B.stride(0))
+                            d_out, d_in, a_es, b_es)
         self._keep = list(linears)
         self.E, self.r, self.n_lin = E, r, len(linears)
         h = ctypes.c_void_p()

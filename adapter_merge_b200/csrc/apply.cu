@@ -252,8 +252,7 @@ __global__ void __launch_bounds__(kApplyThreads, 1) apply_fused_kernel(const __g
                 UnitIt it;
                 it.init(a.lins, a.n_lin, u_begin);
                 for (int ui = 0; ui < nunits && !stop; ++ui) {
-                    const LinDesc& L = a.lins[it.l];
-                    const int nKb = (L.d_in + kChunkK - 1) / kChunkK;
+                    const int nKb = (__ldg(&a.lins[it.l].d_in) + kChunkK - 1) / kChunkK;
                     const int m0 = it.mt * kTileM;
                     const CUtensorMap* mW = a.maps + (size_t)it.l * kMapsPerLinear + kMapW;
                     const CUtensorMap* mB = a.maps + (size_t)it.l * kMapsPerLinear + kMapB;
@@ -297,8 +296,7 @@ __global__ void __launch_bounds__(kApplyThreads, 1) apply_fused_kernel(const __g
                 UnitIt it;
                 it.init(a.lins, a.n_lin, u_begin);
                 for (int ui = 0; ui < nunits && !stop; ++ui, ++uc) {
-                    const LinDesc& L = a.lins[it.l];
-                    const int nKb = (L.d_in + kChunkK - 1) / kChunkK;
+                    const int nKb = (__ldg(&a.lins[it.l].d_in) + kChunkK - 1) / kChunkK;
                     const int acc = (int)(uc & 1);
                     if (!mbar_wait(&accempty[acc], (uint32_t)((uc >> 1) & 1) ^ 1u, abort_flag)) { stop = true; break; }
                     tc_fence_after();
@@ -339,10 +337,14 @@ __global__ void __launch_bounds__(kApplyThreads, 1) apply_fused_kernel(const __g
                 UnitIt it;
                 it.init(a.lins, a.n_lin, u_begin);
                 for (int ui = 0; ui < nunits && !stop; ++ui) {
-                    const LinDesc& L = a.lins[it.l];
-                    const int nKb = (L.d_in + kChunkK - 1) / kChunkK;
+                    // Per-unit values live in registers: the cp.async below
+                    // clobber memory, which would force reloads from global.
+                    const int d_in = __ldg(&a.lins[it.l].d_in);
+                    const int nKb = (d_in + kChunkK - 1) / kChunkK;
                     const uint16_t* x = a.x_ptrs[it.l];
                     const uint16_t* Sl = a.S + (int64_t)it.l * a.T * a.Kext;
+                    const int64_t T = a.T;
+                    const int Kext = a.Kext;
                     for (int kc = 0; kc < nKb + nKe; ++kc, ++gc) {
                         const int s = (int)(gc % a.ST);
                         bool ok = mbar_wait(&empty[s], (uint32_t)((gc / a.ST) & 1) ^ 1u, abort_flag);
@@ -357,10 +359,10 @@ __global__ void __launch_bounds__(kApplyThreads, 1) apply_fused_kernel(const __g
                             uint32_t nbytes = 0;
                             if (kc < nKb) {
                                 const int col = kc * kChunkK + c * 8;
-                                if (tabs < a.T && col < L.d_in) { src = x + tabs * L.d_in + col; nbytes = 16; }
+                                if (tabs < T && col < d_in) { src = x + tabs * d_in + col; nbytes = 16; }
                             } else {
                                 const int col = (kc - nKb) * kChunkK + c * 8;
-                                if (tabs < a.T) { src = Sl + tabs * a.Kext + col; nbytes = 16; }
+                                if (tabs < T) { src = Sl + tabs * Kext + col; nbytes = 16; }
                             }
                             cp_async_16(dst, src, nbytes);
                         }
@@ -385,8 +387,9 @@ __global__ void __launch_bounds__(kApplyThreads, 1) apply_fused_kernel(const __g
                     bool ok = mbar_wait(&accfull[acc], (uint32_t)((uc >> 1) & 1), abort_flag);
                     if (!__all_sync(0xffffffffu, ok)) { stop = true; break; }
                     tc_fence_after();
-                    const LinDesc& L = a.lins[it.l];
+                    const int d_out = __ldg(&a.lins[it.l].d_out);
                     uint16_t* y = a.y_ptrs[it.l];
+                    const int64_t T = a.T;
                     const int row = it.mt * kTileM + q * 32 + lane;
                     const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)acc * a.acc_stride;
                     for (int c0 = 0; c0 < a.Npad; c0 += 32) {
@@ -400,12 +403,13 @@ __global__ void __launch_bounds__(kApplyThreads, 1) apply_fused_kernel(const __g
                             for (int i = 0; i < 16; ++i) { v[i] = h[i]; v[16 + i] = 0; }
                         }
                         tc_wait_ld();
-                        if (row < L.d_out) {
-                            const int ncol = min(32, a.Npad - c0);
-                            for (int i = 0; i < ncol; ++i) {
-                                const int64_t t = (int64_t)tt * kApplyMaxN + c0 + i;
-                                if (t < a.T)
-                                    y[t * L.d_out + row] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[i])));
+                        if (row < d_out) {
+                            const int64_t t0 = (int64_t)tt * kApplyMaxN + c0;
+                            uint16_t* yp = y + t0 * d_out + row;
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) {
+                                if (c0 + i < a.Npad && t0 + i < T)
+                                    yp[(int64_t)i * d_out] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[i])));
                             }
                         }
                     }

@@ -26,9 +26,10 @@ struct LinDesc {
     int32_t n_strips;      // ceil(d_in / 128)
 };
 
-// Tensor maps kept per linear: W (load), W_out (load/store), B (3-D stack).
-constexpr int kMapsPerLinear = 3;
-constexpr int kMapW = 0, kMapWout = 1, kMapB = 2;
+// Tensor maps kept per linear: W (load, 64x128 boxes), W_out (load, 64x128
+// boxes), B (3-D stack), W_out store (64x32 boxes: one per epilogue warp).
+constexpr int kMapsPerLinear = 4;
+constexpr int kMapW = 0, kMapWout = 1, kMapB = 2, kMapWoutStore = 3;
 
 constexpr int kTileM = 128;      // output rows per tile (MMA M, TMEM lanes)
 constexpr int kTileN = 128;      // merge: d_in columns per tile (MMA N)

@@ -17,10 +17,10 @@
 //   warps 2-3   build Acat for a 128-column strip once per strip: gate-scaled
 //               A rows (fp32 multiply, bf16 round) in the MN-major core-matrix
 //               layout; double-buffered, reused by every row tile of the strip.
-//   warps 4-11  epilogue: dW from TMEM (tcgen05.ld), W from the swizzled smem
-//               tile, W + dW rounded to bf16 in place, then one thread stores
-//               the tile with TMA.  The stage is released once the store has
-//               read it.
+//   warps 4-11  epilogue: each warp takes a 32-row x 64-column slice: dW from
+//               TMEM (tcgen05.ld), W from the swizzled smem tile, W + dW
+//               rounded to bf16 in place, and a TMA store of the slice.  The
+//               stage is released once all eight stores have read it.
 // HBM traffic is W read + W' write (4 bytes per element) plus the selected
 // adapters; the tensor cores carry the rank-(k*r) contraction (16*k*r/4 FLOP/B).
 #include <algorithm>
@@ -140,7 +140,7 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_fused_kernel(const __g
     const uint32_t ABytes = (uint32_t)a.Kp * 256u;     // Kp rows x 128 cols bf16
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < a.SW; ++i) { mbar_init(&wfull[i], 1); mbar_init(&wempty[i], 1); }
+        for (int i = 0; i < a.SW; ++i) { mbar_init(&wfull[i], 1); mbar_init(&wempty[i], kEpiWarps); }
         for (int i = 0; i < a.SB; ++i) { mbar_init(&bfull[i], 1); mbar_init(&bempty[i], 1); }
         for (int i = 0; i < a.NA; ++i) { mbar_init(&afull[i], 2); mbar_init(&aempty[i], 1); }
         for (int i = 0; i < 2; ++i) { mbar_init(&accfull[i], 1); mbar_init(&accempty[i], kEpiWarps); }
@@ -321,61 +321,62 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_fused_kernel(const __g
         }
     } else {
         // ------------------------------------------------------------ epilogue
+        // Warp (q, h) owns rows 32q..32q+31 and columns 64h..64h+63 of the
+        // tile: it reads that slice of dW from TMEM, adds it to the W slice in
+        // shared memory, and stores the slice itself with one TMA store.  A W
+        // stage is released (8 arrivals) once every warp's store has read it.
         const int ew = warp - 4;            // 0..7
         const int q = warp & 3;             // TMEM lane quarter this warp may access
         const int h = ew >> 2;              // column half (64 columns)
         const int row = q * 32 + lane;
-        const bool leader = (ew == 0 && lane == 0);
-        bool aborted = false;
         TileIt it;
         if (count > 0) it.init(a.lins, a.n_lin, t_begin);
+        int64_t stored = 0;
         for (int64_t i = 0; i < count; ++i) {
             const int acc = (int)(i & 1);
             const int sw = (int)(i % a.SW);
             bool ok = mbar_wait(&accfull[acc], (uint32_t)((i >> 1) & 1), abort_flag);
             ok = ok && mbar_wait(&wfull[sw], (uint32_t)((i / a.SW) & 1), abort_flag);
             ok = __all_sync(0xffffffffu, ok);
-            if (ok) {
-                tc_fence_after();
-                uint32_t va[32], vb[32];
-                const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)acc * kTileN + (uint32_t)h * 64u;
-                tc_ld_x32(taddr, va);
-                tc_ld_x32(taddr + 32u, vb);
-                tc_wait_ld();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&accempty[acc]);
-                const uint32_t wrow = smem_u32(sW + (size_t)sw * kWTileBytes + (size_t)h * kWBoxBytes) + (uint32_t)row * 128u;
+            if (!ok) break;
+            tc_fence_after();
+            uint32_t va[32], vb[32];
+            const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)acc * kTileN + (uint32_t)h * 64u;
+            tc_ld_x32(taddr, va);
+            tc_ld_x32(taddr + 32u, vb);
+            tc_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&accempty[acc]);
+            uint8_t* slice = sW + (size_t)sw * kWTileBytes + (size_t)h * kWBoxBytes + (size_t)q * 32 * 128;
+            const uint32_t wrow = smem_u32(slice) + (uint32_t)lane * 128u;
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    const uint32_t addr = wrow + ((uint32_t)(c ^ (row & 7)) << 4);
-                    const uint4 w = ld_shared_v4(addr);
-                    const uint32_t* d = (c < 4) ? &va[c * 8] : &vb[(c - 4) * 8];
-                    uint4 o;
-                    o.x = add_bf16x2(w.x, d[0], d[1]);
-                    o.y = add_bf16x2(w.y, d[2], d[3]);
-                    o.z = add_bf16x2(w.z, d[4], d[5]);
-                    o.w = add_bf16x2(w.w, d[6], d[7]);
-                    st_shared_v4(addr, o);
-                }
-                fence_proxy_async_smem();
+            for (int c = 0; c < 8; ++c) {
+                const uint32_t addr = wrow + ((uint32_t)(c ^ (row & 7)) << 4);
+                const uint4 w = ld_shared_v4(addr);
+                const uint32_t* d = (c < 4) ? &va[c * 8] : &vb[(c - 4) * 8];
+                uint4 o;
+                o.x = add_bf16x2(w.x, d[0], d[1]);
+                o.y = add_bf16x2(w.y, d[2], d[3]);
+                o.z = add_bf16x2(w.z, d[4], d[5]);
+                o.w = add_bf16x2(w.w, d[6], d[7]);
+                st_shared_v4(addr, o);
             }
-            if (named_bar_red_or(1, kEpiWarps * 32, !ok || *abort_flag != 0)) { aborted = true; break; }
-            if (leader) {
-                const CUtensorMap* mO = a.maps + (size_t)it.l * kMapsPerLinear + kMapWout;
-                const int n0 = it.strip * kTileN, m0 = it.rt * kTileM;
-                uint8_t* src = sW + (size_t)sw * kWTileBytes;
-                tma_store_2d(mO, src, n0, m0);
-                tma_store_2d(mO, src + kWBoxBytes, n0 + 64, m0);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                const CUtensorMap* mO = a.maps + (size_t)it.l * kMapsPerLinear + kMapWoutStore;
+                tma_store_2d(mO, slice, it.strip * kTileN + h * 64, it.rt * kTileM + q * 32);
                 bulk_commit_group();
                 bulk_wait_group_read<1>();
                 if (i > 0) mbar_arrive(&wempty[(i - 1) % a.SW]);
             }
+            stored = i + 1;
             if (i + 1 < count) it.next(a.lins, a.n_lin);
         }
-        if (leader) {
+        if (lane == 0) {
             bulk_wait_group<0>();
-            if (count > 0 && !aborted) mbar_arrive(&wempty[(count - 1) % a.SW]);
+            if (stored > 0) mbar_arrive(&wempty[(stored - 1) % a.SW]);
         }
     }
 

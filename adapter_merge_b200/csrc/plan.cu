@@ -28,12 +28,13 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// W-shaped map: 2-D [rows, cols] bf16 row-major, box 64 cols x 128 rows, 128-byte swizzle.
-bool encode_w(CUtensorMap* m, const void* ptr, int rows, int cols)
+// W-shaped map: 2-D [rows, cols] bf16 row-major, box 64 cols x box_rows rows,
+// 128-byte swizzle.
+bool encode_w(CUtensorMap* m, const void* ptr, int rows, int cols, int box_rows = 128)
 {
     cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
     cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
-    cuuint32_t box[2] = {64, 128};
+    cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
     cuuint32_t estr[2] = {1, 1};
     return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -125,6 +126,7 @@ extern "C" int adafuse_plan_create(adafuse_plan** out, const adafuse_linear* lin
         for (int m = 0; m < d.n_rt; ++m) unit_cost.push_back((L.d_in + kChunkK - 1) / kChunkK + 2);
         if (!encode_w(&maps[(size_t)l * kMapsPerLinear + kMapW], L.W, L.d_out, L.d_in) ||
             !encode_w(&maps[(size_t)l * kMapsPerLinear + kMapWout], L.W_out, L.d_out, L.d_in) ||
+            !encode_w(&maps[(size_t)l * kMapsPerLinear + kMapWoutStore], L.W_out, L.d_out, L.d_in, 32) ||
             !encode_b(&maps[(size_t)l * kMapsPerLinear + kMapB], L.B, E, L.d_out, r, L.b_expert_stride)) {
             free_plan(p);
             return ADAFUSE_ERR_UNSUPPORTED;

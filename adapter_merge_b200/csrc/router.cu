@@ -9,9 +9,9 @@
 //
 // One CTA per decision.  Warp 0 lane e owns expert e: its logit is the fp32 sum
 // of the products x_j * W_r[e, j] in ascending j (products rounded before the
-// add), so the decision is a fixed function of the inputs.  Warps 1-3 stage
-// the next 128-column chunk of x and W_r in shared memory while warp 0
-// consumes the current one.  Softmax and top-k are warp shuffles over the
+// add), so the decision is a fixed function of the inputs.  W_r streams
+// through a 4-stage cp.async ring (three 256-column chunks ahead) and warps
+// 1-3 stage the next chunk of x while warp 0 consumes the current one.  Softmax and top-k are warp shuffles over the
 // lanes (ties to the lower index, NaN ranked last).
 #include "internal.h"
 #include "ptx.cuh"
@@ -20,10 +20,16 @@ namespace af {
 
 namespace {
 
-constexpr int kChunk = 128;      // keeps the double-buffered stage under 48 KB
+constexpr int kChunk = 256;          // columns of x and W_r per pipeline stage
+constexpr int kStages = 4;           // W_r chunks in flight: kStages - 1 ahead
 constexpr int kRouterThreads = 128;
 
 __device__ __forceinline__ float bf16_at(const uint16_t* p) { return __uint_as_float((uint32_t)(*p) << 16); }
+
+__device__ __forceinline__ void cp_async_4(uint32_t dst, const void* src)
+{
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
 
 // Is (c1, z1, e1) ranked before (c0, z0, e0)?  Class 0 = finite or infinite
 // logit, 1 = NaN, 2 = no expert / already taken.
@@ -34,20 +40,36 @@ __device__ __forceinline__ bool ranks_before(int c1, float z1, int e1, int c0, f
     return e1 < e0;
 }
 
+__host__ __device__ constexpr int stage_floats(int E) { return E * (kChunk + 1) + kChunk; }
+
 __global__ void __launch_bounds__(kRouterThreads) pregate_kernel(const uint16_t* x, int64_t T, int32_t H,
                                                                   int64_t ldx, const float* Wr, const float* br,
                                                                   int32_t E, int32_t k, uint32_t flags,
                                                                   int32_t* idx, float* gate)
 {
-    __shared__ float xs[2][kChunk];
-    __shared__ float ws[2][kMaxE][kChunk + 1];
+    extern __shared__ float rsm[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const bool pool = (flags & ADAFUSE_POOL_MEAN) != 0;
     const int64_t t = pool ? 0 : blockIdx.x;
     const int nchunks = (H + kChunk - 1) / kChunk;
+    const int SF = stage_floats(E);
 
-    // Stage chunk c into buffer b: x row (or the column means) and W_r columns.
-    auto stage = [&](int c, int b, int t0, int nt) {
+    // W_r columns of chunk c -> stage buffer (ws[e][jj], rows padded to kChunk+1).
+    auto issue_w = [&](int c) {
+        if (c < nchunks) {
+            float* ws = rsm + (c % kStages) * SF;
+            const int j0 = c * kChunk;
+            const int n = min(kChunk, H - j0);
+            for (int id = tid; id < E * kChunk; id += kRouterThreads) {
+                const int e = id / kChunk, jj = id - e * kChunk;
+                if (jj < n) cp_async_4(smem_u32(ws + e * (kChunk + 1) + jj), Wr + (int64_t)e * H + j0 + jj);
+            }
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    // x (or the column means of x) for chunk c -> stage buffer, threads t0.. step nt.
+    auto load_x = [&](int c, int t0, int nt) {
+        float* xs = rsm + (c % kStages) * SF + E * (kChunk + 1);
         const int j0 = c * kChunk;
         for (int jj = t0; jj < kChunk; jj += nt) {
             const int j = j0 + jj;
@@ -61,29 +83,28 @@ __global__ void __launch_bounds__(kRouterThreads) pregate_kernel(const uint16_t*
                     v = bf16_at(x + t * ldx + j);
                 }
             }
-            xs[b][jj] = v;
-        }
-        for (int id = t0; id < E * kChunk; id += nt) {
-            const int e = id / kChunk, jj = id - e * kChunk;
-            const int j = j0 + jj;
-            ws[b][e][jj] = (j < H) ? Wr[(int64_t)e * H + j] : 0.f;
+            xs[jj] = v;
         }
     };
 
-    stage(0, 0, tid, kRouterThreads);
-    __syncthreads();
+    for (int c = 0; c < kStages - 1; ++c) issue_w(c);
+    load_x(0, tid, kRouterThreads);
     float z = 0.f;
     for (int c = 0; c < nchunks; ++c) {
-        const int b = c & 1;
+        issue_w(c + kStages - 1);
+        asm volatile("cp.async.wait_group %0;" ::"n"(kStages - 1) : "memory");
+        __syncthreads();                       // chunk c is in shared memory
         if (warp == 0) {
             if (lane < E) {
+                const float* ws = rsm + (c % kStages) * SF + lane * (kChunk + 1);
+                const float* xs = rsm + (c % kStages) * SF + E * (kChunk + 1);
                 const int n = min(kChunk, H - c * kChunk);
-                for (int jj = 0; jj < n; ++jj) z = __fadd_rn(z, __fmul_rn(xs[b][jj], ws[b][lane][jj]));
+                for (int jj = 0; jj < n; ++jj) z = __fadd_rn(z, __fmul_rn(xs[jj], ws[jj]));
             }
         } else if (c + 1 < nchunks) {
-            stage(c + 1, b ^ 1, tid - 32, kRouterThreads - 32);
+            load_x(c + 1, tid - 32, kRouterThreads - 32);
         }
-        __syncthreads();
+        __syncthreads();                       // stage c % kStages may be refilled
     }
     if (warp != 0) return;
 
@@ -137,7 +158,11 @@ extern "C" int adafuse_pregate(const void* x, int64_t T, int32_t H, int64_t x_ro
     const bool pool = (flags & ADAFUSE_POOL_MEAN) != 0;
     if (!pool && T > 0x7fffffff) return ADAFUSE_ERR_UNSUPPORTED;
     const unsigned grid = pool ? 1u : (unsigned)T;
-    af::pregate_kernel<<<grid, af::kRouterThreads, 0, (cudaStream_t)stream>>>(
+    const size_t smem = sizeof(float) * af::kStages * af::stage_floats(E);
+    if (smem > 48 * 1024 &&
+        cudaFuncSetAttribute(af::pregate_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+        return ADAFUSE_ERR_CUDA;
+    af::pregate_kernel<<<grid, af::kRouterThreads, smem, (cudaStream_t)stream>>>(
         static_cast<const uint16_t*>(x), T, H, x_row_stride, W_r, b_r, E, k, flags, idx, gate);
     return af::cuda_err(cudaGetLastError());
 }

@@ -112,34 +112,43 @@ class ClockSampler:
                 "power_w_max": max(r[2] for r in rows), "samples": len(rows), "reasons": reasons}
 
 
-def cpu_oracle_merge(cfg, target_s: float, nthreads: int):
-    """Time the CPU oracle on a bounded sample of the merge workload: whole
-    rows of the first q/gate/down linears; returns (GB/s, seconds, sample)."""
-    import numpy as np
-    import torch
-    import oracle
-    import synth
-    picks = [0, 4, 6]     # q (4096x4096), gate (11008x4096), down (4096x11008)
-    sub = synth.custom([(cfg.linears[i].d_out, cfg.linears[i].d_in) for i in picks], cfg.E, cfg.r, cfg.k, 1,
-                       name="cpu-sample")
-    w = synth.make_weights(sub, 0, device="cpu")
-    idx, gate = [1, 5], [0.4, 0.3]
-    mats = [(w.W_views[i].view(torch.int16).numpy().view(np.uint16),
-             w.A_views[i].view(torch.int16).numpy().view(np.uint16),
-             w.B_views[i].view(torch.int16).numpy().view(np.uint16)) for i in range(len(picks))]
+class OracleMergeSample:
+    """The CPU oracle on a bounded sample of the merge workload: whole rows of
+    the first q (4096x4096), gate (11008x4096) and down (4096x11008) linears."""
 
-    def run(rows):
+    def __init__(self, cfg, nthreads: int):
+        import numpy as np
+        import torch
+        import synth
+        picks = [0, 4, 6]
+        sub = synth.custom([(cfg.linears[i].d_out, cfg.linears[i].d_in) for i in picks], cfg.E, cfg.r, cfg.k, 1,
+                           name="cpu-sample")
+        w = synth.make_weights(sub, 0, device="cpu")
+        self.r = cfg.r
+        self.nthreads = nthreads
+        self.idx, self.gate = [1, 5], [0.4, 0.3]
+        u = lambda t: t.view(torch.int16).numpy().view(np.uint16)
+        self.mats = [(u(w.W_views[i]), u(w.A_views[i]), u(w.B_views[i])) for i in range(len(picks))]
+
+    def run(self, rows):
+        import oracle
         nbytes = 0
         t0 = time.perf_counter()
-        for (W, A, B) in mats:
-            oracle.merge_linear(W, A, B, idx, gate, rows=(0, rows), nthreads=nthreads)
-            nbytes += rows * W.shape[1] * 4 + len(idx) * cfg.r * (rows + W.shape[1]) * 2
+        for (W, A, B) in self.mats:
+            oracle.merge_linear(W, A, B, self.idx, self.gate, rows=(0, rows), nthreads=self.nthreads)
+            nbytes += rows * W.shape[1] * 4 + len(self.idx) * self.r * (rows + W.shape[1]) * 2
         return nbytes, time.perf_counter() - t0
 
-    nb, dt = run(nthreads)
-    rows = max(nthreads, int(nthreads * target_s / max(dt, 1e-6)))
-    rows = min(rows, 4096)
-    nb, dt = run(rows)
+    def calibrate(self, target_s: float) -> int:
+        nb, dt = self.run(self.nthreads)
+        return int(min(4096, max(self.nthreads, self.nthreads * target_s / max(dt, 1e-6))))
+
+
+def cpu_oracle_merge(cfg, target_s: float, nthreads: int):
+    """(GB/s, seconds, sample) of the CPU oracle on about target_s of work."""
+    smp = OracleMergeSample(cfg, nthreads)
+    rows = smp.calibrate(target_s)
+    nb, dt = smp.run(rows)
     return nb / dt / 1e9, dt, f"{rows} rows of each of q, gate, down (k=2, r=16)"
 
 
@@ -179,13 +188,14 @@ def run_reference(args):
     import synth
     cfg = synth.llama7b()
     cores = oracle.max_threads()
+    smp = OracleMergeSample(cfg, cores)
+    rows = smp.calibrate(0.25)
+    sample = f"{rows} rows of each of q, gate, down (k=2, r=16)"
     per_step = []
-    nbytes_total = 0
-    sample = ""
     for s in range(args.warmup + args.steps):
-        gbs, dt, sample = cpu_oracle_merge(cfg, 0.25, cores)
+        nb, dt = smp.run(rows)
         if s >= args.warmup:
-            per_step.append(gbs)
+            per_step.append(nb / dt / 1e9)
     value = statistics.median(per_step)
     line = {
         "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
@@ -208,6 +218,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--config", default="7b", choices=["7b", "13b"])
+    ap.add_argument("--layers", type=int, default=0,
+                    help="use only the first N layers (small profiling case); 0 = the full model")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()
@@ -236,7 +248,10 @@ def main():
     import adapter_merge_b200 as am
     import synth
 
-    cfg = synth.llama7b() if args.config == "7b" else synth.llama13b()
+    if args.config == "7b":
+        cfg = synth.llama7b(args.layers) if args.layers else synth.llama7b()
+    else:
+        cfg = synth.llama13b(args.layers) if args.layers else synth.llama13b()
     seed = 1000 + rank                       # every rank serves its own request and batch
     w = synth.make_weights(cfg, seed, device=dev)
     W_out = torch.empty_like(w.W)
@@ -328,53 +343,87 @@ def main():
     apply_tps = world * T / (a_part * 1e-3)
     apply_gbs = ab / (a_call * 1e-3) / 1e9
 
-    # end to end through the public API with host buffers: H2D of each step's
-    # inputs from pinned memory, D2H of its results, inside the timed region.
+    # End to end through the public API with HOST buffers: every step copies
+    # the call's inputs from pinned host memory to the device and reads its
+    # results back, inside the timed region.
+    #   merge: W, the adapter stacks and the router input in; W' and the
+    #          selection out (PCIe-bound: the whole model crosses twice);
+    #   apply: every linear's x and the first tokens in; every y out (the
+    #          backbone and adapters stay resident, as in serving).
+    # "resident" repeats the merge with only the router input and the
+    # selection crossing PCIe.
     e2e = None
     if not args.no_e2e:
+        h_W = torch.empty(w.W.shape, dtype=w.W.dtype, pin_memory=True)
+        h_W.copy_(w.W)
+        h_A = torch.empty(w.A.shape, dtype=w.A.dtype, pin_memory=True)
+        h_A.copy_(w.A)
+        h_B = torch.empty(w.B.shape, dtype=w.B.dtype, pin_memory=True)
+        h_B.copy_(w.B)
+        h_Wout = torch.empty(W_out.shape, dtype=W_out.dtype, pin_memory=True)
         h_xreq = x_req.cpu().pin_memory()
         h_first = x_first.cpu().pin_memory()
         h_X = X.cpu().pin_memory()
-        h_Y = torch.empty(Y.shape, dtype=Y.dtype).pin_memory()
-        h_sel = torch.empty((2 + 2 * T, cfg.k), dtype=torch.float32).pin_memory()
-        ne = max(5, min(30, args.steps))
+        h_Y = torch.empty(Y.shape, dtype=Y.dtype, pin_memory=True)
+        h_sel = torch.empty((4, cfg.k), dtype=torch.float32, pin_memory=True)
+        ne = 3
 
-        def e2e_step(ev):
+        def e2e_merge(ev, resident):
             ev[0].record(stream)
+            if not resident:
+                w.W.copy_(h_W, non_blocking=True)
+                w.A.copy_(h_A, non_blocking=True)
+                w.B.copy_(h_B, non_blocking=True)
             x_req.copy_(h_xreq, non_blocking=True)
             idx1, gate1 = am.pregate(x_req, w.W_r, cfg.k)
             plan.merge(idx1[0], gate1[0])
+            if not resident:
+                h_Wout.copy_(W_out, non_blocking=True)
             h_sel[0].copy_(idx1[0].view(torch.float32), non_blocking=True)
             h_sel[1].copy_(gate1[0], non_blocking=True)
             ev[1].record(stream)
+
+        def e2e_apply(ev):
+            ev[0].record(stream)
             x_first.copy_(h_first, non_blocking=True)
             X.copy_(h_X, non_blocking=True)
             idxT, gateT = am.pregate(x_first, w.W_r, cfg.k)
             plan.apply(xp, yp, T, idxT, gateT, ws)
             h_Y.copy_(Y, non_blocking=True)
-            ev[2].record(stream)
+            h_sel[2].copy_(idxT[0].view(torch.float32), non_blocking=True)
+            ev[1].record(stream)
 
-        for _ in range(2):
-            e2e_step([torch.cuda.Event(enable_timing=True) for _ in range(3)])
-        torch.cuda.synchronize()
-        eev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(ne)]
-        if world > 1:
-            dist.barrier()
-        for i in range(ne):
-            e2e_step(eev[i])
-        torch.cuda.synchronize()
-        em = torch.tensor([mean([e[0].elapsed_time(e[1]) for e in eev]),
-                           mean([e[1].elapsed_time(e[2]) for e in eev])], dtype=torch.float64, device=dev)
+        def timed(fn, n, *a):
+            evs_ = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n)]
+            fn([torch.cuda.Event(enable_timing=True) for _ in range(2)], *a)      # warm-up
+            torch.cuda.synchronize()
+            if world > 1:
+                dist.barrier()
+            for i in range(n):
+                fn(evs_[i], *a)
+            torch.cuda.synchronize()
+            return mean([e[0].elapsed_time(e[1]) for e in evs_])
+
+        em = torch.tensor([timed(e2e_merge, ne, False), timed(e2e_apply, 10), timed(e2e_merge, 10, True)],
+                          dtype=torch.float64, device=dev)
         if world > 1:
             dist.all_reduce(em, op=dist.ReduceOp.MAX)
-        em_m, em_a = em.tolist()
-        h2d = x_req.numel() * 2 + x_first.numel() * 2 + X.numel() * 2
-        d2h = 2 * cfg.k * 4 + Y.numel() * 2
-        e2e = {"value": round(world * mb / (em_m * 1e-3) / 1e9, 2), "unit": "GB/s",
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "apply_tokens_per_s": round(world * T / (em_a * 1e-3), 1),
-               "note": "merge part: router input H2D + pregate + merge + selection D2H; "
-                       "apply part: x H2D + pregate + apply + y D2H (pinned host buffers)"}
+        em_m, em_a, em_r = em.tolist()
+        h2d_m = (w.W.numel() + w.A.numel() + w.B.numel() + x_req.numel()) * 2
+        d2h_m = W_out.numel() * 2 + 2 * cfg.k * 4
+        h2d_a = (x_first.numel() + X.numel()) * 2
+        d2h_a = Y.numel() * 2 + cfg.k * 4
+        e2e = {"value": round(world * mb / (em_m * 1e-3) / 1e9, 3), "unit": "GB/s",
+               "h2d_bytes_per_step": h2d_m + h2d_a, "d2h_bytes_per_step": d2h_m + d2h_a,
+               "merge_ms": round(em_m, 3), "merge_h2d_bytes": h2d_m, "merge_d2h_bytes": d2h_m,
+               "apply_tokens_per_s": round(world * T / (em_a * 1e-3), 1), "apply_ms": round(em_a, 3),
+               "apply_h2d_bytes": h2d_a, "apply_d2h_bytes": d2h_a,
+               "resident": {"value": round(world * mb / (em_r * 1e-3) / 1e9, 2), "unit": "GB/s",
+                            "h2d_bytes_per_step": x_req.numel() * 2, "d2h_bytes_per_step": 2 * cfg.k * 4,
+                            "note": "weights and adapters resident; only the router input and the selection cross"},
+               "note": "merge with W, A, B in and W' out through pinned host buffers each step; apply with "
+                       "x in and y out (weights resident)"}
+        del h_W, h_A, h_B, h_Wout
 
     cpu = None
     if rank == 0 and not args.no_cpu_baseline:
