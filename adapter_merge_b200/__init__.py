@@ -11,7 +11,7 @@ import os
 from typing import Optional, Sequence
 
 __all__ = [
-    "AdafuseError", "lib", "library_path", "pregate", "segments", "Plan",
+    "AdafuseError", "lib", "library_path", "pregate", "segments", "Plan", "PointerArrays",
     "RENORM", "POOL_MEAN", "STATUS_BAD_INDEX", "STATUS_TIMEOUT",
 ]
 
@@ -188,10 +188,13 @@ class Plan:
     def workspace_bytes(self, T: int, k: int) -> int:
         return int(lib().adafuse_apply_workspace_bytes(self._h, T, k))
 
-    def apply(self, x_ptrs, y_ptrs, T: int, idx, gate, workspace, stream=None):
-        """x_ptrs / y_ptrs: int64 device tensors [n_lin] holding data pointers."""
+    def apply(self, xs, ys, T: int, idx, gate, workspace, stream=None):
+        """Segmented-gather apply over every linear.  xs / ys: per-linear device
+        tensors (x_l [T, d_in], y_l [T, d_out]) or a PointerArrays built once
+        from them (cheaper per call)."""
         k = idx.shape[1]
-        _check(lib().adafuse_apply(self._h, _ptr(x_ptrs), _ptr(y_ptrs), T, _ptr(idx), _ptr(gate), k,
+        ptrs = xs if isinstance(xs, PointerArrays) else PointerArrays(xs, ys)
+        _check(lib().adafuse_apply(self._h, ptrs.x, ptrs.y, T, _ptr(idx), _ptr(gate), k,
                                    _ptr(workspace), workspace.numel() * workspace.element_size(),
                                    _stream(stream)), "adafuse_apply")
 
@@ -217,7 +220,11 @@ class Plan:
             pass
 
 
-def pointer_table(tensors, device):
-    """int64 device tensor of the tensors' data pointers (for apply)."""
-    import torch
-    return torch.tensor([t.data_ptr() for t in tensors], dtype=torch.int64, device=device)
+class PointerArrays:
+    """Host arrays of the device pointers of x_l and y_l, in linear order."""
+
+    def __init__(self, xs, ys):
+        addr = lambda t: t if isinstance(t, int) else t.data_ptr()
+        self.x = (ctypes.c_void_p * len(xs))(*[addr(t) for t in xs])
+        self.y = (ctypes.c_void_p * len(ys))(*[addr(t) for t in ys])
+        self._keep = (list(xs), list(ys))

@@ -39,7 +39,8 @@ def build(force: bool = False, verbose: bool = False, extra=()) -> str:
     if not force and up_to_date():
         return LIB
     tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [NVCC, *FLAGS, *extra, "-o", tmp, *sources()]
+    inc = os.path.join(os.path.dirname(HERE), "include")
+    cmd = [NVCC, *FLAGS, "-I", inc, *extra, "-o", tmp, *sources()]
     if verbose:
         print(" ".join(cmd))
     subprocess.check_call(cmd)

@@ -14,8 +14,14 @@
 //                D[128 x Npad] = W_tile x^T (d_in/64 swizzled K chunks) then
 //                + Bcat_tile S^T (the used experts' B rows, gathered by TMA),
 //                all into one fp32 TMEM accumulator, then y = bf16(D^T).
-// W is streamed exactly once per token tile; the x and S tiles come from L2.
+// Every operand moves by TMA: W and the experts' B rows through the plan's
+// tensor maps, x and S through per-call maps that the host builds (and caches
+// by pointer set, T and workspace) before the launches.  W is streamed exactly
+// once per token tile; the x and S tiles come from L2.
+#include <cudaTypedefs.h>
+
 #include <algorithm>
+#include <cstring>
 
 #include "internal.h"
 #include "ptx.cuh"
@@ -153,20 +159,20 @@ __global__ void __launch_bounds__(kShrinkThreads) shrink_kernel(const LinDesc* l
 
 struct ApplyArgs {
     const LinDesc* lins;
-    const CUtensorMap* maps;
-    const uint16_t* const* x_ptrs;
-    uint16_t* const* y_ptrs;
+    const CUtensorMap* maps;        // plan maps (W, B) per linear
+    const CUtensorMap* xmaps;       // per call: x_l maps [n_lin], then the shrink-output map
+    uint16_t* const* y_ptrs;        // per call, device table
     const int32_t* used;
-    const uint16_t* S;
     const int32_t* cta_start;
     int32_t* status;
     int64_t T;
-    int32_t n_lin, r, Kext, Npad, n_tt;
+    int32_t n_lin, r, Npad, n_tt;
     int32_t ST;
     uint32_t stage_bytes, off_bar, acc_stride, tmem_cols;
 };
 
-constexpr int kApplyThreads = 256;
+constexpr int kApplyThreads = 192;
+constexpr int kApplyEpiWarps = 4;
 constexpr uint32_t kAChunkBytes = kTileM * kChunkK * 2;     // 16 KB
 
 struct UnitIt {
@@ -200,6 +206,11 @@ __device__ __forceinline__ bool mbar_wait_drain2(uint64_t* bar, uint32_t parity)
     return true;
 }
 
+// Warp roles: 0 = TMA producer, 1 = TMEM owner and MMA issuer, 2-5 = epilogue.
+// Stage s holds a 128 x 64 A-operand chunk (W rows, or the used experts' B
+// rows) and an Npad x 64 B-operand chunk (x rows, or shrink-output rows),
+// both K-major; W and x use the 128-byte swizzle, B rows the plain
+// core-matrix layout.
 __global__ void __launch_bounds__(kApplyThreads, 1) apply_fused_kernel(const __grid_constant__ ApplyArgs a)
 {
     extern __shared__ uint8_t smem_raw[];
@@ -215,14 +226,14 @@ __global__ void __launch_bounds__(kApplyThreads, 1) apply_fused_kernel(const __g
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
-        for (int i = 0; i < a.ST; ++i) { mbar_init(&full[i], 1 + 64); mbar_init(&empty[i], 1); }
-        for (int i = 0; i < 2; ++i) { mbar_init(&accfull[i], 1); mbar_init(&accempty[i], 4); }
+        for (int i = 0; i < a.ST; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
+        for (int i = 0; i < 2; ++i) { mbar_init(&accfull[i], 1); mbar_init(&accempty[i], kApplyEpiWarps); }
         mbar_init(donebar, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
     if (threadIdx.x <= kMaxE) s_used[threadIdx.x] = a.used[threadIdx.x];
-    // Zero the A regions: expert chunks load only the groups they use.
+    // Zero the A regions: expert chunks load only the 8-column groups they use.
     for (int s = 0; s < a.ST; ++s)
         for (uint32_t o = threadIdx.x * 16; o < kAChunkBytes; o += kApplyThreads * 16)
             st_shared_v4(smem_u32(base + (size_t)s * a.stage_bytes + o), make_uint4(0, 0, 0, 0));
@@ -242,46 +253,50 @@ __global__ void __launch_bounds__(kApplyThreads, 1) apply_fused_kernel(const __g
 
     const int u_begin = a.cta_start[blockIdx.x], u_end = a.cta_start[blockIdx.x + 1];
     const int nunits = u_end - u_begin;
+    const uint32_t xbytes = (uint32_t)a.Npad * 128u;
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0 && nunits > 0) {
             int64_t gc = 0, issued = 0;
             bool stop = false;
+            const CUtensorMap* mS = a.xmaps + a.n_lin;
             for (int tt = 0; tt < a.n_tt && !stop; ++tt) {
                 UnitIt it;
                 it.init(a.lins, a.n_lin, u_begin);
                 for (int ui = 0; ui < nunits && !stop; ++ui) {
                     const int nKb = (__ldg(&a.lins[it.l].d_in) + kChunkK - 1) / kChunkK;
                     const int m0 = it.mt * kTileM;
+                    const int t0 = tt * kApplyMaxN;
                     const CUtensorMap* mW = a.maps + (size_t)it.l * kMapsPerLinear + kMapW;
                     const CUtensorMap* mB = a.maps + (size_t)it.l * kMapsPerLinear + kMapB;
+                    const CUtensorMap* mX = a.xmaps + it.l;
                     for (int kc = 0; kc < nKb + nKe; ++kc, ++gc) {
                         const int s = (int)(gc % a.ST);
                         if (!mbar_wait(&empty[s], (uint32_t)((gc / a.ST) & 1) ^ 1u, abort_flag)) { stop = true; break; }
                         uint8_t* dst = base + (size_t)s * a.stage_bytes;
                         if (kc < nKb) {
-                            mbar_arrive_expect_tx(&full[s], kAChunkBytes);
+                            mbar_arrive_expect_tx(&full[s], kAChunkBytes + xbytes);
                             tma_load_2d(dst, mW, &full[s], kc * kChunkK, m0);
+                            tma_load_2d(dst + kAChunkBytes, mX, &full[s], kc * kChunkK, t0);
                         } else {
                             const int col0 = (kc - nKb) * kChunkK;
                             int ng = 0;
                             for (int g = 0; g < 8; ++g) if (col0 + g * 8 < U * a.r) ++ng;
-                            mbar_arrive_expect_tx(&full[s], (uint32_t)ng * 2048u);
-                            for (int g = 0; g < 8; ++g) {
+                            mbar_arrive_expect_tx(&full[s], (uint32_t)ng * 2048u + xbytes);
+                            for (int g = 0; g < ng; ++g) {
                                 const int c = col0 + g * 8;
-                                if (c >= U * a.r) break;
                                 const int qq = c / a.r, j0 = c - qq * a.r;
                                 tma_load_3d(dst + (size_t)g * 2048u, mB, &full[s], j0, m0, s_used[1 + qq]);
                             }
+                            tma_load_3d(dst + kAChunkBytes, mS, &full[s], col0, t0, it.l);
                         }
                         issued = gc + 1;
                     }
                     if (ui + 1 < nunits) it.next(a.lins, a.n_lin);
                 }
             }
-            // Drain the TMA loads still in flight (the last ST stages).  The
-            // loaders' cp.async arrivals complete the same phases.
+            // Drain the TMA loads still in flight before the CTA may exit.
             for (int64_t g = std::max<int64_t>(0, issued - a.ST); g < issued; ++g)
                 mbar_wait_drain2(&full[g % a.ST], (uint32_t)((g / a.ST) & 1));
         }
@@ -305,7 +320,6 @@ __global__ void __launch_bounds__(kApplyThreads, 1) apply_fused_kernel(const __g
                         const int s = (int)(gc % a.ST);
                         if (!mbar_wait(&full[s], (uint32_t)((gc / a.ST) & 1), abort_flag)) { stop = true; break; }
                         tc_fence_after();
-                        fence_proxy_async_smem();
                         const uint32_t aaddr = smem_u32(base + (size_t)s * a.stage_bytes);
                         const uint32_t baddr = aaddr + kAChunkBytes;
 #pragma unroll
@@ -327,55 +341,9 @@ __global__ void __launch_bounds__(kApplyThreads, 1) apply_fused_kernel(const __g
             mbar_wait_drain2(donebar, 0);
         }
         __syncwarp();
-    } else if (warp == 2 || warp == 3) {
-        // ------------------------------------------------------------ x / S loaders
-        if (nunits > 0) {
-            const int tl = (warp - 2) * 32 + lane;
-            int64_t gc = 0;
-            bool stop = false;
-            for (int tt = 0; tt < a.n_tt && !stop; ++tt) {
-                UnitIt it;
-                it.init(a.lins, a.n_lin, u_begin);
-                for (int ui = 0; ui < nunits && !stop; ++ui) {
-                    // Per-unit values live in registers: the cp.async below
-                    // clobber memory, which would force reloads from global.
-                    const int d_in = __ldg(&a.lins[it.l].d_in);
-                    const int nKb = (d_in + kChunkK - 1) / kChunkK;
-                    const uint16_t* x = a.x_ptrs[it.l];
-                    const uint16_t* Sl = a.S + (int64_t)it.l * a.T * a.Kext;
-                    const int64_t T = a.T;
-                    const int Kext = a.Kext;
-                    for (int kc = 0; kc < nKb + nKe; ++kc, ++gc) {
-                        const int s = (int)(gc % a.ST);
-                        bool ok = mbar_wait(&empty[s], (uint32_t)((gc / a.ST) & 1) ^ 1u, abort_flag);
-                        if (!__all_sync(0xffffffffu, ok)) { stop = true; break; }
-                        const uint32_t bdst = smem_u32(base + (size_t)s * a.stage_bytes + kAChunkBytes);
-                        for (int id = tl; id < a.Npad * 8; id += 64) {
-                            const int t = id >> 3, c = id & 7;
-                            const int64_t tabs = (int64_t)tt * kApplyMaxN + t;
-                            const uint32_t dst = bdst + (uint32_t)(t >> 3) * 1024u + (uint32_t)(t & 7) * 128u
-                                               + ((uint32_t)(c ^ (t & 7)) << 4);
-                            const uint16_t* src = x;
-                            uint32_t nbytes = 0;
-                            if (kc < nKb) {
-                                const int col = kc * kChunkK + c * 8;
-                                if (tabs < T && col < d_in) { src = x + tabs * d_in + col; nbytes = 16; }
-                            } else {
-                                const int col = (kc - nKb) * kChunkK + c * 8;
-                                if (tabs < T) { src = Sl + tabs * Kext + col; nbytes = 16; }
-                            }
-                            cp_async_16(dst, src, nbytes);
-                        }
-                        cp_async_mbar_arrive_noinc(&full[s]);
-                    }
-                    if (ui + 1 < nunits) it.next(a.lins, a.n_lin);
-                }
-            }
-            asm volatile("cp.async.wait_all;" ::: "memory");
-        }
     } else {
         // ------------------------------------------------------------ epilogue
-        const int q = warp & 3;
+        const int q = warp & 3;        // TMEM lane quarter: warps 2,3,4,5 -> 2,3,0,1
         if (nunits > 0) {
             int64_t uc = 0;
             bool stop = false;
@@ -430,6 +398,24 @@ __global__ void __launch_bounds__(kApplyThreads, 1) apply_fused_kernel(const __g
     if (threadIdx.x == 0 && *abort_flag) atomicOr(a.status, ADAFUSE_STATUS_TIMEOUT);
 }
 
+bool encode_tile_map(CUtensorMap* m, const void* ptr, int rank, const cuuint64_t* dims, const cuuint64_t* strides,
+                     const cuuint32_t* box)
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return false;
+        fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    }
+    cuuint32_t estr[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(ptr), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace
 
 size_t apply_workspace_bytes(const Plan* p, int64_t T, int32_t k)
@@ -437,16 +423,65 @@ size_t apply_workspace_bytes(const Plan* p, int64_t T, int32_t k)
     return ws_layout(p, T, k).total;
 }
 
+size_t apply_call_bytes(int n_lin)
+{
+    return (size_t)(n_lin + 1) * sizeof(CUtensorMap) + (size_t)n_lin * 2 * sizeof(void*);
+}
+
 int launch_apply(Plan* p, const void* const* x_ptrs, void* const* y_ptrs, int64_t T, const int32_t* idx,
                  const float* gate, int32_t k, void* ws, size_t ws_bytes, cudaStream_t s)
 {
     const WsLayout w = ws_layout(p, T, k);
     if (ws_bytes < w.total) return ADAFUSE_ERR_WORKSPACE_TOO_SMALL;
+    for (int l = 0; l < p->n_lin; ++l) {
+        if (!x_ptrs[l] || !y_ptrs[l]) return ADAFUSE_ERR_INVALID_ARG;
+        if ((reinterpret_cast<uintptr_t>(x_ptrs[l]) & 15u) || (reinterpret_cast<uintptr_t>(y_ptrs[l]) & 1u))
+            return ADAFUSE_ERR_UNSUPPORTED;
+    }
     uint8_t* wsb = static_cast<uint8_t*>(ws);
     int32_t* offsets = reinterpret_cast<int32_t*>(wsb + w.off_offsets);
     int32_t* used = reinterpret_cast<int32_t*>(wsb + w.off_used);
     int32_t* perm = reinterpret_cast<int32_t*>(wsb + w.off_perm);
     uint16_t* S = reinterpret_cast<uint16_t*>(wsb + w.off_S);
+    const int32_t Npad = (int32_t)std::min<int64_t>(kApplyMaxN, ((T + 15) / 16) * 16);
+
+    // Per-call descriptors: rebuilt and uploaded only when something changed.
+    CUtensorMap* d_maps = reinterpret_cast<CUtensorMap*>(p->d_call);
+    uint8_t* d_ptrs = p->d_call + (size_t)(p->n_lin + 1) * sizeof(CUtensorMap);
+    const void* const* d_xp = reinterpret_cast<const void* const*>(d_ptrs);
+    void* const* d_yp = reinterpret_cast<void* const*>(d_ptrs + sizeof(void*) * p->n_lin);
+    const bool hit = p->call_valid && p->call_T == T && p->call_ws == ws &&
+                     std::equal(x_ptrs, x_ptrs + p->n_lin, p->call_x.begin()) &&
+                     std::equal(y_ptrs, y_ptrs + p->n_lin, p->call_y.begin());
+    if (!hit) {
+        std::vector<uint8_t> stage(apply_call_bytes(p->n_lin));
+        CUtensorMap* hm = reinterpret_cast<CUtensorMap*>(stage.data());
+        for (int l = 0; l < p->n_lin; ++l) {
+            const int d_in = p->h_desc[l].d_in;
+            cuuint64_t dims[2] = {(cuuint64_t)d_in, (cuuint64_t)T};
+            cuuint64_t strides[1] = {(cuuint64_t)d_in * 2};
+            cuuint32_t box[2] = {64, (cuuint32_t)Npad};
+            if (!encode_tile_map(&hm[l], x_ptrs[l], 2, dims, strides, box)) return ADAFUSE_ERR_UNSUPPORTED;
+        }
+        {
+            cuuint64_t dims[3] = {(cuuint64_t)w.Kext, (cuuint64_t)T, (cuuint64_t)p->n_lin};
+            cuuint64_t strides[2] = {(cuuint64_t)w.Kext * 2, (cuuint64_t)T * w.Kext * 2};
+            cuuint32_t box[3] = {64, (cuuint32_t)Npad, 1};
+            if (!encode_tile_map(&hm[p->n_lin], S, 3, dims, strides, box)) return ADAFUSE_ERR_UNSUPPORTED;
+        }
+        std::memcpy(stage.data() + (size_t)(p->n_lin + 1) * sizeof(CUtensorMap), x_ptrs, sizeof(void*) * p->n_lin);
+        std::memcpy(stage.data() + (size_t)(p->n_lin + 1) * sizeof(CUtensorMap) + sizeof(void*) * p->n_lin, y_ptrs,
+                    sizeof(void*) * p->n_lin);
+        // From pageable memory the copy is staged before the call returns, so
+        // `stage` may go out of scope; it is ordered on `s` before the kernels.
+        if (cudaMemcpyAsync(p->d_call, stage.data(), stage.size(), cudaMemcpyHostToDevice, s) != cudaSuccess)
+            return ADAFUSE_ERR_CUDA;
+        p->call_valid = true;
+        p->call_T = T;
+        p->call_ws = ws;
+        p->call_x.assign(x_ptrs, x_ptrs + p->n_lin);
+        p->call_y.assign(y_ptrs, y_ptrs + p->n_lin);
+    }
 
     int rc = launch_segments(idx, T, k, p->E, offsets, perm, used, p->d_status, s);
     if (rc != ADAFUSE_OK) return rc;
@@ -458,25 +493,23 @@ int launch_apply(Plan* p, const void* const* x_ptrs, void* const* y_ptrs, int64_
             return ADAFUSE_ERR_CUDA;
     }
     shrink_kernel<<<dim3((unsigned)p->n_lin, (unsigned)w.Umax), kShrinkThreads, shrink_smem, s>>>(
-        p->d_desc, reinterpret_cast<const uint16_t* const*>(x_ptrs), T, k, p->r, offsets, perm, used, gate, S, w.Kext,
+        p->d_desc, reinterpret_cast<const uint16_t* const*>(d_xp), T, k, p->r, offsets, perm, used, gate, S, w.Kext,
         w.Umax);
     if (cudaGetLastError() != cudaSuccess) return ADAFUSE_ERR_CUDA;
 
     ApplyArgs a{};
     a.lins = p->d_desc;
     a.maps = p->d_maps;
-    a.x_ptrs = reinterpret_cast<const uint16_t* const*>(x_ptrs);
-    a.y_ptrs = reinterpret_cast<uint16_t* const*>(y_ptrs);
+    a.xmaps = d_maps;
+    a.y_ptrs = reinterpret_cast<uint16_t* const*>(d_yp);
     a.used = used;
-    a.S = S;
     a.cta_start = p->d_apply_start;
     a.status = p->d_status;
     a.T = T;
     a.n_lin = p->n_lin;
     a.r = p->r;
-    a.Kext = w.Kext;
     a.n_tt = (int32_t)((T + kApplyMaxN - 1) / kApplyMaxN);
-    a.Npad = (int32_t)std::min<int64_t>(kApplyMaxN, ((T + 15) / 16) * 16);
+    a.Npad = Npad;
     a.stage_bytes = kAChunkBytes + (uint32_t)a.Npad * 128u;
     uint32_t accs = 32;
     while (accs < (uint32_t)a.Npad) accs <<= 1;

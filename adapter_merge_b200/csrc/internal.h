@@ -7,7 +7,7 @@
 
 #include <vector>
 
-#include "../../include/adafuse.h"
+#include "adafuse.h"
 
 namespace af {
 
@@ -54,6 +54,14 @@ struct Plan {
     int32_t apply_grid = 0;
     int32_t* d_apply_start = nullptr;   // [apply_grid + 1] first unit per CTA
     int32_t last_launches = 0;
+    // Per-call apply descriptors: TMA maps of every x_l and of the shrink
+    // output, and the x / y pointer tables, rebuilt only when the caller's
+    // pointers, T or workspace change.
+    uint8_t* d_call = nullptr;
+    bool call_valid = false;
+    int64_t call_T = 0;
+    const void* call_ws = nullptr;
+    std::vector<const void*> call_x, call_y;
 };
 
 }  // namespace af
@@ -69,6 +77,7 @@ int launch_merge_per_linear(Plan* p, const int32_t* idx, const float* gate, int3
 int launch_segments(const int32_t* idx, int64_t T, int32_t k, int32_t E, int32_t* offsets, int32_t* perm,
                     int32_t* used, int32_t* status, cudaStream_t s);
 size_t apply_workspace_bytes(const Plan* p, int64_t T, int32_t k);
+size_t apply_call_bytes(int n_lin);
 int launch_apply(Plan* p, const void* const* x_ptrs, void* const* y_ptrs, int64_t T, const int32_t* idx,
                  const float* gate, int32_t k, void* ws, size_t ws_bytes, cudaStream_t s);
 

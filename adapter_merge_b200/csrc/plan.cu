@@ -61,6 +61,7 @@ void free_plan(Plan* p)
     if (p->d_maps) cudaFree(p->d_maps);
     if (p->d_status) cudaFree(p->d_status);
     if (p->d_apply_start) cudaFree(p->d_apply_start);
+    if (p->d_call) cudaFree(p->d_call);
     delete static_cast<adafuse_plan*>(p);
 }
 
@@ -153,7 +154,8 @@ extern "C" int adafuse_plan_create(adafuse_plan** out, const adafuse_linear* lin
     bool ok = cudaMalloc(&p->d_desc, sizeof(LinDesc) * n_lin) == cudaSuccess &&
               cudaMalloc(&p->d_maps, sizeof(CUtensorMap) * maps.size()) == cudaSuccess &&
               cudaMalloc(&p->d_status, sizeof(int32_t)) == cudaSuccess &&
-              cudaMalloc(&p->d_apply_start, sizeof(int32_t) * start.size()) == cudaSuccess;
+              cudaMalloc(&p->d_apply_start, sizeof(int32_t) * start.size()) == cudaSuccess &&
+              cudaMalloc(&p->d_call, apply_call_bytes(n_lin)) == cudaSuccess;
     ok = ok && cudaMemcpy(p->d_desc, p->h_desc.data(), sizeof(LinDesc) * n_lin, cudaMemcpyHostToDevice) == cudaSuccess;
     ok = ok && cudaMemcpy(p->d_maps, maps.data(), sizeof(CUtensorMap) * maps.size(), cudaMemcpyHostToDevice) == cudaSuccess;
     ok = ok && cudaMemcpy(p->d_apply_start, start.data(), sizeof(int32_t) * start.size(), cudaMemcpyHostToDevice) == cudaSuccess;

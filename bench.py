@@ -270,7 +270,8 @@ def main():
     for l in cfg.linears:
         ys.append(Y[o:o + T * l.d_out].view(T, l.d_out))
         o += T * l.d_out
-    xp, yp = am.pointer_table(xs, dev), am.pointer_table(ys, dev)
+    xp = am.PointerArrays(xs, ys)
+    yp = None
     ws = torch.empty(plan.workspace_bytes(T, cfg.k), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 

@@ -191,12 +191,20 @@ ADAFUSE_API size_t adafuse_apply_workspace_bytes(const adafuse_plan* plan, int64
  * gated, rounded to bf16), then one tensor-core kernel over all linears that
  * streams W once and adds the expand (the used experts' B rows against the
  * shrink) into the same fp32 accumulator.
- *   x_ptrs   device array [n_lin] of device pointers, x_l bf16 [T, d_in_l] row-major
- *   y_ptrs   device array [n_lin] of device pointers, y_l bf16 [T, d_out_l] row-major
+ *   x_ptrs   HOST array [n_lin] of device pointers, x_l bf16 [T, d_in_l] row-major,
+ *            16-byte aligned
+ *   y_ptrs   HOST array [n_lin] of device pointers, y_l bf16 [T, d_out_l] row-major
  *   idx/gate int32 / fp32 [T, k] (device), e.g. pregate's output
  *   workspace device, >= adafuse_apply_workspace_bytes(plan, T, k), 256-byte aligned
- * Tokens are processed in tiles of 256; T larger than 256 streams W once per tile.
- * Errors: INVALID_ARG, WORKSPACE_TOO_SMALL, UNSUPPORTED (k < 1, k > E).
+ * The call builds TMA descriptors for the x_l and the workspace and uploads
+ * them (with the pointer tables) on `stream`; they are kept in the plan and
+ * rebuilt only when the pointers, T or the workspace differ from the previous
+ * call, so a serving loop that reuses its buffers does no host work beyond the
+ * three launches.  Tokens are processed in tiles of 256; T larger than 256
+ * streams W once per tile.  Each row of idx should hold distinct experts (as
+ * pregate's does); a repeated expert adds its gates.
+ * Errors: INVALID_ARG, WORKSPACE_TOO_SMALL, UNSUPPORTED (k < 1, k > E,
+ * misaligned x_l).
  */
 ADAFUSE_API int adafuse_apply(adafuse_plan* plan, const void* const* x_ptrs, void* const* y_ptrs,
                   int64_t T, const int32_t* idx, const float* gate, int32_t k,

@@ -255,7 +255,8 @@ def apply_setup(cfg, dev, T, seed=0, zero_w=False, sel=None):
     xs_dev = [x.to(dev) for x in xs]
     ys = [torch.empty((T, l.d_out), dtype=torch.bfloat16, device=dev) for l in cfg.linears]
     import adapter_merge_b200 as am
-    xp, yp = am.pointer_table(xs_dev, dev), am.pointer_table(ys, dev)
+    xp = am.PointerArrays(xs_dev, ys)
+    yp = None
     if sel is None:
         idx, gate = synth.random_selection(T, cfg.E, cfg.k, seed + 11, f"asel{cfg.name}{T}")
     else:
@@ -339,6 +340,22 @@ def test_apply_zero_gates_poison_bad_and_duplicate(am, cuda_device):
     check_apply(m, xs, ys, bad.numpy(), gate.numpy().astype(np.float64), "bad/dup")
 
 
+def test_apply_descriptor_cache_follows_pointers_and_T(am, cuda_device):
+    """The per-call TMA descriptors are cached by (pointers, T, workspace):
+    new buffers, a new T and a new workspace must each be picked up."""
+    cfg = synth.custom([(256, 392), (136, 264)], 5, 16, 2, 16, name="acache")
+    m = Model(cfg, cuda_device)
+    for T, seed in ((16, 1), (16, 2), (9, 3), (16, 1)):
+        X, xs = synth.make_apply_inputs(cfg, T, seed)
+        xd = [x.to(cuda_device) for x in xs]
+        ys = [torch.full((T, l.d_out), 7.0, dtype=torch.bfloat16, device=cuda_device) for l in cfg.linears]
+        idx, gate = synth.random_selection(T, cfg.E, cfg.k, seed, "acache")
+        ws = torch.empty(m.plan.workspace_bytes(T, cfg.k) + 256 * seed, dtype=torch.uint8, device=cuda_device)
+        m.plan.apply(xd, ys, T, idx.to(cuda_device), gate.to(cuda_device), ws)
+        torch.cuda.synchronize()
+        check_apply(m, xs, ys, idx.numpy(), gate.numpy().astype(np.float64), f"cache T={T} seed={seed}")
+
+
 def test_apply_equals_merged_weights(am, cuda_device):
     """Merged form equals unmerged: with one shared selection, apply(x) agrees
     with x W'^T for the GPU's own merged W' to within the bf16 rounding of W'."""
@@ -399,7 +416,8 @@ def test_full_size_apply_sampled(am, cuda_device, cfg_fn):
     m = Model(cfg, cuda_device)
     X, xs_dev = synth.make_apply_inputs(cfg, T, 0, device=cuda_device)
     ys = [torch.empty((T, l.d_out), dtype=torch.bfloat16, device=cuda_device) for l in cfg.linears]
-    xp, yp = am.pointer_table(xs_dev, cuda_device), am.pointer_table(ys, cuda_device)
+    xp = am.PointerArrays(xs_dev, ys)
+    yp = None
     xr = synth.make_router_input(cfg, T, 0, device=cuda_device, tag="xfirst")
     idx, gate = am.pregate(xr, m.w.W_r, cfg.k)
     ws = torch.empty(m.plan.workspace_bytes(T, cfg.k), dtype=torch.uint8, device=cuda_device)
