@@ -33,8 +33,9 @@ namespace {
 // ------------------------------------------------------------------ workspace
 
 struct WsLayout {
-    size_t off_offsets, off_used, off_perm, off_S, total;
-    int32_t Umax, Kext;
+    size_t off_offsets, off_used, off_perm, off_S, off_P, total;
+    int32_t Umax, Kext, Mt, Npad, n_tt;
+    int64_t n_su;           // shrink units per token tile: Mt x total K-slices
 };
 
 WsLayout ws_layout(const Plan* p, int64_t T, int32_t k)
@@ -43,115 +44,261 @@ WsLayout ws_layout(const Plan* p, int64_t T, int32_t k)
     const int64_t P = T * k;
     w.Umax = (int32_t)std::min<int64_t>(p->E, P);
     w.Kext = ((w.Umax * p->r + 63) / 64) * 64;
+    w.Mt = (w.Umax * p->r + kTileM - 1) / kTileM;
+    w.Npad = (int32_t)std::min<int64_t>(kApplyMaxN, ((T + 15) / 16) * 16);
+    w.n_tt = (int32_t)((T + kApplyMaxN - 1) / kApplyMaxN);
+    w.n_su = (int64_t)w.Mt * p->total_ks;
+    auto up = [](size_t b) { return ((b + 255) / 256) * 256; };
     w.off_offsets = 0;
     w.off_used = 256;
     w.off_perm = 512;
-    w.off_S = 512 + (((size_t)P * 4 + 255) / 256) * 256;
-    w.total = w.off_S + (((size_t)p->n_lin * (size_t)T * (size_t)w.Kext * 2 + 255) / 256) * 256;
+    w.off_S = 512 + up((size_t)P * 4);
+    w.off_P = w.off_S + up((size_t)p->n_lin * (size_t)T * (size_t)w.Kext * 2);
+    w.total = w.off_P + up((size_t)w.n_tt * (size_t)w.n_su * (size_t)w.Npad * kTileM * 4);
     return w;
 }
 
-// ------------------------------------------------------------------ shrink
-
-constexpr int kShrinkThreads = 256;
-constexpr int kShrinkChunk = 128;               // d_in columns per smem stage
-constexpr int kShrinkWords = kShrinkChunk / 2 + 1;   // padded row (bf16 pairs)
-
-__global__ void __launch_bounds__(kShrinkThreads) shrink_kernel(const LinDesc* lins, const uint16_t* const* x_ptrs,
-                                                                 int64_t T, int32_t k, int32_t r,
-                                                                 const int32_t* offsets, const int32_t* perm,
-                                                                 const int32_t* used, const float* gate, uint16_t* S,
-                                                                 int32_t Kext, int32_t Umax)
+// Shared by the shrink and apply kernels: the per-unit iteration state.
+__device__ __forceinline__ bool mbar_wait_drain2(uint64_t* bar, uint32_t parity)
 {
-    extern __shared__ uint32_t sm_shrink[];
-    const int NB = max(1, kShrinkThreads / r);           // tokens per batch
-    uint32_t* As = sm_shrink;                            // [r][kShrinkWords]
-    uint32_t* Xs = As + r * kShrinkWords;                // [NB][kShrinkWords]
-    int* tok = reinterpret_cast<int*>(Xs + NB * kShrinkWords);   // [NB]
-    float* coef = reinterpret_cast<float*>(tok + NB);            // [NB]
-    __shared__ int s_nb, s_cursor;
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+    }
+    return true;
+}
 
-    const int l = blockIdx.x, q = blockIdx.y, tid = threadIdx.x;
-    const LinDesc L = lins[l];
-    const uint16_t* x = x_ptrs[l];
-    uint16_t* Sl = S + (int64_t)l * T * Kext;
-    const int U = used[0];
+constexpr uint32_t kAChunkBytes = kTileM * kChunkK * 2;     // 16 KB: 128 rows x 64 cols bf16
 
-    // Zero this block's columns for every token (and the padding columns).
+// ------------------------------------------------------------------ shrink
+//
+// S^T = Acat x^T for every linear, on the tensor cores: Acat stacks the A rows
+// of the U used experts (U*r rows, gathered by TMA in 8-row boxes), x^T is the
+// token tile.  Work units are (128-row tile of Acat, 1024-column K-slice of a
+// linear); each unit writes its fp32 partial [Npad x 128] to the workspace and
+// the finalize kernel adds the slices in order, applies the gates and rounds.
+
+struct ShrinkArgs {
+    const LinDesc* lins;
+    const CUtensorMap* maps;
+    const CUtensorMap* xmaps;
+    const int32_t* used;
+    float* P;
+    int32_t* status;
+    int64_t n_su;
+    int32_t n_lin, r, Npad, n_tt, total_ks;
+    int32_t ST, box_rows;
+    uint32_t stage_bytes, off_bar, acc_stride, tmem_cols;
+};
+
+constexpr int kShrinkThreads = 192;
+
+struct ShrinkUnit {
+    int l, mq, ks, k0, nK;
+    __device__ void at(const LinDesc* lins, int n_lin, int total_ks, int64_t u)
     {
-        const int c0 = q * r, c1 = (q == Umax - 1) ? Kext : (q + 1) * r;
-        const int per_row = (c1 - c0) / 8;
-        for (int64_t id = tid; id < T * per_row; id += kShrinkThreads) {
-            const int64_t t = id / per_row;
-            const int cc = (int)(id - t * per_row);
-            *reinterpret_cast<uint4*>(Sl + t * Kext + c0 + cc * 8) = make_uint4(0, 0, 0, 0);
+        mq = (int)(u / total_ks);
+        const int g = (int)(u - (int64_t)mq * total_ks);
+        int lo = 0, hi = n_lin - 1;
+        while (lo < hi) {
+            int mid = (lo + hi + 1) >> 1;
+            if (__ldg(&lins[mid].ks_base) <= g) lo = mid; else hi = mid - 1;
+        }
+        l = lo;
+        ks = g - __ldg(&lins[l].ks_base);
+        k0 = ks * kShrinkKS;
+        const int k1 = min(__ldg(&lins[l].d_in), k0 + kShrinkKS);
+        nK = (k1 - k0 + kChunkK - 1) / kChunkK;
+    }
+};
+
+__global__ void __launch_bounds__(kShrinkThreads, 1) shrink_tc_kernel(const __grid_constant__ ShrinkArgs a)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(base + a.off_bar);
+    uint64_t* empty = full + a.ST;
+    uint64_t* accfull = empty + a.ST;
+    uint64_t* accempty = accfull + 2;
+    uint64_t* donebar = accempty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(donebar + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    int* s_used = reinterpret_cast<int*>(tmem_slot + 4);     // [1 + kMaxE]
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < a.ST; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
+        for (int i = 0; i < 2; ++i) { mbar_init(&accfull[i], 1); mbar_init(&accempty[i], 4); }
+        mbar_init(donebar, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (threadIdx.x <= kMaxE) s_used[threadIdx.x] = a.used[threadIdx.x];
+    for (int s = 0; s < a.ST; ++s)
+        for (uint32_t o = threadIdx.x * 16; o < kAChunkBytes; o += kShrinkThreads * 16)
+            st_shared_v4(smem_u32(base + (size_t)s * a.stage_bytes + o), make_uint4(0, 0, 0, 0));
+    fence_proxy_async_smem();
+    __syncthreads();
+    const int rows = s_used[0] * a.r;          // live rows of Acat
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, a.tmem_cols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    const int64_t total = a.n_su * a.n_tt;
+    const int64_t u_begin = (int64_t)blockIdx.x * total / gridDim.x;
+    const int64_t u_end = ((int64_t)blockIdx.x + 1) * total / gridDim.x;
+    const uint32_t xbytes = (uint32_t)a.Npad * 128u;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int64_t gc = 0, issued = 0;
+            bool stop = false;
+            for (int64_t ua = u_begin; ua < u_end && !stop; ++ua) {
+                const int tt = (int)(ua / a.n_su);
+                ShrinkUnit su;
+                su.at(a.lins, a.n_lin, a.total_ks, ua - (int64_t)tt * a.n_su);
+                if (su.mq * kTileM >= rows) continue;
+                const CUtensorMap* mA = a.maps + (size_t)su.l * kMapsPerLinear + kMapA;
+                const CUtensorMap* mX = a.xmaps + su.l;
+                const int R = a.box_rows;               // A rows per box (divides r and 128)
+                int ng = 0;
+                for (int g = 0; g < kTileM / R; ++g) if (su.mq * kTileM + g * R < rows) ++ng;
+                for (int kc = 0; kc < su.nK; ++kc, ++gc) {
+                    const int s = (int)(gc % a.ST);
+                    if (!mbar_wait(&empty[s], (uint32_t)((gc / a.ST) & 1) ^ 1u, abort_flag)) { stop = true; break; }
+                    uint8_t* dst = base + (size_t)s * a.stage_bytes;
+                    const int col = su.k0 + kc * kChunkK;
+                    mbar_arrive_expect_tx(&full[s], (uint32_t)(ng * R) * 128u + xbytes);
+                    for (int g = 0; g < ng; ++g) {
+                        const int c = su.mq * kTileM + g * R;
+                        const int qq = c / a.r, j0 = c - qq * a.r;
+                        tma_load_3d(dst + (size_t)g * R * 128u, mA, &full[s], col, j0, s_used[1 + qq]);
+                    }
+                    tma_load_2d(dst + kAChunkBytes, mX, &full[s], col, tt * kApplyMaxN);
+                    issued = gc + 1;
+                }
+            }
+            for (int64_t g = std::max<int64_t>(0, issued - a.ST); g < issued; ++g)
+                mbar_wait_drain2(&full[g % a.ST], (uint32_t)((g / a.ST) & 1));
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t idesc = make_idesc_bf16(kTileM, (uint32_t)a.Npad, 0u, 0u);
+            int64_t gc = 0, uc = 0;
+            bool stop = false;
+            for (int64_t ua = u_begin; ua < u_end && !stop; ++ua) {
+                const int tt = (int)(ua / a.n_su);
+                ShrinkUnit su;
+                su.at(a.lins, a.n_lin, a.total_ks, ua - (int64_t)tt * a.n_su);
+                if (su.mq * kTileM >= rows) continue;
+                const int acc = (int)(uc & 1);
+                if (!mbar_wait(&accempty[acc], (uint32_t)((uc >> 1) & 1) ^ 1u, abort_flag)) break;
+                tc_fence_after();
+                const uint32_t d = tmem_base + (uint32_t)acc * a.acc_stride;
+                for (int kc = 0; kc < su.nK; ++kc, ++gc) {
+                    const int s = (int)(gc % a.ST);
+                    if (!mbar_wait(&full[s], (uint32_t)((gc / a.ST) & 1), abort_flag)) { stop = true; break; }
+                    tc_fence_after();
+                    const uint32_t aaddr = smem_u32(base + (size_t)s * a.stage_bytes);
+#pragma unroll
+                    for (int kk = 0; kk < kChunkK / 16; ++kk)
+                        tc_mma_bf16(d, make_sdesc(aaddr + (uint32_t)kk * 32u, 16u, 1024u, kLayoutSw128),
+                                    make_sdesc(aaddr + kAChunkBytes + (uint32_t)kk * 32u, 16u, 1024u, kLayoutSw128),
+                                    idesc, (kc | kk) ? 1u : 0u);
+                    tc_commit(&empty[s]);
+                }
+                if (stop) break;
+                tc_commit(&accfull[acc]);
+                ++uc;
+            }
+            tc_commit(donebar);
+            mbar_wait_drain2(donebar, 0);
+        }
+        __syncwarp();
+    } else {
+        const int q = warp & 3;
+        int64_t uc = 0;
+        for (int64_t ua = u_begin; ua < u_end; ++ua) {
+            const int tt = (int)(ua / a.n_su);
+            const int64_t u = ua - (int64_t)tt * a.n_su;
+            ShrinkUnit su;
+            su.at(a.lins, a.n_lin, a.total_ks, u);
+            if (su.mq * kTileM >= rows) continue;
+            const int acc = (int)(uc & 1);
+            bool ok = mbar_wait(&accfull[acc], (uint32_t)((uc >> 1) & 1), abort_flag);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            tc_fence_after();
+            float* Pu = a.P + ((int64_t)tt * a.n_su + u) * a.Npad * kTileM + q * 32 + lane;
+            const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)acc * a.acc_stride;
+            for (int c0 = 0; c0 < a.Npad; c0 += 32) {
+                uint32_t v[32];
+                if (a.Npad - c0 >= 32) {
+                    tc_ld_x32(tbase + (uint32_t)c0, v);
+                } else {
+                    uint32_t h[16];
+                    tc_ld_x16(tbase + (uint32_t)c0, h);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) { v[i] = h[i]; v[16 + i] = 0; }
+                }
+                tc_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    if (c0 + i < a.Npad) Pu[(int64_t)(c0 + i) * kTileM] = __uint_as_float(v[i]);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&accempty[acc]);
+            ++uc;
         }
     }
-    if (q >= U) return;
-    const int e = used[1 + q];
-    const int seg0 = offsets[e], seg1 = offsets[e + 1];
-    const uint16_t* Ae = L.A + (int64_t)e * L.a_es;
-    if (tid == 0) s_cursor = seg0;
     __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, a.tmem_cols);
+    }
+    if (threadIdx.x == 0 && *abort_flag) atomicOr(a.status, ADAFUSE_STATUS_TIMEOUT);
+}
 
-    const int j = tid % r, bi = tid / r;
-    while (true) {
-        if (tid == 0) {
-            // Next batch of distinct tokens of this segment; pairs of one token
-            // are adjacent (ascending pair id), their gates add up.
-            int nb = 0, c = s_cursor;
-            while (c < seg1) {
-                const int pr = perm[c];
-                const int t = pr / k;
-                if (nb > 0 && tok[nb - 1] == t) { coef[nb - 1] += gate[pr]; ++c; continue; }
-                if (nb == NB) break;
-                tok[nb] = t;
-                coef[nb] = gate[pr];
-                ++nb;
-                ++c;
+// S[l, t, c] = bf16( coef(t, c) * sum over the K-slices of linear l of the
+// partials ), c < U*r; zero for the padding columns up to Kext.  coef(t, c) is
+// the sum of token t's gates on expert used[1 + c/r] (zero if t did not pick it).
+__global__ void __launch_bounds__(128) shrink_finalize_kernel(const LinDesc* lins, const float* P, const int32_t* used,
+                                                               const int32_t* idx, const float* gate, uint16_t* S,
+                                                               int64_t T, int32_t k, int32_t r, int32_t Kext,
+                                                               int32_t Npad, int64_t n_su, int32_t total_ks)
+{
+    __shared__ int s_used[kMaxE + 1];
+    __shared__ int s_idx[kMaxSlots];
+    __shared__ float s_gate[kMaxSlots];
+    const int l = blockIdx.x;
+    const int64_t t = blockIdx.y;
+    if (threadIdx.x <= kMaxE) s_used[threadIdx.x] = used[threadIdx.x];
+    if (threadIdx.x < k) { s_idx[threadIdx.x] = idx[t * k + threadIdx.x]; s_gate[threadIdx.x] = gate[t * k + threadIdx.x]; }
+    __syncthreads();
+    const int rows = s_used[0] * r;
+    const int ks_base = __ldg(&lins[l].ks_base), n_ks = __ldg(&lins[l].n_ks);
+    const int tt = (int)(t / kApplyMaxN), tl = (int)(t - (int64_t)tt * kApplyMaxN);
+    uint16_t* Srow = S + ((int64_t)l * T + t) * Kext;
+    for (int c = threadIdx.x; c < Kext; c += blockDim.x) {
+        float v = 0.f;
+        if (c < rows) {
+            const int e = s_used[1 + c / r];
+            float coef = 0.f;
+            for (int s = 0; s < k; ++s) if (s_idx[s] == e) coef += s_gate[s];
+            if (coef != 0.f) {
+                const int mq = c / kTileM, cl = c - mq * kTileM;
+                const float* p = P + (((int64_t)tt * n_su + (int64_t)mq * total_ks + ks_base) * Npad + tl) * kTileM + cl;
+                float sum = 0.f;
+                for (int ks = 0; ks < n_ks; ++ks) sum += p[(int64_t)ks * Npad * kTileM];
+                v = coef * sum;
             }
-            s_cursor = c;
-            s_nb = nb;
         }
-        __syncthreads();
-        const int nb = s_nb;
-        if (nb == 0) break;
-        float acc = 0.f;
-        for (int c0 = 0; c0 < L.d_in; c0 += kShrinkChunk) {
-            // stage A_e rows and the batch's x rows (bf16 pairs, padded rows)
-            for (int id = tid; id < (r + nb) * (kShrinkChunk / 8); id += kShrinkThreads) {
-                const int row = id / (kShrinkChunk / 8), cc = id % (kShrinkChunk / 8);
-                const int col = c0 + cc * 8;
-                uint4 v = make_uint4(0, 0, 0, 0);
-                uint32_t* dst;
-                if (row < r) {
-                    if (col < L.d_in) v = ld_global_nc_v4(Ae + (int64_t)row * L.d_in + col);
-                    dst = As + row * kShrinkWords + cc * 4;
-                } else {
-                    const int bt = row - r;
-                    if (col < L.d_in) v = ld_global_nc_v4(x + (int64_t)tok[bt] * L.d_in + col);
-                    dst = Xs + bt * kShrinkWords + cc * 4;
-                }
-                dst[0] = v.x; dst[1] = v.y; dst[2] = v.z; dst[3] = v.w;
-            }
-            __syncthreads();
-            if (bi < nb) {
-                const uint32_t* ar = As + j * kShrinkWords;
-                const uint32_t* xr = Xs + bi * kShrinkWords;
-#pragma unroll 8
-                for (int w = 0; w < kShrinkChunk / 2; ++w) {
-                    const uint32_t aw = ar[w], xw = xr[w];
-                    acc = fmaf(bf16lo(xw), bf16lo(aw), acc);
-                    acc = fmaf(bf16hi(xw), bf16hi(aw), acc);
-                }
-            }
-            __syncthreads();
-        }
-        if (bi < nb) {
-            const float v = coef[bi] * acc;
-            Sl[(int64_t)tok[bi] * Kext + q * r + j] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
-        }
-        __syncthreads();
+        Srow[c] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
     }
 }
 
@@ -173,7 +320,6 @@ struct ApplyArgs {
 
 constexpr int kApplyThreads = 192;
 constexpr int kApplyEpiWarps = 4;
-constexpr uint32_t kAChunkBytes = kTileM * kChunkK * 2;     // 16 KB
 
 struct UnitIt {
     int l, mt, n_rt;
@@ -197,14 +343,6 @@ struct UnitIt {
     }
 };
 
-__device__ __forceinline__ bool mbar_wait_drain2(uint64_t* bar, uint32_t parity)
-{
-    const uint64_t t0 = globaltimer_ns();
-    while (!mbar_try_wait(bar, parity)) {
-        if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
-    }
-    return true;
-}
 
 // Warp roles: 0 = TMA producer, 1 = TMEM owner and MMA issuer, 2-5 = epilogue.
 // Stage s holds a 128 x 64 A-operand chunk (W rows, or the used experts' B
@@ -443,12 +581,11 @@ int launch_apply(Plan* p, const void* const* x_ptrs, void* const* y_ptrs, int64_
     int32_t* used = reinterpret_cast<int32_t*>(wsb + w.off_used);
     int32_t* perm = reinterpret_cast<int32_t*>(wsb + w.off_perm);
     uint16_t* S = reinterpret_cast<uint16_t*>(wsb + w.off_S);
-    const int32_t Npad = (int32_t)std::min<int64_t>(kApplyMaxN, ((T + 15) / 16) * 16);
+    const int32_t Npad = w.Npad;
 
     // Per-call descriptors: rebuilt and uploaded only when something changed.
     CUtensorMap* d_maps = reinterpret_cast<CUtensorMap*>(p->d_call);
     uint8_t* d_ptrs = p->d_call + (size_t)(p->n_lin + 1) * sizeof(CUtensorMap);
-    const void* const* d_xp = reinterpret_cast<const void* const*>(d_ptrs);
     void* const* d_yp = reinterpret_cast<void* const*>(d_ptrs + sizeof(void*) * p->n_lin);
     const bool hit = p->call_valid && p->call_T == T && p->call_ws == ws &&
                      std::equal(x_ptrs, x_ptrs + p->n_lin, p->call_x.begin()) &&
@@ -486,16 +623,44 @@ int launch_apply(Plan* p, const void* const* x_ptrs, void* const* y_ptrs, int64_
     int rc = launch_segments(idx, T, k, p->E, offsets, perm, used, p->d_status, s);
     if (rc != ADAFUSE_OK) return rc;
 
-    const int NB = std::max(1, kShrinkThreads / p->r);
-    const size_t shrink_smem = (size_t)(p->r + NB) * kShrinkWords * 4 + (size_t)NB * 8;
-    if (shrink_smem > 48 * 1024) {
-        if (cudaFuncSetAttribute(shrink_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)shrink_smem) != cudaSuccess)
+    uint32_t accs = 32;
+    while (accs < (uint32_t)Npad) accs <<= 1;
+    const uint32_t stage_bytes = kAChunkBytes + (uint32_t)Npad * 128u;
+    const uint32_t kSmemMax = 232448u;
+    int ST = std::min(8, (int)((kSmemMax - 2048u) / stage_bytes));
+    if (ST < 2) return ADAFUSE_ERR_UNSUPPORTED;
+    const uint32_t smem = (uint32_t)ST * stage_bytes + 1024u + 1024u;
+
+    {
+        ShrinkArgs sa{};
+        sa.lins = p->d_desc;
+        sa.maps = p->d_maps;
+        sa.xmaps = d_maps;
+        sa.used = used;
+        sa.P = reinterpret_cast<float*>(wsb + w.off_P);
+        sa.status = p->d_status;
+        sa.n_su = w.n_su;
+        sa.n_lin = p->n_lin;
+        sa.r = p->r;
+        sa.Npad = Npad;
+        sa.n_tt = w.n_tt;
+        sa.total_ks = p->total_ks;
+        sa.ST = ST;
+        sa.box_rows = p->a_box_rows;
+        sa.stage_bytes = stage_bytes;
+        sa.off_bar = (uint32_t)ST * stage_bytes;
+        sa.acc_stride = accs;
+        sa.tmem_cols = 2 * accs;
+        if (cudaFuncSetAttribute(shrink_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
             return ADAFUSE_ERR_CUDA;
+        const int64_t units = w.n_su * w.n_tt;
+        const int grid = (int)std::min<int64_t>(p->num_sms, units);
+        shrink_tc_kernel<<<grid, kShrinkThreads, smem, s>>>(sa);
+        if (cudaGetLastError() != cudaSuccess) return ADAFUSE_ERR_CUDA;
+        shrink_finalize_kernel<<<dim3((unsigned)p->n_lin, (unsigned)T), 128, 0, s>>>(
+            p->d_desc, sa.P, used, idx, gate, S, T, k, p->r, w.Kext, Npad, w.n_su, p->total_ks);
+        if (cudaGetLastError() != cudaSuccess) return ADAFUSE_ERR_CUDA;
     }
-    shrink_kernel<<<dim3((unsigned)p->n_lin, (unsigned)w.Umax), kShrinkThreads, shrink_smem, s>>>(
-        p->d_desc, reinterpret_cast<const uint16_t* const*>(d_xp), T, k, p->r, offsets, perm, used, gate, S, w.Kext,
-        w.Umax);
-    if (cudaGetLastError() != cudaSuccess) return ADAFUSE_ERR_CUDA;
 
     ApplyArgs a{};
     a.lins = p->d_desc;
@@ -508,24 +673,17 @@ int launch_apply(Plan* p, const void* const* x_ptrs, void* const* y_ptrs, int64_
     a.T = T;
     a.n_lin = p->n_lin;
     a.r = p->r;
-    a.n_tt = (int32_t)((T + kApplyMaxN - 1) / kApplyMaxN);
+    a.n_tt = w.n_tt;
     a.Npad = Npad;
-    a.stage_bytes = kAChunkBytes + (uint32_t)a.Npad * 128u;
-    uint32_t accs = 32;
-    while (accs < (uint32_t)a.Npad) accs <<= 1;
+    a.stage_bytes = stage_bytes;
     a.acc_stride = accs;
     a.tmem_cols = 2 * accs;
-    const uint32_t kSmemMax = 232448u;
-    int ST = (int)((kSmemMax - 2048u) / a.stage_bytes);
-    ST = std::min(ST, 8);
-    if (ST < 2) return ADAFUSE_ERR_UNSUPPORTED;
     a.ST = ST;
-    a.off_bar = (uint32_t)ST * a.stage_bytes;
-    const uint32_t smem = a.off_bar + 1024u + 1024u;
+    a.off_bar = (uint32_t)ST * stage_bytes;
     if (cudaFuncSetAttribute(apply_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return ADAFUSE_ERR_CUDA;
     apply_fused_kernel<<<p->apply_grid, kApplyThreads, smem, s>>>(a);
-    p->last_launches = 3;
+    p->last_launches = 4;
     return cuda_err(cudaGetLastError());
 }
 

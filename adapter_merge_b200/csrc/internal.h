@@ -24,12 +24,17 @@ struct LinDesc {
     int32_t d_out, d_in;
     int32_t n_rt;          // ceil(d_out / 128)
     int32_t n_strips;      // ceil(d_in / 128)
+    int32_t ks_base;       // first shrink K-slice (kShrinkKS columns) of this linear
+    int32_t n_ks;          // ceil(d_in / kShrinkKS)
 };
 
 // Tensor maps kept per linear: W (load, 64x128 boxes), W_out (load, 64x128
-// boxes), B (3-D stack), W_out store (64x32 boxes: one per epilogue warp).
-constexpr int kMapsPerLinear = 4;
-constexpr int kMapW = 0, kMapWout = 1, kMapB = 2, kMapWoutStore = 3;
+// boxes), B (3-D stack, 8x128x1 boxes), W_out store (64x32 boxes: one per
+// merge epilogue warp), A (3-D stack, 64 x a_box_rows x 1 boxes, 128-byte
+// swizzle).
+constexpr int kMapsPerLinear = 5;
+constexpr int kMapW = 0, kMapWout = 1, kMapB = 2, kMapWoutStore = 3, kMapA = 4;
+constexpr int kShrinkKS = 1024;  // d_in columns per shrink work unit
 
 constexpr int kTileM = 128;      // output rows per tile (MMA M, TMEM lanes)
 constexpr int kTileN = 128;      // merge: d_in columns per tile (MMA N)
@@ -51,6 +56,8 @@ struct Plan {
     int32_t* d_status = nullptr;
     int64_t merge_tiles = 0;
     int64_t apply_units = 0;
+    int32_t total_ks = 0;             // shrink K-slices over all linears
+    int32_t a_box_rows = 8;           // rows per A-stack TMA box: largest power of two <= 128 dividing r
     int32_t apply_grid = 0;
     int32_t* d_apply_start = nullptr;   // [apply_grid + 1] first unit per CTA
     int32_t last_launches = 0;

@@ -41,6 +41,19 @@ bool encode_w(CUtensorMap* m, const void* ptr, int rows, int cols, int box_rows 
                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// A stack: 3-D [E, r, d_in] bf16, box 64 (d_in) x rows x 1 (expert), 128-byte
+// swizzle: a box is rows/8 whole 1 KB swizzle atoms of A rows.
+bool encode_a(CUtensorMap* m, const void* ptr, int E, int r, int d_in, int64_t a_es, int rows)
+{
+    cuuint64_t dims[3] = {(cuuint64_t)d_in, (cuuint64_t)r, (cuuint64_t)E};
+    cuuint64_t strides[2] = {(cuuint64_t)d_in * 2, (cuuint64_t)a_es * 2};
+    cuuint32_t box[3] = {64, (cuuint32_t)rows, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+                       CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                       CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // B stack: 3-D [E, d_out, r] bf16, box 8 (r) x 128 (rows) x 1 (expert), no swizzle:
 // one box is 16 stacked 8x8 core matrices (2 KB).
 bool encode_b(CUtensorMap* m, const void* ptr, int E, int d_out, int r, int64_t b_es)
@@ -105,7 +118,10 @@ extern "C" int adafuse_plan_create(adafuse_plan** out, const adafuse_linear* lin
     p->h_desc.resize(n_lin);
 
     std::vector<CUtensorMap> maps((size_t)n_lin * kMapsPerLinear);
+    p->a_box_rows = 8;
+    while (p->a_box_rows < 128 && r % (2 * p->a_box_rows) == 0) p->a_box_rows *= 2;
     int64_t tiles = 0, units = 0;
+    int32_t kslices = 0;
     std::vector<int64_t> unit_cost;
     for (int l = 0; l < n_lin; ++l) {
         const adafuse_linear& L = lins[l];
@@ -122,13 +138,17 @@ extern "C" int adafuse_plan_create(adafuse_plan** out, const adafuse_linear* lin
         d.n_strips = (L.d_in + kTileN - 1) / kTileN;
         d.tile_base = tiles;
         d.unit_base = units;
+        d.n_ks = (L.d_in + kShrinkKS - 1) / kShrinkKS;
+        d.ks_base = kslices;
+        kslices += d.n_ks;
         tiles += (int64_t)d.n_rt * d.n_strips;
         units += d.n_rt;
         for (int m = 0; m < d.n_rt; ++m) unit_cost.push_back((L.d_in + kChunkK - 1) / kChunkK + 2);
         if (!encode_w(&maps[(size_t)l * kMapsPerLinear + kMapW], L.W, L.d_out, L.d_in) ||
             !encode_w(&maps[(size_t)l * kMapsPerLinear + kMapWout], L.W_out, L.d_out, L.d_in) ||
             !encode_w(&maps[(size_t)l * kMapsPerLinear + kMapWoutStore], L.W_out, L.d_out, L.d_in, 32) ||
-            !encode_b(&maps[(size_t)l * kMapsPerLinear + kMapB], L.B, E, L.d_out, r, L.b_expert_stride)) {
+            !encode_b(&maps[(size_t)l * kMapsPerLinear + kMapB], L.B, E, L.d_out, r, L.b_expert_stride) ||
+            !encode_a(&maps[(size_t)l * kMapsPerLinear + kMapA], L.A, E, r, L.d_in, L.a_expert_stride, p->a_box_rows)) {
             free_plan(p);
             return ADAFUSE_ERR_UNSUPPORTED;
         }
@@ -136,6 +156,7 @@ extern "C" int adafuse_plan_create(adafuse_plan** out, const adafuse_linear* lin
     if (units > 0x7fffffff) { free_plan(p); return ADAFUSE_ERR_UNSUPPORTED; }
     p->merge_tiles = tiles;
     p->apply_units = units;
+    p->total_ks = kslices;
 
     // Apply: contiguous unit ranges of (nearly) equal streamed bytes per CTA.
     p->apply_grid = (int32_t)std::min<int64_t>(p->num_sms, units);

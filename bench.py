@@ -65,6 +65,20 @@ def apply_bytes(cfg, T, U):
     return b
 
 
+def max_over_ranks(values, dist=None, device=None):
+    """Element-wise maximum of per-rank timings (all ranks must call it)."""
+    import torch
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    if dist is not None and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_throughput(world: int, bytes_per_rank: float, ms: float) -> float:
+    """Whole-job GB/s: every rank moved bytes_per_rank in (at most) ms."""
+    return world * bytes_per_rank / (ms * 1e-3) / 1e9
+
+
 class ClockSampler:
     """nvidia-smi clocks/throttle sampling during the timed region."""
 
@@ -330,16 +344,13 @@ def main():
     def mean(v):
         return sum(v) / len(v)
 
-    times = torch.tensor([total_ms, mean(merge_part), mean(merge_kernel), mean(apply_part), mean(apply_call)],
-                         dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(times, op=dist.ReduceOp.MAX)
-    total_ms, m_part, m_kern, a_part, a_call = times.tolist()
+    total_ms, m_part, m_kern, a_part, a_call = max_over_ranks(
+        [total_ms, mean(merge_part), mean(merge_kernel), mean(apply_part), mean(apply_call)], dist, dev)
 
     mb = merge_bytes(cfg, cfg.k)
     ab = apply_bytes(cfg, T, U)
     peak, peak_kind = read_peaks()
-    merge_gbs = world * mb / (m_part * 1e-3) / 1e9
+    merge_gbs = job_throughput(world, mb, m_part)
     kern_gbs = mb / (m_kern * 1e-3) / 1e9
     apply_tps = world * T / (a_part * 1e-3)
     apply_gbs = ab / (a_call * 1e-3) / 1e9
@@ -405,21 +416,18 @@ def main():
             torch.cuda.synchronize()
             return mean([e[0].elapsed_time(e[1]) for e in evs_])
 
-        em = torch.tensor([timed(e2e_merge, ne, False), timed(e2e_apply, 10), timed(e2e_merge, 10, True)],
-                          dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(em, op=dist.ReduceOp.MAX)
-        em_m, em_a, em_r = em.tolist()
+        em_m, em_a, em_r = max_over_ranks([timed(e2e_merge, ne, False), timed(e2e_apply, 10),
+                                           timed(e2e_merge, 10, True)], dist, dev)
         h2d_m = (w.W.numel() + w.A.numel() + w.B.numel() + x_req.numel()) * 2
         d2h_m = W_out.numel() * 2 + 2 * cfg.k * 4
         h2d_a = (x_first.numel() + X.numel()) * 2
         d2h_a = Y.numel() * 2 + cfg.k * 4
-        e2e = {"value": round(world * mb / (em_m * 1e-3) / 1e9, 3), "unit": "GB/s",
+        e2e = {"value": round(job_throughput(world, mb, em_m), 3), "unit": "GB/s",
                "h2d_bytes_per_step": h2d_m + h2d_a, "d2h_bytes_per_step": d2h_m + d2h_a,
                "merge_ms": round(em_m, 3), "merge_h2d_bytes": h2d_m, "merge_d2h_bytes": d2h_m,
                "apply_tokens_per_s": round(world * T / (em_a * 1e-3), 1), "apply_ms": round(em_a, 3),
                "apply_h2d_bytes": h2d_a, "apply_d2h_bytes": d2h_a,
-               "resident": {"value": round(world * mb / (em_r * 1e-3) / 1e9, 2), "unit": "GB/s",
+               "resident": {"value": round(job_throughput(world, mb, em_r), 2), "unit": "GB/s",
                             "h2d_bytes_per_step": x_req.numel() * 2, "d2h_bytes_per_step": 2 * cfg.k * 4,
                             "note": "weights and adapters resident; only the router input and the selection cross"},
                "note": "merge with W, A, B in and W' out through pinned host buffers each step; apply with "
@@ -452,11 +460,11 @@ def main():
             "apply": {"tokens_per_s": round(apply_tps, 1), "ms": round(a_part, 4), "call_ms": round(a_call, 4),
                       "gbs": round(apply_gbs, 2), "bytes": ab, "distinct_experts": U,
                       "frac_of_peak": round(apply_gbs / peak, 4),
-                      "note": "call = segments + shrink + fused apply (3 launches)"},
+                      "note": "call = segments + shrink + finalize + fused apply (4 launches)"},
             "roofline": {"bound": "hbm", "kernel": "merge_fused_kernel", "achieved": round(kern_gbs, 2),
                          "peak": peak, "unit": "GB/s", "frac": round(kern_gbs / peak, 4),
                          "peak_source": f"{peak_kind} hbm_gbs", "traffic": None},
-            "gpu_launches": 6 * args.steps,
+            "gpu_launches": 7 * args.steps,
             "clocks": clocks,
             "e2e": e2e,
             "cpu_baseline": cpu,

@@ -186,11 +186,13 @@ ADAFUSE_API size_t adafuse_apply_workspace_bytes(const adafuse_plan* plan, int64
 /*
  * Segmented-gather apply, unmerged, for every linear of the plan:
  *   y_l[t, :] = bf16_rne( x_l[t, :] W_l^T + sum_s gate[t,s] (x_l[t, :] A_{idx[t,s]}^T) B_{idx[t,s]}^T )
- * with fp32 accumulation.  Steps: segment build (stable sort of the pairs by
- * expert), shrink (for each used expert, its segment's tokens times A_e^T,
- * gated, rounded to bf16), then one tensor-core kernel over all linears that
- * streams W once and adds the expand (the used experts' B rows against the
- * shrink) into the same fp32 accumulator.
+ * with fp32 accumulation.  Four launches, whatever the number of linears:
+ * segment build (stable sort of the pairs by expert; gives the U experts the
+ * batch uses), shrink (the used experts' A rows times x^T on the tensor cores,
+ * split over 1024-column K-slices), finalize (slices summed in order, gates
+ * applied, rounded to bf16), then one tensor-core kernel over all linears
+ * that streams W once and adds the expand (the used experts' B rows against
+ * the shrink) into the same fp32 accumulator.
  *   x_ptrs   HOST array [n_lin] of device pointers, x_l bf16 [T, d_in_l] row-major,
  *            16-byte aligned
  *   y_ptrs   HOST array [n_lin] of device pointers, y_l bf16 [T, d_out_l] row-major

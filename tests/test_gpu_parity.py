@@ -293,7 +293,7 @@ def test_apply_tiny_chain_with_pregate(am, cuda_device):
     assert np.array_equal(idx.cpu().numpy(), idx_ref)
     check_apply(m, xs, ys, idx_ref, gate_ref, "tiny apply")
     assert m.plan.status() == (0, 0)
-    assert m.plan.last_launches == 3
+    assert m.plan.last_launches == 4
 
 
 @pytest.mark.parametrize("T", [1, 5, 16, 17, 64, 130, 256, 300])
