@@ -310,45 +310,38 @@ struct ApplyArgs {
     const CUtensorMap* xmaps;       // per call: x_l maps [n_lin], then the shrink-output map
     uint16_t* const* y_ptrs;        // per call, device table
     const int32_t* used;
-    const int32_t* cta_start;
+    const int2* order;              // units (linear, 128-row tile), longest first
+    int32_t* sched;                 // [0] next unit, [1] CTAs finished (both back to 0 at exit)
     int32_t* status;
     int64_t T;
-    int32_t n_lin, r, Npad, n_tt;
+    int32_t n_lin, r, Npad, n_tt, n_units;
     int32_t ST;
     uint32_t stage_bytes, off_bar, acc_stride, tmem_cols;
 };
 
 constexpr int kApplyThreads = 192;
 constexpr int kApplyEpiWarps = 4;
+constexpr int kUnitRing = 4;
 
-struct UnitIt {
-    int l, mt, n_rt;
-    __device__ void init(const LinDesc* lins, int n_lin, int64_t u)
-    {
-        int lo = 0, hi = n_lin - 1;
-        while (lo < hi) {
-            int mid = (lo + hi + 1) >> 1;
-            if (lins[mid].unit_base <= u) lo = mid; else hi = mid - 1;
-        }
-        l = lo;
-        n_rt = lins[l].n_rt;
-        mt = (int)(u - lins[l].unit_base);
+// Last CTA out puts the work counters back to zero for the next launch.
+__device__ __forceinline__ void release_counters(int32_t* sched)
+{
+    __threadfence();
+    if (atomicAdd(&sched[1], 1) == (int)gridDim.x - 1) {
+        atomicExch(&sched[0], 0);
+        atomicExch(&sched[1], 0);
+        __threadfence();
     }
-    __device__ void next(const LinDesc* lins, int n_lin)
-    {
-        if (++mt == n_rt) {
-            mt = 0;
-            if (++l < n_lin) n_rt = lins[l].n_rt;
-        }
-    }
-};
+}
 
-
-// Warp roles: 0 = TMA producer, 1 = TMEM owner and MMA issuer, 2-5 = epilogue.
+// Warp roles: 0 = TMA producer and work fetcher, 1 = TMEM owner and MMA
+// issuer, 2-5 = epilogue.  Units are fetched from a global counter (longest
+// first), so SMs that stream faster take more of them; the producer passes
+// each unit id to the other roles through a small ring in shared memory.
 // Stage s holds a 128 x 64 A-operand chunk (W rows, or the used experts' B
-// rows) and an Npad x 64 B-operand chunk (x rows, or shrink-output rows),
-// both K-major; W and x use the 128-byte swizzle, B rows the plain
-// core-matrix layout.
+// rows) and an Npad x 64 B-operand chunk (x rows, or shrink-output rows), both
+// K-major; W and x use the 128-byte swizzle, B rows the plain core-matrix
+// layout.
 __global__ void __launch_bounds__(kApplyThreads, 1) apply_fused_kernel(const __grid_constant__ ApplyArgs a)
 {
     extern __shared__ uint8_t smem_raw[];
@@ -357,15 +350,19 @@ __global__ void __launch_bounds__(kApplyThreads, 1) apply_fused_kernel(const __g
     uint64_t* empty = full + a.ST;
     uint64_t* accfull = empty + a.ST;
     uint64_t* accempty = accfull + 2;
-    uint64_t* donebar = accempty + 2;
+    uint64_t* ufull = accempty + 2;
+    uint64_t* uempty = ufull + kUnitRing;
+    uint64_t* donebar = uempty + kUnitRing;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(donebar + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-    int* s_used = reinterpret_cast<int*>(tmem_slot + 4);     // [1 + kMaxE]
+    int* s_unit = reinterpret_cast<int*>(tmem_slot + 4);       // [kUnitRing]
+    int* s_used = s_unit + kUnitRing;                           // [1 + kMaxE]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         for (int i = 0; i < a.ST; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
         for (int i = 0; i < 2; ++i) { mbar_init(&accfull[i], 1); mbar_init(&accempty[i], kApplyEpiWarps); }
+        for (int i = 0; i < kUnitRing; ++i) { mbar_init(&ufull[i], 1); mbar_init(&uempty[i], 1 + kApplyEpiWarps); }
         mbar_init(donebar, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -389,50 +386,55 @@ __global__ void __launch_bounds__(kApplyThreads, 1) apply_fused_kernel(const __g
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
-    const int u_begin = a.cta_start[blockIdx.x], u_end = a.cta_start[blockIdx.x + 1];
-    const int nunits = u_end - u_begin;
+    const int total = a.n_units * a.n_tt;
     const uint32_t xbytes = (uint32_t)a.Npad * 128u;
 
     if (warp == 0) {
-        // ------------------------------------------------------------ TMA producer
-        if (lane == 0 && nunits > 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
             int64_t gc = 0, issued = 0;
-            bool stop = false;
             const CUtensorMap* mS = a.xmaps + a.n_lin;
-            for (int tt = 0; tt < a.n_tt && !stop; ++tt) {
-                UnitIt it;
-                it.init(a.lins, a.n_lin, u_begin);
-                for (int ui = 0; ui < nunits && !stop; ++ui) {
-                    const int nKb = (__ldg(&a.lins[it.l].d_in) + kChunkK - 1) / kChunkK;
-                    const int m0 = it.mt * kTileM;
-                    const int t0 = tt * kApplyMaxN;
-                    const CUtensorMap* mW = a.maps + (size_t)it.l * kMapsPerLinear + kMapW;
-                    const CUtensorMap* mB = a.maps + (size_t)it.l * kMapsPerLinear + kMapB;
-                    const CUtensorMap* mX = a.xmaps + it.l;
-                    for (int kc = 0; kc < nKb + nKe; ++kc, ++gc) {
-                        const int s = (int)(gc % a.ST);
-                        if (!mbar_wait(&empty[s], (uint32_t)((gc / a.ST) & 1) ^ 1u, abort_flag)) { stop = true; break; }
-                        uint8_t* dst = base + (size_t)s * a.stage_bytes;
-                        if (kc < nKb) {
-                            mbar_arrive_expect_tx(&full[s], kAChunkBytes + xbytes);
-                            tma_load_2d(dst, mW, &full[s], kc * kChunkK, m0);
-                            tma_load_2d(dst + kAChunkBytes, mX, &full[s], kc * kChunkK, t0);
-                        } else {
-                            const int col0 = (kc - nKb) * kChunkK;
-                            int ng = 0;
-                            for (int g = 0; g < 8; ++g) if (col0 + g * 8 < U * a.r) ++ng;
-                            mbar_arrive_expect_tx(&full[s], (uint32_t)ng * 2048u + xbytes);
-                            for (int g = 0; g < ng; ++g) {
-                                const int c = col0 + g * 8;
-                                const int qq = c / a.r, j0 = c - qq * a.r;
-                                tma_load_3d(dst + (size_t)g * 2048u, mB, &full[s], j0, m0, s_used[1 + qq]);
-                            }
-                            tma_load_3d(dst + kAChunkBytes, mS, &full[s], col0, t0, it.l);
+            for (int ui = 0;; ++ui) {
+                const int j = ui & (kUnitRing - 1);
+                if (!mbar_wait(&uempty[j], (uint32_t)((ui / kUnitRing) & 1) ^ 1u, abort_flag)) break;
+                int u = atomicAdd(&a.sched[0], 1);
+                if (u >= total) u = -1;
+                s_unit[j] = u;
+                mbar_arrive(&ufull[j]);
+                if (u < 0) break;
+                const int tt = u / a.n_units;
+                const int2 lm = a.order[u - tt * a.n_units];
+                const int l = lm.x;
+                const int nKb = (__ldg(&a.lins[l].d_in) + kChunkK - 1) / kChunkK;
+                const int m0 = lm.y * kTileM;
+                const int t0 = tt * kApplyMaxN;
+                const CUtensorMap* mW = a.maps + (size_t)l * kMapsPerLinear + kMapW;
+                const CUtensorMap* mB = a.maps + (size_t)l * kMapsPerLinear + kMapB;
+                const CUtensorMap* mX = a.xmaps + l;
+                bool stop = false;
+                for (int kc = 0; kc < nKb + nKe; ++kc, ++gc) {
+                    const int s = (int)(gc % a.ST);
+                    if (!mbar_wait(&empty[s], (uint32_t)((gc / a.ST) & 1) ^ 1u, abort_flag)) { stop = true; break; }
+                    uint8_t* dst = base + (size_t)s * a.stage_bytes;
+                    if (kc < nKb) {
+                        mbar_arrive_expect_tx(&full[s], kAChunkBytes + xbytes);
+                        tma_load_2d(dst, mW, &full[s], kc * kChunkK, m0);
+                        tma_load_2d(dst + kAChunkBytes, mX, &full[s], kc * kChunkK, t0);
+                    } else {
+                        const int col0 = (kc - nKb) * kChunkK;
+                        int ng = 0;
+                        for (int g = 0; g < 8; ++g) if (col0 + g * 8 < U * a.r) ++ng;
+                        mbar_arrive_expect_tx(&full[s], (uint32_t)ng * 2048u + xbytes);
+                        for (int g = 0; g < ng; ++g) {
+                            const int c = col0 + g * 8;
+                            const int qq = c / a.r, j0 = c - qq * a.r;
+                            tma_load_3d(dst + (size_t)g * 2048u, mB, &full[s], j0, m0, s_used[1 + qq]);
                         }
-                        issued = gc + 1;
+                        tma_load_3d(dst + kAChunkBytes, mS, &full[s], col0, t0, l);
                     }
-                    if (ui + 1 < nunits) it.next(a.lins, a.n_lin);
+                    issued = gc + 1;
                 }
+                if (stop) break;
             }
             // Drain the TMA loads still in flight before the CTA may exit.
             for (int64_t g = std::max<int64_t>(0, issued - a.ST); g < issued; ++g)
@@ -440,40 +442,40 @@ __global__ void __launch_bounds__(kApplyThreads, 1) apply_fused_kernel(const __g
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0 && nunits > 0) {
+        if (lane == 0) {
             const uint32_t idesc = make_idesc_bf16(kTileM, (uint32_t)a.Npad, 0u, 0u);
             int64_t gc = 0;
-            int64_t uc = 0;
             bool stop = false;
-            for (int tt = 0; tt < a.n_tt && !stop; ++tt) {
-                UnitIt it;
-                it.init(a.lins, a.n_lin, u_begin);
-                for (int ui = 0; ui < nunits && !stop; ++ui, ++uc) {
-                    const int nKb = (__ldg(&a.lins[it.l].d_in) + kChunkK - 1) / kChunkK;
-                    const int acc = (int)(uc & 1);
-                    if (!mbar_wait(&accempty[acc], (uint32_t)((uc >> 1) & 1) ^ 1u, abort_flag)) { stop = true; break; }
+            for (int ui = 0; !stop; ++ui) {
+                const int j = ui & (kUnitRing - 1);
+                if (!mbar_wait(&ufull[j], (uint32_t)((ui / kUnitRing) & 1), abort_flag)) break;
+                const int u = s_unit[j];
+                mbar_arrive(&uempty[j]);
+                if (u < 0) break;
+                const int l = a.order[u % a.n_units].x;
+                const int nKb = (__ldg(&a.lins[l].d_in) + kChunkK - 1) / kChunkK;
+                const int acc = ui & 1;
+                if (!mbar_wait(&accempty[acc], (uint32_t)((ui >> 1) & 1) ^ 1u, abort_flag)) break;
+                tc_fence_after();
+                const uint32_t d = tmem_base + (uint32_t)acc * a.acc_stride;
+                for (int kc = 0; kc < nKb + nKe; ++kc, ++gc) {
+                    const int s = (int)(gc % a.ST);
+                    if (!mbar_wait(&full[s], (uint32_t)((gc / a.ST) & 1), abort_flag)) { stop = true; break; }
                     tc_fence_after();
-                    const uint32_t d = tmem_base + (uint32_t)acc * a.acc_stride;
-                    for (int kc = 0; kc < nKb + nKe; ++kc, ++gc) {
-                        const int s = (int)(gc % a.ST);
-                        if (!mbar_wait(&full[s], (uint32_t)((gc / a.ST) & 1), abort_flag)) { stop = true; break; }
-                        tc_fence_after();
-                        const uint32_t aaddr = smem_u32(base + (size_t)s * a.stage_bytes);
-                        const uint32_t baddr = aaddr + kAChunkBytes;
+                    const uint32_t aaddr = smem_u32(base + (size_t)s * a.stage_bytes);
+                    const uint32_t baddr = aaddr + kAChunkBytes;
 #pragma unroll
-                        for (int kk = 0; kk < kChunkK / 16; ++kk) {
-                            const uint64_t adesc = (kc < nKb)
-                                ? make_sdesc(aaddr + (uint32_t)kk * 32u, 16u, 1024u, kLayoutSw128)
-                                : make_sdesc(aaddr + (uint32_t)kk * 4096u, 2048u, 128u, kLayoutNone);
-                            const uint64_t bdesc = make_sdesc(baddr + (uint32_t)kk * 32u, 16u, 1024u, kLayoutSw128);
-                            tc_mma_bf16(d, adesc, bdesc, idesc, (kc | kk) ? 1u : 0u);
-                        }
-                        tc_commit(&empty[s]);
+                    for (int kk = 0; kk < kChunkK / 16; ++kk) {
+                        const uint64_t adesc = (kc < nKb)
+                            ? make_sdesc(aaddr + (uint32_t)kk * 32u, 16u, 1024u, kLayoutSw128)
+                            : make_sdesc(aaddr + (uint32_t)kk * 4096u, 2048u, 128u, kLayoutNone);
+                        const uint64_t bdesc = make_sdesc(baddr + (uint32_t)kk * 32u, 16u, 1024u, kLayoutSw128);
+                        tc_mma_bf16(d, adesc, bdesc, idesc, (kc | kk) ? 1u : 0u);
                     }
-                    if (stop) break;
-                    tc_commit(&accfull[acc]);
-                    if (ui + 1 < nunits) it.next(a.lins, a.n_lin);
+                    tc_commit(&empty[s]);
                 }
+                if (stop) break;
+                tc_commit(&accfull[acc]);
             }
             tc_commit(donebar);
             mbar_wait_drain2(donebar, 0);
@@ -482,49 +484,49 @@ __global__ void __launch_bounds__(kApplyThreads, 1) apply_fused_kernel(const __g
     } else {
         // ------------------------------------------------------------ epilogue
         const int q = warp & 3;        // TMEM lane quarter: warps 2,3,4,5 -> 2,3,0,1
-        if (nunits > 0) {
-            int64_t uc = 0;
-            bool stop = false;
-            for (int tt = 0; tt < a.n_tt && !stop; ++tt) {
-                UnitIt it;
-                it.init(a.lins, a.n_lin, u_begin);
-                for (int ui = 0; ui < nunits; ++ui, ++uc) {
-                    const int acc = (int)(uc & 1);
-                    bool ok = mbar_wait(&accfull[acc], (uint32_t)((uc >> 1) & 1), abort_flag);
-                    if (!__all_sync(0xffffffffu, ok)) { stop = true; break; }
-                    tc_fence_after();
-                    const int d_out = __ldg(&a.lins[it.l].d_out);
-                    uint16_t* y = a.y_ptrs[it.l];
-                    const int64_t T = a.T;
-                    const int row = it.mt * kTileM + q * 32 + lane;
-                    const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)acc * a.acc_stride;
-                    for (int c0 = 0; c0 < a.Npad; c0 += 32) {
-                        uint32_t v[32];
-                        if (a.Npad - c0 >= 32) {
-                            tc_ld_x32(tbase + (uint32_t)c0, v);
-                        } else {
-                            uint32_t h[16];
-                            tc_ld_x16(tbase + (uint32_t)c0, h);
+        for (int ui = 0;; ++ui) {
+            const int j = ui & (kUnitRing - 1);
+            bool ok = mbar_wait(&ufull[j], (uint32_t)((ui / kUnitRing) & 1), abort_flag);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            const int u = s_unit[j];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&uempty[j]);
+            if (u < 0) break;
+            const int tt = u / a.n_units;
+            const int2 lm = a.order[u - tt * a.n_units];
+            const int acc = ui & 1;
+            ok = mbar_wait(&accfull[acc], (uint32_t)((ui >> 1) & 1), abort_flag);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            tc_fence_after();
+            const int d_out = __ldg(&a.lins[lm.x].d_out);
+            uint16_t* y = a.y_ptrs[lm.x];
+            const int64_t T = a.T;
+            const int row = lm.y * kTileM + q * 32 + lane;
+            const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)acc * a.acc_stride;
+            for (int c0 = 0; c0 < a.Npad; c0 += 32) {
+                uint32_t v[32];
+                if (a.Npad - c0 >= 32) {
+                    tc_ld_x32(tbase + (uint32_t)c0, v);
+                } else {
+                    uint32_t h[16];
+                    tc_ld_x16(tbase + (uint32_t)c0, h);
 #pragma unroll
-                            for (int i = 0; i < 16; ++i) { v[i] = h[i]; v[16 + i] = 0; }
-                        }
-                        tc_wait_ld();
-                        if (row < d_out) {
-                            const int64_t t0 = (int64_t)tt * kApplyMaxN + c0;
-                            uint16_t* yp = y + t0 * d_out + row;
+                    for (int i = 0; i < 16; ++i) { v[i] = h[i]; v[16 + i] = 0; }
+                }
+                tc_wait_ld();
+                if (row < d_out) {
+                    const int64_t t0 = (int64_t)tt * kApplyMaxN + c0;
+                    uint16_t* yp = y + t0 * d_out + row;
 #pragma unroll
-                            for (int i = 0; i < 32; ++i) {
-                                if (c0 + i < a.Npad && t0 + i < T)
-                                    yp[(int64_t)i * d_out] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[i])));
-                            }
-                        }
+                    for (int i = 0; i < 32; ++i) {
+                        if (c0 + i < a.Npad && t0 + i < T)
+                            yp[(int64_t)i * d_out] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[i])));
                     }
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&accempty[acc]);
-                    if (ui + 1 < nunits) it.next(a.lins, a.n_lin);
                 }
             }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&accempty[acc]);
         }
     }
 
@@ -533,7 +535,10 @@ __global__ void __launch_bounds__(kApplyThreads, 1) apply_fused_kernel(const __g
         tc_fence_after();
         tmem_dealloc(tmem_base, a.tmem_cols);
     }
-    if (threadIdx.x == 0 && *abort_flag) atomicOr(a.status, ADAFUSE_STATUS_TIMEOUT);
+    if (threadIdx.x == 0) {
+        if (*abort_flag) atomicOr(a.status, ADAFUSE_STATUS_TIMEOUT);
+        release_counters(a.sched);
+    }
 }
 
 bool encode_tile_map(CUtensorMap* m, const void* ptr, int rank, const cuuint64_t* dims, const cuuint64_t* strides,
@@ -668,7 +673,9 @@ int launch_apply(Plan* p, const void* const* x_ptrs, void* const* y_ptrs, int64_
     a.xmaps = d_maps;
     a.y_ptrs = reinterpret_cast<uint16_t* const*>(d_yp);
     a.used = used;
-    a.cta_start = p->d_apply_start;
+    a.order = p->d_apply_order;
+    a.sched = p->d_sched;
+    a.n_units = (int32_t)p->apply_units;
     a.status = p->d_status;
     a.T = T;
     a.n_lin = p->n_lin;
@@ -682,7 +689,7 @@ int launch_apply(Plan* p, const void* const* x_ptrs, void* const* y_ptrs, int64_
     a.off_bar = (uint32_t)ST * stage_bytes;
     if (cudaFuncSetAttribute(apply_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return ADAFUSE_ERR_CUDA;
-    apply_fused_kernel<<<p->apply_grid, kApplyThreads, smem, s>>>(a);
+    apply_fused_kernel<<<(int)std::min<int64_t>(p->num_sms, (int64_t)a.n_units * a.n_tt), kApplyThreads, smem, s>>>(a);
     p->last_launches = 4;
     return cuda_err(cudaGetLastError());
 }

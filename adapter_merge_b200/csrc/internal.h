@@ -58,8 +58,8 @@ struct Plan {
     int64_t apply_units = 0;
     int32_t total_ks = 0;             // shrink K-slices over all linears
     int32_t a_box_rows = 8;           // rows per A-stack TMA box: largest power of two <= 128 dividing r
-    int32_t apply_grid = 0;
-    int32_t* d_apply_start = nullptr;   // [apply_grid + 1] first unit per CTA
+    int2* d_apply_order = nullptr;      // apply units (linear, row tile), longest first
+    int32_t* d_sched = nullptr;         // work counters of the persistent kernels (zero between launches)
     int32_t last_launches = 0;
     // Per-call apply descriptors: TMA maps of every x_l and of the shrink
     // output, and the x / y pointer tables, rebuilt only when the caller's

@@ -73,7 +73,8 @@ void free_plan(Plan* p)
     if (p->d_desc) cudaFree(p->d_desc);
     if (p->d_maps) cudaFree(p->d_maps);
     if (p->d_status) cudaFree(p->d_status);
-    if (p->d_apply_start) cudaFree(p->d_apply_start);
+    if (p->d_apply_order) cudaFree(p->d_apply_order);
+    if (p->d_sched) cudaFree(p->d_sched);
     if (p->d_call) cudaFree(p->d_call);
     delete static_cast<adafuse_plan*>(p);
 }
@@ -122,7 +123,6 @@ extern "C" int adafuse_plan_create(adafuse_plan** out, const adafuse_linear* lin
     while (p->a_box_rows < 128 && r % (2 * p->a_box_rows) == 0) p->a_box_rows *= 2;
     int64_t tiles = 0, units = 0;
     int32_t kslices = 0;
-    std::vector<int64_t> unit_cost;
     for (int l = 0; l < n_lin; ++l) {
         const adafuse_linear& L = lins[l];
         LinDesc& d = p->h_desc[l];
@@ -143,7 +143,6 @@ extern "C" int adafuse_plan_create(adafuse_plan** out, const adafuse_linear* lin
         kslices += d.n_ks;
         tiles += (int64_t)d.n_rt * d.n_strips;
         units += d.n_rt;
-        for (int m = 0; m < d.n_rt; ++m) unit_cost.push_back((L.d_in + kChunkK - 1) / kChunkK + 2);
         if (!encode_w(&maps[(size_t)l * kMapsPerLinear + kMapW], L.W, L.d_out, L.d_in) ||
             !encode_w(&maps[(size_t)l * kMapsPerLinear + kMapWout], L.W_out, L.d_out, L.d_in) ||
             !encode_w(&maps[(size_t)l * kMapsPerLinear + kMapWoutStore], L.W_out, L.d_out, L.d_in, 32) ||
@@ -158,28 +157,26 @@ extern "C" int adafuse_plan_create(adafuse_plan** out, const adafuse_linear* lin
     p->apply_units = units;
     p->total_ks = kslices;
 
-    // Apply: contiguous unit ranges of (nearly) equal streamed bytes per CTA.
-    p->apply_grid = (int32_t)std::min<int64_t>(p->num_sms, units);
-    std::vector<int32_t> start(p->apply_grid + 1, 0);
-    {
-        std::vector<int64_t> prefix(unit_cost.size() + 1, 0);
-        for (size_t u = 0; u < unit_cost.size(); ++u) prefix[u + 1] = prefix[u] + unit_cost[u];
-        const int64_t total = prefix.back();
-        for (int c = 0; c <= p->apply_grid; ++c) {
-            const int64_t target = total * c / p->apply_grid;
-            start[c] = (int32_t)(std::lower_bound(prefix.begin(), prefix.end(), target) - prefix.begin());
-        }
-        start[p->apply_grid] = (int32_t)units;
-    }
+    // Apply units in decreasing order of the W bytes they stream (stable), so
+    // that dynamic scheduling ends with short units.
+    std::vector<int2> order;
+    order.reserve((size_t)units);
+    for (int l = 0; l < n_lin; ++l)
+        for (int m = 0; m < p->h_desc[l].n_rt; ++m) order.push_back(make_int2(l, m));
+    std::stable_sort(order.begin(), order.end(), [&](const int2& x, const int2& y) {
+        return p->h_desc[x.x].d_in > p->h_desc[y.x].d_in;
+    });
 
     bool ok = cudaMalloc(&p->d_desc, sizeof(LinDesc) * n_lin) == cudaSuccess &&
               cudaMalloc(&p->d_maps, sizeof(CUtensorMap) * maps.size()) == cudaSuccess &&
               cudaMalloc(&p->d_status, sizeof(int32_t)) == cudaSuccess &&
-              cudaMalloc(&p->d_apply_start, sizeof(int32_t) * start.size()) == cudaSuccess &&
+              cudaMalloc(&p->d_apply_order, sizeof(int2) * order.size()) == cudaSuccess &&
+              cudaMalloc(&p->d_sched, sizeof(int32_t) * 8) == cudaSuccess &&
               cudaMalloc(&p->d_call, apply_call_bytes(n_lin)) == cudaSuccess;
     ok = ok && cudaMemcpy(p->d_desc, p->h_desc.data(), sizeof(LinDesc) * n_lin, cudaMemcpyHostToDevice) == cudaSuccess;
     ok = ok && cudaMemcpy(p->d_maps, maps.data(), sizeof(CUtensorMap) * maps.size(), cudaMemcpyHostToDevice) == cudaSuccess;
-    ok = ok && cudaMemcpy(p->d_apply_start, start.data(), sizeof(int32_t) * start.size(), cudaMemcpyHostToDevice) == cudaSuccess;
+    ok = ok && cudaMemcpy(p->d_apply_order, order.data(), sizeof(int2) * order.size(), cudaMemcpyHostToDevice) == cudaSuccess;
+    ok = ok && cudaMemset(p->d_sched, 0, sizeof(int32_t) * 8) == cudaSuccess;
     ok = ok && cudaMemset(p->d_status, 0, sizeof(int32_t)) == cudaSuccess;
     ok = ok && cudaDeviceSynchronize() == cudaSuccess;
     if (!ok) { free_plan(p); return ADAFUSE_ERR_CUDA; }
