@@ -36,6 +36,7 @@ EXPORTS = (
     "adafuse_switch", "adafuse_merge_per_linear", "adafuse_segments",
     "adafuse_apply_workspace_bytes", "adafuse_apply", "adafuse_plan_status",
     "adafuse_plan_last_launches", "adafuse_strerror", "adafuse_version",
+    "adafuse_apply_noalloc",
 )
 
 
@@ -82,6 +83,7 @@ def lib():
     L.adafuse_apply_workspace_bytes.argtypes = [P, i64, i32]
     L.adafuse_apply_workspace_bytes.restype = ctypes.c_size_t
     L.adafuse_apply.argtypes = [P, P, P, i64, P, P, i32, P, ctypes.c_size_t, P]
+    L.adafuse_apply_noalloc.argtypes = [P, P, P, i64, P, P, i32, P]
     L.adafuse_plan_status.argtypes = [P, P, ctypes.POINTER(i32)]
     L.adafuse_plan_last_launches.argtypes = [P]
     L.adafuse_plan_last_launches.restype = i32
@@ -197,6 +199,16 @@ class Plan:
         _check(lib().adafuse_apply(self._h, ptrs.x, ptrs.y, T, _ptr(idx), _ptr(gate), k,
                                    _ptr(workspace), workspace.numel() * workspace.element_size(),
                                    _stream(stream)), "adafuse_apply")
+
+    def apply_noalloc(self, xs, ys, T: int, idx, gate, stream=None) -> int:
+        """As apply, with the library's own fixed device scratch instead of a
+        workspace (for callers that cannot allocate device memory).  Returns the
+        C return code (ADAFUSE_ERR_WORKSPACE_TOO_SMALL when the call does not
+        fit the scratch) instead of raising, so callers can fall back to apply."""
+        k = idx.shape[1]
+        ptrs = xs if isinstance(xs, PointerArrays) else PointerArrays(xs, ys)
+        return int(lib().adafuse_apply_noalloc(self._h, ptrs.x, ptrs.y, T, _ptr(idx), _ptr(gate), k,
+                                               _stream(stream)))
 
     def status(self, stream=None):
         """(return code, device status bits); clears the status word."""

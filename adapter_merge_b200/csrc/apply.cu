@@ -22,6 +22,7 @@
 
 #include <algorithm>
 #include <cstring>
+#include <mutex>
 
 #include "internal.h"
 #include "ptx.cuh"
@@ -695,3 +696,173 @@ int launch_apply(Plan* p, const void* const* x_ptrs, void* const* y_ptrs, int64_
 }
 
 }  // namespace af
+
+// ------------------------------------------------------------------ apply without allocation
+//
+// Scratch for adafuse_apply_noalloc: the apply workspace and the per-call TMA
+// descriptor area live in this fixed device array instead of caller- or
+// plan-allocated memory.  Every GPU that loads the library holds it until the
+// process exits.  Host code never uses the symbol itself as an address: the
+// address comes from cudaGetSymbolAddress, once per device.
+
+namespace af {
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = 16u << 20;          // 16 MiB
+constexpr int kNoAllocMaxLinears = 1024;                     // host staging lives on the stack
+constexpr int kMaxDevices = 64;
+
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[kMaxDevices] = {};
+std::mutex g_noalloc_stage_mu;
+alignas(64) uint8_t g_noalloc_stage[(kNoAllocMaxLinears + 1) * sizeof(CUtensorMap) + kNoAllocMaxLinears * sizeof(void*)];
+
+// Device address of the scratch array on the current device, looked up the
+// first time each device calls in.
+int noalloc_scratch(void** out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ADAFUSE_ERR_DEVICE;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_addr[dev]) {
+        void* ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return ADAFUSE_ERR_CUDA;
+        g_noalloc_addr[dev] = ptr;
+    }
+    *out = g_noalloc_addr[dev];
+    return ADAFUSE_OK;
+}
+
+}  // namespace
+
+int launch_apply_noalloc(Plan* p, const void* const* x_ptrs, void* const* y_ptrs, int64_t T, const int32_t* idx,
+                         const float* gate, int32_t k, cudaStream_t s)
+{
+    if (p->n_lin > kNoAllocMaxLinears) return ADAFUSE_ERR_UNSUPPORTED;
+    const WsLayout w = ws_layout(p, T, k);
+    const size_t desc_bytes = (((size_t)(p->n_lin + 1) * sizeof(CUtensorMap) + sizeof(void*) * p->n_lin + 255) / 256) * 256;
+    if (desc_bytes + w.total > kNoAllocScratchBytes) return ADAFUSE_ERR_WORKSPACE_TOO_SMALL;
+    for (int l = 0; l < p->n_lin; ++l) {
+        if (!x_ptrs[l] || !y_ptrs[l]) return ADAFUSE_ERR_INVALID_ARG;
+        if ((reinterpret_cast<uintptr_t>(x_ptrs[l]) & 15u) || (reinterpret_cast<uintptr_t>(y_ptrs[l]) & 1u))
+            return ADAFUSE_ERR_UNSUPPORTED;
+    }
+    void* scratch = nullptr;
+    int rc = noalloc_scratch(&scratch);
+    if (rc != ADAFUSE_OK) return rc;
+
+    // Scratch layout: [descriptor area | apply workspace].
+    uint8_t* d_desc = static_cast<uint8_t*>(scratch);
+    CUtensorMap* d_maps = reinterpret_cast<CUtensorMap*>(d_desc);
+    void* const* d_yp = reinterpret_cast<void* const*>(d_desc + (size_t)(p->n_lin + 1) * sizeof(CUtensorMap));
+    uint8_t* wsb = d_desc + desc_bytes;
+    int32_t* offsets = reinterpret_cast<int32_t*>(wsb + w.off_offsets);
+    int32_t* used = reinterpret_cast<int32_t*>(wsb + w.off_used);
+    int32_t* perm = reinterpret_cast<int32_t*>(wsb + w.off_perm);
+    uint16_t* S = reinterpret_cast<uint16_t*>(wsb + w.off_S);
+    float* P = reinterpret_cast<float*>(wsb + w.off_P);
+    const int32_t Npad = w.Npad;
+
+    // Descriptors for this call, staged in a static host buffer (no heap) under
+    // the lock and copied from pageable memory, which the runtime stages
+    // before cudaMemcpyAsync returns, so the buffer is free again at unlock.
+    std::lock_guard<std::mutex> lock(g_noalloc_stage_mu);
+    uint8_t* stage = g_noalloc_stage;
+    CUtensorMap* hm = reinterpret_cast<CUtensorMap*>(stage);
+    for (int l = 0; l < p->n_lin; ++l) {
+        const int d_in = p->h_desc[l].d_in;
+        cuuint64_t dims[2] = {(cuuint64_t)d_in, (cuuint64_t)T};
+        cuuint64_t strides[1] = {(cuuint64_t)d_in * 2};
+        cuuint32_t box[2] = {64, (cuuint32_t)Npad};
+        if (!encode_tile_map(&hm[l], x_ptrs[l], 2, dims, strides, box)) return ADAFUSE_ERR_UNSUPPORTED;
+    }
+    {
+        cuuint64_t dims[3] = {(cuuint64_t)w.Kext, (cuuint64_t)T, (cuuint64_t)p->n_lin};
+        cuuint64_t strides[2] = {(cuuint64_t)w.Kext * 2, (cuuint64_t)T * w.Kext * 2};
+        cuuint32_t box[3] = {64, (cuuint32_t)Npad, 1};
+        if (!encode_tile_map(&hm[p->n_lin], S, 3, dims, strides, box)) return ADAFUSE_ERR_UNSUPPORTED;
+    }
+    const size_t map_bytes = (size_t)(p->n_lin + 1) * sizeof(CUtensorMap);
+    std::memcpy(stage + map_bytes, y_ptrs, sizeof(void*) * p->n_lin);
+    if (cudaMemcpyAsync(d_desc, stage, map_bytes + sizeof(void*) * p->n_lin, cudaMemcpyHostToDevice, s) != cudaSuccess)
+        return ADAFUSE_ERR_CUDA;
+
+    rc = launch_segments(idx, T, k, p->E, offsets, perm, used, p->d_status, s);
+    if (rc != ADAFUSE_OK) return rc;
+
+    uint32_t accs = 32;
+    while (accs < (uint32_t)Npad) accs <<= 1;
+    const uint32_t stage_bytes = kAChunkBytes + (uint32_t)Npad * 128u;
+    const uint32_t kSmemMax = 232448u;
+    const int ST = std::min(8, (int)((kSmemMax - 2048u) / stage_bytes));
+    if (ST < 2) return ADAFUSE_ERR_UNSUPPORTED;
+    const uint32_t smem = (uint32_t)ST * stage_bytes + 1024u + 1024u;
+
+    ShrinkArgs sa{};
+    sa.lins = p->d_desc;
+    sa.maps = p->d_maps;
+    sa.xmaps = d_maps;
+    sa.used = used;
+    sa.P = P;
+    sa.status = p->d_status;
+    sa.n_su = w.n_su;
+    sa.n_lin = p->n_lin;
+    sa.r = p->r;
+    sa.Npad = Npad;
+    sa.n_tt = w.n_tt;
+    sa.total_ks = p->total_ks;
+    sa.ST = ST;
+    sa.box_rows = p->a_box_rows;
+    sa.stage_bytes = stage_bytes;
+    sa.off_bar = (uint32_t)ST * stage_bytes;
+    sa.acc_stride = accs;
+    sa.tmem_cols = 2 * accs;
+    if (cudaFuncSetAttribute(shrink_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+        return ADAFUSE_ERR_CUDA;
+    shrink_tc_kernel<<<(int)std::min<int64_t>(p->num_sms, w.n_su * w.n_tt), kShrinkThreads, smem, s>>>(sa);
+    if (cudaGetLastError() != cudaSuccess) return ADAFUSE_ERR_CUDA;
+    shrink_finalize_kernel<<<dim3((unsigned)p->n_lin, (unsigned)T), 128, 0, s>>>(
+        p->d_desc, P, used, idx, gate, S, T, k, p->r, w.Kext, Npad, w.n_su, p->total_ks);
+    if (cudaGetLastError() != cudaSuccess) return ADAFUSE_ERR_CUDA;
+
+    ApplyArgs a{};
+    a.lins = p->d_desc;
+    a.maps = p->d_maps;
+    a.xmaps = d_maps;
+    a.y_ptrs = reinterpret_cast<uint16_t* const*>(d_yp);
+    a.used = used;
+    a.order = p->d_apply_order;
+    a.sched = p->d_sched;
+    a.n_units = (int32_t)p->apply_units;
+    a.status = p->d_status;
+    a.T = T;
+    a.n_lin = p->n_lin;
+    a.r = p->r;
+    a.n_tt = w.n_tt;
+    a.Npad = Npad;
+    a.stage_bytes = stage_bytes;
+    a.acc_stride = accs;
+    a.tmem_cols = 2 * accs;
+    a.ST = ST;
+    a.off_bar = (uint32_t)ST * stage_bytes;
+    if (cudaFuncSetAttribute(apply_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+        return ADAFUSE_ERR_CUDA;
+    apply_fused_kernel<<<(int)std::min<int64_t>(p->num_sms, (int64_t)a.n_units * a.n_tt), kApplyThreads, smem, s>>>(a);
+    p->last_launches = 4;
+    return cuda_err(cudaGetLastError());
+}
+
+size_t apply_noalloc_limit_bytes() { return kNoAllocScratchBytes; }
+
+}  // namespace af
+
+extern "C" int adafuse_apply_noalloc(adafuse_plan* plan, const void* const* x_ptrs, void* const* y_ptrs, int64_t T,
+                                     const int32_t* idx, const float* gate, int32_t k, adafuse_stream_t stream)
+{
+    if (!plan || !x_ptrs || !y_ptrs || !idx || !gate || T < 1) return ADAFUSE_ERR_INVALID_ARG;
+    if (k < 1 || k > plan->E) return ADAFUSE_ERR_UNSUPPORTED;
+    if (T * (int64_t)k > 0x7fffffff) return ADAFUSE_ERR_UNSUPPORTED;
+    return af::launch_apply_noalloc(plan, x_ptrs, y_ptrs, T, idx, gate, k, (cudaStream_t)stream);
+}

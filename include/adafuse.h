@@ -213,6 +213,41 @@ ADAFUSE_API int adafuse_apply(adafuse_plan* plan, const void* const* x_ptrs, voi
                   void* workspace, size_t ws_bytes, adafuse_stream_t stream);
 
 /*
+ * adafuse_apply without any allocation.  (No counterpart in the paper: this is
+ * a convenience of this library.)
+ *
+ * Computes exactly what adafuse_apply computes, through the same kernels, but
+ * takes no workspace: the workspace and the per-call TMA descriptors live in a
+ * fixed 16 MiB array inside the library's own device memory.  It is for
+ * callers that cannot allocate device memory on their hot path -- a runtime
+ * that hands all GPU memory to its own pool at start-up and has none left to
+ * give out, or code that must not call cudaMalloc there because cudaMalloc can
+ * synchronise the device -- and for callers that would rather not manage a
+ * workspace at all.  It calls no cudaMalloc, cudaFree or other allocating
+ * routine, on the device or the host.
+ *   - Limit: the call needs adafuse_apply_workspace_bytes(plan, T, k) plus
+ *     about 128 bytes per linear for descriptors; if that exceeds 16 MiB it
+ *     returns ADAFUSE_ERR_WORKSPACE_TOO_SMALL and launches nothing (e.g. the
+ *     224-linear Llama-2-7B plan with E = 8, r = 16, top-2 fits up to T = 16).
+ *     At most 1024 linears (ADAFUSE_ERR_UNSUPPORTED beyond).
+ *   - The array exists on every GPU that loads the library, until the process
+ *     exits, whether or not this entry point is used.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture begins.
+ *   - Every call on a device uses the same array and leaves its contents
+ *     behind; nothing in it has to start at zero, because each call writes
+ *     every byte it later reads.  Calls whose work overlaps on the GPU (other
+ *     streams, other plans, other threads) race on the array: the caller must
+ *     order them, e.g. by issuing them on one stream.
+ *   - The descriptors are rebuilt on every call (adafuse_apply caches them).
+ * Arguments, outputs and other errors as adafuse_apply.
+ */
+ADAFUSE_API int adafuse_apply_noalloc(adafuse_plan* plan, const void* const* x_ptrs, void* const* y_ptrs,
+                                      int64_t T, const int32_t* idx, const float* gate, int32_t k,
+                                      adafuse_stream_t stream);
+
+/*
  * Synchronise `stream`, read the plan's device status word into
  * *device_status (host) and clear it.  Returns ADAFUSE_ERR_TIMEOUT if the
  * TIMEOUT bit was set, else ADAFUSE_OK (a BAD_INDEX bit alone is reported in
