@@ -29,6 +29,7 @@ RENORM = 1 << 0
 POOL_MEAN = 1 << 1
 STATUS_BAD_INDEX = 1 << 0
 STATUS_TIMEOUT = 1 << 1
+PLAN_TEST_STALL = 1 << 31
 
 # Every entry point the header declares.
 EXPORTS = (
@@ -151,7 +152,7 @@ class Plan:
     alive while the plan exists.
     """
 
-    def __init__(self, linears: Sequence, E: int, r: int):
+    def __init__(self, linears: Sequence, E: int, r: int, flags: int = 0):
         arr = (Linear * len(linears))()
         for i, (W, W_out, A, B) in enumerate(linears):
             d_out, d_in = W.shape
@@ -166,7 +167,7 @@ class Plan:
         self._keep = list(linears)
         self.E, self.r, self.n_lin = E, r, len(linears)
         h = ctypes.c_void_p()
-        _check(lib().adafuse_plan_create(ctypes.byref(h), arr, len(linears), E, r, 0), "adafuse_plan_create")
+        _check(lib().adafuse_plan_create(ctypes.byref(h), arr, len(linears), E, r, flags), "adafuse_plan_create")
         self._h = h
 
     @property

@@ -54,7 +54,7 @@ WsLayout ws_layout(const Plan* p, int64_t T, int32_t k)
     w.off_used = 256;
     w.off_perm = 512;
     w.off_S = 512 + up((size_t)P * 4);
-    w.off_P = w.off_S + up((size_t)p->n_lin * (size_t)T * (size_t)w.Kext * 2);
+    w.off_P = w.off_S + up((size_t)p->n_lin * (size_t)T * (size_t)(2 * w.Kext) * 2);
     w.total = w.off_P + up((size_t)w.n_tt * (size_t)w.n_su * (size_t)w.Npad * kTileM * 4);
     return w;
 }
@@ -265,9 +265,13 @@ __global__ void __launch_bounds__(kShrinkThreads, 1) shrink_tc_kernel(const __gr
     if (threadIdx.x == 0 && *abort_flag) atomicOr(a.status, ADAFUSE_STATUS_TIMEOUT);
 }
 
-// S[l, t, c] = bf16( coef(t, c) * sum over the K-slices of linear l of the
-// partials ), c < U*r; zero for the padding columns up to Kext.  coef(t, c) is
-// the sum of token t's gates on expert used[1 + c/r] (zero if t did not pick it).
+// s = coef(t, c) * (sum over the K-slices of linear l of the partials), for
+// c < U*r (zero for the padding columns up to Kext); coef(t, c) is the sum of
+// token t's gates on expert used[1 + c/r] (zero if t did not pick it).  s is
+// stored as two bf16 values, S[l, t, c] = bf16(s) and S[l, t, Kext + c] =
+// bf16(s - bf16(s)), whose sum carries s to about 2^-17 relative: the expand
+// multiplies both halves by the same B rows, so the LoRA term keeps close to
+// fp32 precision even where it cancels most of the base product.
 __global__ void __launch_bounds__(128) shrink_finalize_kernel(const LinDesc* lins, const float* P, const int32_t* used,
                                                                const int32_t* idx, const float* gate, uint16_t* S,
                                                                int64_t T, int32_t k, int32_t r, int32_t Kext,
@@ -284,7 +288,7 @@ __global__ void __launch_bounds__(128) shrink_finalize_kernel(const LinDesc* lin
     const int rows = s_used[0] * r;
     const int ks_base = __ldg(&lins[l].ks_base), n_ks = __ldg(&lins[l].n_ks);
     const int tt = (int)(t / kApplyMaxN), tl = (int)(t - (int64_t)tt * kApplyMaxN);
-    uint16_t* Srow = S + ((int64_t)l * T + t) * Kext;
+    uint16_t* Srow = S + ((int64_t)l * T + t) * (2 * Kext);
     for (int c = threadIdx.x; c < Kext; c += blockDim.x) {
         float v = 0.f;
         if (c < rows) {
@@ -299,7 +303,9 @@ __global__ void __launch_bounds__(128) shrink_finalize_kernel(const LinDesc* lin
                 v = coef * sum;
             }
         }
-        Srow[c] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+        const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+        Srow[c] = __bfloat16_as_ushort(hi);
+        Srow[Kext + c] = __bfloat16_as_ushort(__float2bfloat16_rn(v - __bfloat162float(hi)));
     }
 }
 
@@ -315,7 +321,7 @@ struct ApplyArgs {
     int32_t* sched;                 // [0] next unit, [1] CTAs finished (both back to 0 at exit)
     int32_t* status;
     int64_t T;
-    int32_t n_lin, r, Npad, n_tt, n_units;
+    int32_t n_lin, r, Npad, n_tt, n_units, Kext;
     int32_t ST;
     uint32_t stage_bytes, off_bar, acc_stride, tmem_cols;
 };
@@ -376,7 +382,8 @@ __global__ void __launch_bounds__(kApplyThreads, 1) apply_fused_kernel(const __g
     fence_proxy_async_smem();
     __syncthreads();
     const int U = s_used[0];
-    const int nKe = (U * a.r + kChunkK - 1) / kChunkK;
+    const int nKh = (U * a.r + kChunkK - 1) / kChunkK;     // expand chunks per half (hi, lo)
+    const int nKe = 2 * nKh;
 
     if (warp == 1) {
         tmem_alloc(tmem_slot, a.tmem_cols);
@@ -422,7 +429,11 @@ __global__ void __launch_bounds__(kApplyThreads, 1) apply_fused_kernel(const __g
                         tma_load_2d(dst, mW, &full[s], kc * kChunkK, m0);
                         tma_load_2d(dst + kAChunkBytes, mX, &full[s], kc * kChunkK, t0);
                     } else {
-                        const int col0 = (kc - nKb) * kChunkK;
+                        // expand: the hi half of S, then the lo half, each
+                        // against the same B rows of the used experts
+                        const int ke = kc - nKb;
+                        const int half = ke >= nKh ? 1 : 0;
+                        const int col0 = (ke - half * nKh) * kChunkK;
                         int ng = 0;
                         for (int g = 0; g < 8; ++g) if (col0 + g * 8 < U * a.r) ++ng;
                         mbar_arrive_expect_tx(&full[s], (uint32_t)ng * 2048u + xbytes);
@@ -431,7 +442,7 @@ __global__ void __launch_bounds__(kApplyThreads, 1) apply_fused_kernel(const __g
                             const int qq = c / a.r, j0 = c - qq * a.r;
                             tma_load_3d(dst + (size_t)g * 2048u, mB, &full[s], j0, m0, s_used[1 + qq]);
                         }
-                        tma_load_3d(dst + kAChunkBytes, mS, &full[s], col0, t0, l);
+                        tma_load_3d(dst + kAChunkBytes, mS, &full[s], half * a.Kext + col0, t0, l);
                     }
                     issued = gc + 1;
                 }
@@ -607,8 +618,8 @@ int launch_apply(Plan* p, const void* const* x_ptrs, void* const* y_ptrs, int64_
             if (!encode_tile_map(&hm[l], x_ptrs[l], 2, dims, strides, box)) return ADAFUSE_ERR_UNSUPPORTED;
         }
         {
-            cuuint64_t dims[3] = {(cuuint64_t)w.Kext, (cuuint64_t)T, (cuuint64_t)p->n_lin};
-            cuuint64_t strides[2] = {(cuuint64_t)w.Kext * 2, (cuuint64_t)T * w.Kext * 2};
+            cuuint64_t dims[3] = {(cuuint64_t)(2 * w.Kext), (cuuint64_t)T, (cuuint64_t)p->n_lin};
+            cuuint64_t strides[2] = {(cuuint64_t)w.Kext * 4, (cuuint64_t)T * w.Kext * 4};
             cuuint32_t box[3] = {64, (cuuint32_t)Npad, 1};
             if (!encode_tile_map(&hm[p->n_lin], S, 3, dims, strides, box)) return ADAFUSE_ERR_UNSUPPORTED;
         }
@@ -677,6 +688,7 @@ int launch_apply(Plan* p, const void* const* x_ptrs, void* const* y_ptrs, int64_
     a.order = p->d_apply_order;
     a.sched = p->d_sched;
     a.n_units = (int32_t)p->apply_units;
+    a.Kext = w.Kext;
     a.status = p->d_status;
     a.T = T;
     a.n_lin = p->n_lin;
@@ -779,8 +791,8 @@ int launch_apply_noalloc(Plan* p, const void* const* x_ptrs, void* const* y_ptrs
         if (!encode_tile_map(&hm[l], x_ptrs[l], 2, dims, strides, box)) return ADAFUSE_ERR_UNSUPPORTED;
     }
     {
-        cuuint64_t dims[3] = {(cuuint64_t)w.Kext, (cuuint64_t)T, (cuuint64_t)p->n_lin};
-        cuuint64_t strides[2] = {(cuuint64_t)w.Kext * 2, (cuuint64_t)T * w.Kext * 2};
+        cuuint64_t dims[3] = {(cuuint64_t)(2 * w.Kext), (cuuint64_t)T, (cuuint64_t)p->n_lin};
+        cuuint64_t strides[2] = {(cuuint64_t)w.Kext * 4, (cuuint64_t)T * w.Kext * 4};
         cuuint32_t box[3] = {64, (cuuint32_t)Npad, 1};
         if (!encode_tile_map(&hm[p->n_lin], S, 3, dims, strides, box)) return ADAFUSE_ERR_UNSUPPORTED;
     }
@@ -836,6 +848,7 @@ int launch_apply_noalloc(Plan* p, const void* const* x_ptrs, void* const* y_ptrs
     a.order = p->d_apply_order;
     a.sched = p->d_sched;
     a.n_units = (int32_t)p->apply_units;
+    a.Kext = w.Kext;
     a.status = p->d_status;
     a.T = T;
     a.n_lin = p->n_lin;

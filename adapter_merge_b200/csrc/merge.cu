@@ -47,6 +47,7 @@ struct MergeArgs {
     int32_t ns;         // slots in this pass: k (merge) or 2k (switch)
     int32_t Kp;         // ns*r rounded up to 16
     int32_t mode;       // 0: merge W -> W_out; 1: switch, W_out in place
+    int32_t stall;      // test hook: CTA 0 withholds its first W stage
     int32_t SW, SB, NA; // W stages, B stages, A buffers
     uint32_t off_B, off_A, off_bar;
 };
@@ -204,10 +205,12 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_fused_kernel(const __g
                 const CUtensorMap* mW = a.maps + (size_t)it.l * kMapsPerLinear + kmap_in;
                 const int n0 = it.strip * kTileN, m0 = it.rt * kTileM;
                 uint8_t* dstW = sW + (size_t)sw * kWTileBytes;
-                mbar_arrive_expect_tx(&wfull[sw], kWTileBytes);
-                tma_load_2d(dstW, mW, &wfull[sw], n0, m0);
-                tma_load_2d(dstW + kWBoxBytes, mW, &wfull[sw], n0 + 64, m0);
-                issued_w = i + 1;
+                if (!(a.stall && blockIdx.x == 0 && i == 0)) {
+                    mbar_arrive_expect_tx(&wfull[sw], kWTileBytes);
+                    tma_load_2d(dstW, mW, &wfull[sw], n0, m0);
+                    tma_load_2d(dstW + kWBoxBytes, mW, &wfull[sw], n0 + 64, m0);
+                    issued_w = i + 1;
+                }
 
                 const int sb = (int)(i % a.SB);
                 if (!mbar_wait(&bempty[sb], (uint32_t)((i / a.SB) & 1) ^ 1u, abort_flag)) break;
@@ -455,6 +458,7 @@ int launch_merge_fused(Plan* p, const int32_t* idx0, const float* gate0, const i
     a.ns = mode == 1 ? 2 * k : k;
     a.Kp = ((a.ns * p->r + 15) / 16) * 16;
     a.mode = mode;
+    a.stall = (p->flags & ADAFUSE_PLAN_TEST_STALL) ? 1 : 0;
     if (a.ns > kMaxSlots || a.Kp > kMaxKr) return ADAFUSE_ERR_UNSUPPORTED;
 
     const uint32_t BBytes = (uint32_t)a.Kp * 256u;

@@ -66,6 +66,15 @@ typedef struct CUstream_st* adafuse_stream_t;   /* same type as cudaStream_t */
 #define ADAFUSE_RENORM     (1u << 0)   /* pregate: divide the k gates by their sum */
 #define ADAFUSE_POOL_MEAN  (1u << 1)   /* pregate: one decision for the mean of the T rows */
 
+/* ---- plan flags ---- */
+/* Test hook for the failure path: every fused merge or switch on a plan
+ * created with this flag withholds the first shared-memory stage of CTA 0, so
+ * that CTA's pipeline wait runs out (after about 1.5 s) instead of the data
+ * arriving.  The launch then completes with ADAFUSE_STATUS_TIMEOUT set and
+ * W_out incomplete, while the GPU context stays usable.  Never set it outside
+ * tests. */
+#define ADAFUSE_PLAN_TEST_STALL  (1u << 31)
+
 /* ---- device status bits (adafuse_plan_status) ---- */
 #define ADAFUSE_STATUS_BAD_INDEX  (1 << 0)   /* an expert index was outside [0, E); slot skipped */
 #define ADAFUSE_STATUS_TIMEOUT    (1 << 1)   /* a pipeline wait exceeded its limit; output invalid */
@@ -94,8 +103,8 @@ typedef struct adafuse_plan adafuse_plan;     /* opaque, library-owned */
  * split of merge and apply, and the status word.  Everything is built once
  * here so that the hot calls do no host work beyond a launch.
  * The `lins` array (host) is copied; the tensors it points to must outlive the
- * plan.  Uses the current CUDA device.
- * Errors: INVALID_ARG (null pointers, n_lin < 1), UNSUPPORTED (E outside
+ * plan.  Uses the current CUDA device.  `flags` is 0 or ADAFUSE_PLAN_TEST_STALL.
+ * Errors: INVALID_ARG (null pointers, n_lin < 1, other flags), UNSUPPORTED (E outside
  * [1, 32], r not a multiple of 8 or r > 256, d_out/d_in not multiples of 8,
  * misaligned pointers or strides), DEVICE (no sm_100 GPU), CUDA.
  */
@@ -190,9 +199,10 @@ ADAFUSE_API size_t adafuse_apply_workspace_bytes(const adafuse_plan* plan, int64
  * segment build (stable sort of the pairs by expert; gives the U experts the
  * batch uses), shrink (the used experts' A rows times x^T on the tensor cores,
  * split over 1024-column K-slices), finalize (slices summed in order, gates
- * applied, rounded to bf16), then one tensor-core kernel over all linears
- * that streams W once and adds the expand (the used experts' B rows against
- * the shrink) into the same fp32 accumulator.
+ * applied, kept as a pair of bf16 values whose sum is the fp32 result), then
+ * one tensor-core kernel over all linears that streams W once and adds the
+ * expand (the used experts' B rows against both halves of the shrink) into
+ * the same fp32 accumulator.
  *   x_ptrs   HOST array [n_lin] of device pointers, x_l bf16 [T, d_in_l] row-major,
  *            16-byte aligned
  *   y_ptrs   HOST array [n_lin] of device pointers, y_l bf16 [T, d_out_l] row-major

@@ -76,6 +76,7 @@ def test_argument_errors_need_no_device(L):
     assert L.adafuse_plan_create(ctypes.byref(h), arr, 1, 0, 8, 0) == am.ERR_UNSUPPORTED
     assert L.adafuse_plan_create(ctypes.byref(h), arr, 1, 4, 12, 0) == am.ERR_UNSUPPORTED
     assert L.adafuse_plan_create(ctypes.byref(h), arr, 1, 4, 8, 3) == am.ERR_INVALID_ARG
+    assert L.adafuse_plan_create(ctypes.byref(h), arr, 1, 4, 8, (1 << 31) | 1) == am.ERR_INVALID_ARG
     bad = (am.Linear * 1)(am.Linear(4096 + 2, 8192, 16384, 32768, 16, 16, 128, 128))
     assert L.adafuse_plan_create(ctypes.byref(h), bad, 1, 4, 8, 0) == am.ERR_UNSUPPORTED
     bad = (am.Linear * 1)(am.Linear(4096, 8192, 16384, 32768, 12, 16, 128, 128))

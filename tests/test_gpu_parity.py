@@ -434,3 +434,42 @@ def test_full_size_apply_sampled(am, cuda_device, cfg_fn):
             ref = oracle.apply_linear(x, W, A, B, idx_ref, g, tokens=(t, t + 1), nthreads=8)
             assert_close_bf16(u16(ys[l][t:t + 1]), ref, f"{cfg.name} apply linear {l} token {t}")
     assert m.plan.status() == (0, 0)
+
+
+# ------------------------------------------------------------------- sweep
+
+SWEEP = [  # (E, r, k, T): single 4096 x 4096 linear, every value of each axis covered
+    (4, 8, 1, 1), (8, 16, 2, 16), (16, 32, 4, 128), (32, 64, 2, 1), (4, 64, 4, 16),
+    (32, 8, 4, 128), (8, 32, 1, 128), (16, 16, 2, 1), (32, 64, 4, 16), (4, 16, 4, 1),
+]
+
+
+@pytest.mark.parametrize("E,r,k,T", SWEEP)
+def test_sweep_point_merge_and_apply(am, cuda_device, E, r, k, T):
+    """The single-layer sweep: gates from the softmax of N(0,1) logits; merge
+    (sampled rows, with the delta check) and apply at batch T (all tokens for
+    T <= 16, sampled tokens above)."""
+    cfg = synth.sweep_point(E, r, k, T)
+    m = Model(cfg, cuda_device)
+    z = synth.normal((T, E), 1.0, torch.float32, 9, f"sweep-logits-{E}-{T}").numpy()
+    idx, gate = oracle.topk_softmax(z, k)
+    gate32 = gate.astype(np.float32)
+    run_merge(am, m, idx[0], gate32[0], cuda_device)
+    W, A, B = u16(m.w.W_views[0]), u16(m.w.A_views[0]), u16(m.w.B_views[0])
+    for rr in ((0, 2), (2047, 2049), (4090, 4096)):
+        ref = oracle.merge_linear(W, A, B, idx[0], gate32[0].astype(np.float64), rows=rr)
+        got = u16(m.W_out[0][rr[0]:rr[1]])
+        assert_close_bf16(got, ref, f"sweep merge rows {rr}")
+        dz = oracle.merge_linear(np.zeros_like(W), A, B, idx[0], gate32[0].astype(np.float64), rows=rr)
+        assert_delta_frobenius(got, W[rr[0]:rr[1]], ref, dz, f"sweep merge rows {rr}")
+    X, xs = synth.make_apply_inputs(cfg, T, 9)
+    xd = [x.to(cuda_device) for x in xs]
+    ys = [torch.empty((T, 4096), dtype=torch.bfloat16, device=cuda_device)]
+    ws = torch.empty(m.plan.workspace_bytes(T, k), dtype=torch.uint8, device=cuda_device)
+    m.plan.apply(xd, ys, T, torch.as_tensor(idx).to(cuda_device), torch.as_tensor(gate32).to(cuda_device), ws)
+    torch.cuda.synchronize()
+    toks = [(0, T)] if T <= 16 else [(0, 1), (T // 2, T // 2 + 1), (T - 1, T)]
+    for tt in toks:
+        ref = oracle.apply_linear(u16(xs[0]), W, A, B, idx, gate32.astype(np.float64), tokens=tt, nthreads=8)
+        assert_close_bf16(u16(ys[0][tt[0]:tt[1]]), ref, f"sweep apply tokens {tt}")
+    assert m.plan.status() == (0, 0)
