@@ -45,6 +45,26 @@ def read_peaks():
     return FALLBACK_HBM_GBS, "fallback"
 
 
+def profiled_traffic(kernel_files, summary, key):
+    """DRAM bytes per launch recorded in a profiles/ summary, if the kernel's
+    sources still hash to the fingerprint recorded with them; else None."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", summary)
+    if not os.path.exists(path):
+        return None
+    rec = {}
+    for line in open(path):
+        parts = line.strip().split(":")
+        if len(parts) == 2:
+            rec[parts[0].strip()] = parts[1].strip()
+    h = hashlib.sha256()
+    for f in kernel_files:
+        h.update(open(os.path.join(ROOT, "adapter_merge_b200", "csrc", f), "rb").read())
+    if rec.get("kernel_sources_sha256_16") != h.hexdigest()[:16] or key not in rec:
+        return None
+    return int(rec[key])
+
+
 def merge_bytes(cfg, k):
     """Algorithmic bytes of one merge: W read + W' write + selected A and B."""
     b = 0
@@ -348,6 +368,10 @@ def main():
         [total_ms, mean(merge_part), mean(merge_kernel), mean(apply_part), mean(apply_call)], dist, dev)
 
     mb = merge_bytes(cfg, cfg.k)
+    traffic = None
+    if cfg.name == "llama2-7b":
+        traffic = profiled_traffic(["merge.cu", "ptx.cuh", "internal.h"], "merge_fused_kernel_llama2-7b-2layer.md",
+                                   "traffic_bytes_per_full_llama2_7b_launch")
     ab = apply_bytes(cfg, T, U)
     peak, peak_kind = read_peaks()
     merge_gbs = job_throughput(world, mb, m_part)
@@ -463,7 +487,11 @@ def main():
                       "note": "call = segments + shrink + finalize + fused apply (4 launches)"},
             "roofline": {"bound": "hbm", "kernel": "merge_fused_kernel", "achieved": round(kern_gbs, 2),
                          "peak": peak, "unit": "GB/s", "frac": round(kern_gbs / peak, 4),
-                         "peak_source": f"{peak_kind} hbm_gbs", "traffic": None},
+                         "peak_source": f"{peak_kind} hbm_gbs (burst copy)",
+                         "algorithmic_bytes": mb,
+                         "traffic": traffic,
+                         "traffic_source": ("ncu dram bytes, 2-layer capture scaled by elements "
+                                            "(profiles/merge_fused_kernel_llama2-7b-2layer.md)") if traffic else None},
             "gpu_launches": 7 * args.steps,
             "clocks": clocks,
             "e2e": e2e,
