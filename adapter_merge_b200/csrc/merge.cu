@@ -48,8 +48,9 @@ struct MergeArgs {
     int32_t Kp;         // ns*r rounded up to 16
     int32_t mode;       // 0: merge W -> W_out; 1: switch, W_out in place
     int32_t stall;      // test hook: CTA 0 withholds its first W stage
-    int32_t SW, SB, NA; // W stages, B stages, A buffers
-    uint32_t off_B, off_A, off_bar;
+    int32_t SW, SB, NA; // W stages, B stages, A buffers (row-order kernel: SB unused)
+    int32_t box_rows;   // rows per A-stack TMA box (row-order kernel)
+    uint32_t off_B, off_A, off_bar, stage_bytes;
 };
 
 constexpr int kMergeThreads = 384;
@@ -391,6 +392,316 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_fused_kernel(const __g
     if (threadIdx.x == 0 && *abort_flag) atomicOr(a.status, ADAFUSE_STATUS_TIMEOUT);
 }
 
+
+// ------------------------------------------------------------------ row order
+
+// Row-order variant (k*r <= 128): tiles are walked along the rows of each
+// 128-row block, so consecutive tiles of a CTA continue the same rows of W
+// (longer contiguous DRAM runs; ~4 % more streaming bandwidth than walking
+// down column strips in a copy-only measurement of this pipeline).  The gate
+// moves to the B side: warps 2-3 build the gate-scaled Bcat (128 rows x Kp,
+// K-major core matrices) once per row block, and warp 0 loads the raw A rows
+// of the tile's 128 columns by TMA (MN-major, 128-byte swizzle) into the same
+// stage as the W tile.  A stage is released by the MMA (A consumed) and the
+// eight epilogue stores (W' read).
+struct RowTileIt {
+    int l, strip, rt, n_rt, n_strips;
+    __device__ void init(const LinDesc* lins, int n_lin, int64_t g)
+    {
+        int lo = 0, hi = n_lin - 1;
+        while (lo < hi) {
+            int mid = (lo + hi + 1) >> 1;
+            if (lins[mid].tile_base <= g) lo = mid; else hi = mid - 1;
+        }
+        l = lo;
+        n_rt = lins[l].n_rt;
+        n_strips = lins[l].n_strips;
+        const int64_t local = g - lins[l].tile_base;
+        rt = (int)(local / n_strips);
+        strip = (int)(local - (int64_t)rt * n_strips);
+    }
+    __device__ void next(const LinDesc* lins, int n_lin)
+    {
+        if (++strip == n_strips) {
+            strip = 0;
+            if (++rt == n_rt) {
+                rt = 0;
+                if (++l < n_lin) {
+                    n_rt = lins[l].n_rt;
+                    n_strips = lins[l].n_strips;
+                }
+            }
+        }
+    }
+};
+
+__global__ void __launch_bounds__(kMergeThreads, 1) merge_rows_kernel(const __grid_constant__ MergeArgs a)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sStage = base;                       // SW x [W tile 32 KB | A tile Kp x 128]
+    uint8_t* sBcat = base + a.off_B;              // NA x [128 x Kp] gate-scaled B rows
+    uint64_t* full = reinterpret_cast<uint64_t*>(base + a.off_bar);
+    uint64_t* empty = full + a.SW;
+    uint64_t* bcfull = empty + a.SW;
+    uint64_t* bcempty = bcfull + a.NA;
+    uint64_t* accfull = bcempty + a.NA;
+    uint64_t* accempty = accfull + 2;
+    uint64_t* donebar = accempty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(donebar + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    int* s_skip = reinterpret_cast<int*>(tmem_slot + 2);
+    int* s_e = reinterpret_cast<int*>(tmem_slot + 4);
+    float* s_g = reinterpret_cast<float*>(s_e + kMaxSlots);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t ATile = (uint32_t)a.Kp * 256u;      // Kp rows x 128 cols bf16
+    const uint32_t BcBytes = (uint32_t)a.Kp * 256u;    // 128 rows x Kp bf16
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < a.SW; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], kEpiWarps + 1); }
+        for (int i = 0; i < a.NA; ++i) { mbar_init(&bcfull[i], 2); mbar_init(&bcempty[i], 1); }
+        for (int i = 0; i < 2; ++i) { mbar_init(&accfull[i], 1); mbar_init(&accempty[i], kEpiWarps); }
+        mbar_init(donebar, 1);
+        *abort_flag = 0;
+        int bad = 0;
+        int same = 1;
+        for (int s = 0; s < a.ns; ++s) {
+            int e;
+            float g;
+            if (s < a.k) { e = a.idx0[s]; g = a.gate0[s]; }
+            else { e = a.idx1[s - a.k]; g = -a.gate1[s - a.k]; }
+            if (e < 0 || e >= a.E) { bad = 1; e = -1; g = 0.f; }
+            s_e[s] = e;
+            s_g[s] = g;
+        }
+        if (a.mode == 1) {
+            for (int s = 0; s < a.k; ++s)
+                if (a.idx0[s] != a.idx1[s] || __float_as_uint(a.gate0[s]) != __float_as_uint(a.gate1[s])) same = 0;
+        } else {
+            same = 0;
+        }
+        *s_skip = same;
+        if (bad && blockIdx.x == 0) atomicOr(a.status, ADAFUSE_STATUS_BAD_INDEX);
+        fence_mbar_init();
+    }
+    // Zero the A part of every stage: the K padding rows and the rows of
+    // skipped slots are never loaded and must read as finite zeros.
+    for (int st = 0; st < a.SW; ++st)
+        for (uint32_t o = threadIdx.x * 16; o < ATile; o += kMergeThreads * 16)
+            st_shared_v4(smem_u32(sStage + (size_t)st * a.stage_bytes + kWTileBytes + o), make_uint4(0, 0, 0, 0));
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (*s_skip) return;       // switch between identical selections: nothing to do
+
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, 256);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    const int64_t G = gridDim.x;
+    const int64_t t_begin = (int64_t)blockIdx.x * a.total_tiles / G;
+    const int64_t t_end = ((int64_t)blockIdx.x + 1) * a.total_tiles / G;
+    const int64_t count = t_end - t_begin;
+    const int kmap_in = a.mode == 1 ? kMapWout : kMapW;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0 && count > 0) {
+            RowTileIt it;
+            it.init(a.lins, a.n_lin, t_begin);
+            int nvalid = 0;
+            for (int s = 0; s < a.ns; ++s) if (s_e[s] >= 0) ++nvalid;
+            const uint32_t abytes = (uint32_t)nvalid * (uint32_t)a.r * 256u;    // 2 halves x r rows x 128 B
+            const int R = a.box_rows;
+            int64_t issued = 0;
+            for (int64_t i = 0; i < count; ++i) {
+                const int sw = (int)(i % a.SW);
+                if (!mbar_wait(&empty[sw], (uint32_t)((i / a.SW) & 1) ^ 1u, abort_flag)) break;
+                const CUtensorMap* mW = a.maps + (size_t)it.l * kMapsPerLinear + kmap_in;
+                const CUtensorMap* mA = a.maps + (size_t)it.l * kMapsPerLinear + kMapA;
+                const int n0 = it.strip * kTileN, m0 = it.rt * kTileM;
+                uint8_t* dst = sStage + (size_t)sw * a.stage_bytes;
+                if (!(a.stall && blockIdx.x == 0 && i == 0)) {
+                    mbar_arrive_expect_tx(&full[sw], kWTileBytes + abytes);
+                    tma_load_2d(dst, mW, &full[sw], n0, m0);
+                    tma_load_2d(dst + kWBoxBytes, mW, &full[sw], n0 + 64, m0);
+                    for (int s = 0; s < a.ns; ++s) {
+                        const int e = s_e[s];
+                        if (e < 0) continue;
+                        for (int h = 0; h < 2; ++h)
+                            for (int j0 = 0; j0 < a.r; j0 += R)
+                                tma_load_3d(dst + kWTileBytes + (size_t)h * a.Kp * 128u + (size_t)((s * a.r + j0) / 8) * 1024u,
+                                            mA, &full[sw], n0 + 64 * h, j0, e);
+                    }
+                    issued = i + 1;
+                }
+                if (i + 1 < count) it.next(a.lins, a.n_lin);
+            }
+            for (int64_t j = std::max<int64_t>(0, issued - a.SW); j < issued; ++j)
+                mbar_wait_drain(&full[j % a.SW], (uint32_t)((j / a.SW) & 1));
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0 && count > 0) {
+            RowTileIt it;
+            it.init(a.lins, a.n_lin, t_begin);
+            const uint32_t idesc = make_idesc_bf16(kTileM, kTileN, 0u, 1u);
+            const uint32_t lbo_a = (uint32_t)a.Kp * 128u;       // 64-column blocks of the A tile
+            int64_t blk_seq = -1;
+            for (int64_t i = 0; i < count; ++i) {
+                const bool first = (i == 0) || (it.strip == 0);
+                const bool last = (i + 1 == count) || (it.strip == it.n_strips - 1);
+                if (first) ++blk_seq;
+                const int bb = (int)(blk_seq % a.NA);
+                const int sw = (int)(i % a.SW);
+                const int acc = (int)(i & 1);
+                if (!mbar_wait(&full[sw], (uint32_t)((i / a.SW) & 1), abort_flag)) break;
+                if (first && !mbar_wait(&bcfull[bb], (uint32_t)((blk_seq / a.NA) & 1), abort_flag)) break;
+                if (!mbar_wait(&accempty[acc], (uint32_t)((i >> 1) & 1) ^ 1u, abort_flag)) break;
+                tc_fence_after();
+                const uint32_t d = tmem_base + (uint32_t)acc * kTileN;
+                const uint32_t bcaddr = smem_u32(sBcat + (size_t)bb * BcBytes);
+                const uint32_t aaddr = smem_u32(sStage + (size_t)sw * a.stage_bytes + kWTileBytes);
+                for (int kk = 0; kk < a.Kp / 16; ++kk) {
+                    const uint64_t adesc = make_sdesc(bcaddr + (uint32_t)kk * 4096u, 2048u, 128u, kLayoutNone);
+                    const uint64_t bdesc = make_sdesc(aaddr + (uint32_t)kk * 2048u, lbo_a, 1024u, kLayoutSw128);
+                    tc_mma_bf16(d, adesc, bdesc, idesc, kk > 0 ? 1u : 0u);
+                }
+                tc_commit(&accfull[acc]);
+                tc_commit(&empty[sw]);
+                if (last) tc_commit(&bcempty[bb]);
+                if (i + 1 < count) it.next(a.lins, a.n_lin);
+            }
+            tc_commit(donebar);
+            mbar_wait_drain(donebar, 0);
+        }
+        __syncwarp();
+    } else if (warp == 2 || warp == 3) {
+        // ------------------------------------------------------------ Bcat builder
+        if (count > 0) {
+            const int tb = (warp - 2) * 32 + lane;
+            RowTileIt it;
+            it.init(a.lins, a.n_lin, t_begin);
+            int64_t blk_seq = -1;
+            for (int64_t i = 0; i < count; ++i) {
+                if (i == 0 || it.strip == 0) {
+                    ++blk_seq;
+                    const int bb = (int)(blk_seq % a.NA);
+                    bool ok = mbar_wait(&bcempty[bb], (uint32_t)((blk_seq / a.NA) & 1) ^ 1u, abort_flag);
+                    ok = __all_sync(0xffffffffu, ok);
+                    if (!ok) break;
+                    const LinDesc L = a.lins[it.l];
+                    const int m0 = it.rt * kTileM;
+                    const uint32_t bbase = smem_u32(sBcat + (size_t)bb * BcBytes);
+                    const int groups = a.Kp / 8;
+                    const int total = kTileM * groups;         // (row, 8-column group) pairs
+                    for (int id0 = 0; id0 < total; id0 += 64 * 8) {
+                        uint4 v[8];
+                        float gs[8];
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) {
+                            const int id = id0 + u * 64 + tb;
+                            v[u] = make_uint4(0, 0, 0, 0);
+                            gs[u] = 0.f;
+                            if (id < total) {
+                                const int row = id / groups, cg = id - row * groups;
+                                const int c = cg * 8;
+                                const int s = c / a.r, j = c - s * a.r;
+                                const int o = m0 + row;
+                                if (s < a.ns && s_e[s] >= 0 && o < L.d_out) {
+                                    v[u] = ld_global_nc_v4(L.B + (int64_t)s_e[s] * L.b_es + (int64_t)o * a.r + j);
+                                    gs[u] = s_g[s];
+                                }
+                            }
+                        }
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) {
+                            const int id = id0 + u * 64 + tb;
+                            if (id < total) {
+                                const int row = id / groups, cg = id - row * groups;
+                                st_shared_v4(bbase + (uint32_t)(row >> 3) * 128u + (uint32_t)cg * 2048u + (uint32_t)(row & 7) * 16u,
+                                             scale_bf16x8(v[u], gs[u]));
+                            }
+                        }
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&bcfull[bb]);
+                }
+                if (i + 1 < count) it.next(a.lins, a.n_lin);
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int ew = warp - 4;
+        const int q = warp & 3;
+        const int h = ew >> 2;
+        const int row = q * 32 + lane;
+        RowTileIt it;
+        if (count > 0) it.init(a.lins, a.n_lin, t_begin);
+        int64_t stored = 0;
+        for (int64_t i = 0; i < count; ++i) {
+            const int acc = (int)(i & 1);
+            const int sw = (int)(i % a.SW);
+            bool ok = mbar_wait(&accfull[acc], (uint32_t)((i >> 1) & 1), abort_flag);
+            ok = ok && mbar_wait(&full[sw], (uint32_t)((i / a.SW) & 1), abort_flag);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+            tc_fence_after();
+            uint32_t va[32], vb[32];
+            const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)acc * kTileN + (uint32_t)h * 64u;
+            tc_ld_x32(taddr, va);
+            tc_ld_x32(taddr + 32u, vb);
+            tc_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&accempty[acc]);
+            uint8_t* slice = sStage + (size_t)sw * a.stage_bytes + (size_t)h * kWBoxBytes + (size_t)q * 32 * 128;
+            const uint32_t wrow = smem_u32(slice) + (uint32_t)lane * 128u;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                const uint32_t addr = wrow + ((uint32_t)(c ^ (row & 7)) << 4);
+                const uint4 w = ld_shared_v4(addr);
+                const uint32_t* dd = (c < 4) ? &va[c * 8] : &vb[(c - 4) * 8];
+                uint4 o;
+                o.x = add_bf16x2(w.x, dd[0], dd[1]);
+                o.y = add_bf16x2(w.y, dd[2], dd[3]);
+                o.z = add_bf16x2(w.z, dd[4], dd[5]);
+                o.w = add_bf16x2(w.w, dd[6], dd[7]);
+                st_shared_v4(addr, o);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                const CUtensorMap* mO = a.maps + (size_t)it.l * kMapsPerLinear + kMapWoutStore;
+                tma_store_2d(mO, slice, it.strip * kTileN + h * 64, it.rt * kTileM + q * 32);
+                bulk_commit_group();
+                bulk_wait_group_read<1>();
+                if (i > 0) mbar_arrive(&empty[(i - 1) % a.SW]);
+            }
+            stored = i + 1;
+            if (i + 1 < count) it.next(a.lins, a.n_lin);
+        }
+        if (lane == 0) {
+            bulk_wait_group<0>();
+            if (stored > 0) mbar_arrive(&empty[(stored - 1) % a.SW]);
+        }
+    }
+
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, 256);
+    }
+    if (threadIdx.x == 0 && *abort_flag) atomicOr(a.status, ADAFUSE_STATUS_TIMEOUT);
+}
+
 // ------------------------------------------------------------------ baseline
 
 // One launch per linear; each thread produces 8 consecutive outputs of a row
@@ -458,12 +769,33 @@ int launch_merge_fused(Plan* p, const int32_t* idx0, const float* gate0, const i
     a.ns = mode == 1 ? 2 * k : k;
     a.Kp = ((a.ns * p->r + 15) / 16) * 16;
     a.mode = mode;
-    a.stall = (p->flags & ADAFUSE_PLAN_TEST_STALL) ? 1 : 0;
     if (a.ns > kMaxSlots || a.Kp > kMaxKr) return ADAFUSE_ERR_UNSUPPORTED;
 
+    const uint32_t kSmemMax = 232448u;
+    a.stall = (p->flags & ADAFUSE_PLAN_TEST_STALL) ? 1 : 0;
+    a.box_rows = p->a_box_rows;
+    if (a.Kp <= 128) {
+        // Row-order kernel: stages of [W tile | A tile], two Bcat buffers.
+        const uint32_t stage = kWTileBytes + (uint32_t)a.Kp * 256u;
+        const uint32_t bc = (uint32_t)a.Kp * 256u;
+        int SW = std::min(4, (int)((kSmemMax - 2048u - 2u * bc) / stage));
+        if (SW >= 2) {
+            a.SW = SW; a.SB = 0; a.NA = 2;
+            a.stage_bytes = stage;
+            a.off_B = (uint32_t)SW * stage;
+            a.off_A = a.off_B;
+            a.off_bar = a.off_B + 2u * bc;
+            const uint32_t smem = a.off_bar + 1024u + 1024u;
+            if (cudaFuncSetAttribute(merge_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+                return ADAFUSE_ERR_CUDA;
+            const int grid = (int)std::min<int64_t>(p->num_sms, p->merge_tiles);
+            merge_rows_kernel<<<grid, kMergeThreads, smem, s>>>(a);
+            p->last_launches = 1;
+            return cuda_err(cudaGetLastError());
+        }
+    }
     const uint32_t BBytes = (uint32_t)a.Kp * 256u;
-    const uint32_t ABytes = BBytes;
-    const uint32_t kSmemMax = 232448u;                  // 227 KB opt-in per block
+    const uint32_t ABytes = BBytes;                  // 227 KB opt-in per block
     const uint32_t extra = 1024u /*alignment*/ + 1024u /*barriers, slots*/;
     int NA = 2, SB = 2, SW = 0;
     auto fits = [&](int sw, int sb, int na) {
