@@ -40,7 +40,10 @@ __device__ __forceinline__ bool ranks_before(int c1, float z1, int e1, int c0, f
     return e1 < e0;
 }
 
-__host__ __device__ constexpr int stage_floats(int E) { return E * (kChunk + 1) + kChunk; }
+// W_r rows in a stage are padded to kChunk + 4 floats: 16-byte aligned for
+// vector reads, and lane e's reads start 4 banks after lane e-1's.
+constexpr int kRowPad = kChunk + 4;
+__host__ __device__ constexpr int stage_floats(int E) { return E * kRowPad + kChunk; }
 
 __global__ void __launch_bounds__(kRouterThreads) pregate_kernel(const uint16_t* x, int64_t T, int32_t H,
                                                                   int64_t ldx, const float* Wr, const float* br,
@@ -62,14 +65,14 @@ __global__ void __launch_bounds__(kRouterThreads) pregate_kernel(const uint16_t*
             const int n = min(kChunk, H - j0);
             for (int id = tid; id < E * kChunk; id += kRouterThreads) {
                 const int e = id / kChunk, jj = id - e * kChunk;
-                if (jj < n) cp_async_4(smem_u32(ws + e * (kChunk + 1) + jj), Wr + (int64_t)e * H + j0 + jj);
+                if (jj < n) cp_async_4(smem_u32(ws + e * kRowPad + jj), Wr + (int64_t)e * H + j0 + jj);
             }
         }
         asm volatile("cp.async.commit_group;" ::: "memory");
     };
     // x (or the column means of x) for chunk c -> stage buffer, threads t0.. step nt.
     auto load_x = [&](int c, int t0, int nt) {
-        float* xs = rsm + (c % kStages) * SF + E * (kChunk + 1);
+        float* xs = rsm + (c % kStages) * SF + E * kRowPad;
         const int j0 = c * kChunk;
         for (int jj = t0; jj < kChunk; jj += nt) {
             const int j = j0 + jj;
@@ -96,10 +99,27 @@ __global__ void __launch_bounds__(kRouterThreads) pregate_kernel(const uint16_t*
         __syncthreads();                       // chunk c is in shared memory
         if (warp == 0) {
             if (lane < E) {
-                const float* ws = rsm + (c % kStages) * SF + lane * (kChunk + 1);
-                const float* xs = rsm + (c % kStages) * SF + E * (kChunk + 1);
+                const float* ws = rsm + (c % kStages) * SF + lane * kRowPad;
+                const float* xs = rsm + (c % kStages) * SF + E * kRowPad;
                 const int n = min(kChunk, H - c * kChunk);
-                for (int jj = 0; jj < n; ++jj) z = __fadd_rn(z, __fmul_rn(xs[jj], ws[jj]));
+                const int n4 = n & ~15;
+                // Same order as the scalar loop: one product, one add, ascending j.
+                for (int jj = 0; jj < n4; jj += 16) {
+                    float4 xv[4], wv[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        xv[u] = *reinterpret_cast<const float4*>(xs + jj + 4 * u);
+                        wv[u] = *reinterpret_cast<const float4*>(ws + jj + 4 * u);
+                    }
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        z = __fadd_rn(z, __fmul_rn(xv[u].x, wv[u].x));
+                        z = __fadd_rn(z, __fmul_rn(xv[u].y, wv[u].y));
+                        z = __fadd_rn(z, __fmul_rn(xv[u].z, wv[u].z));
+                        z = __fadd_rn(z, __fmul_rn(xv[u].w, wv[u].w));
+                    }
+                }
+                for (int jj = n4; jj < n; ++jj) z = __fadd_rn(z, __fmul_rn(xs[jj], ws[jj]));
             }
         } else if (c + 1 < nchunks) {
             load_x(c + 1, tid - 32, kRouterThreads - 32);
