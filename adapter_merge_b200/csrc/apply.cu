@@ -5,19 +5,24 @@
 // section 2.B); the pages print no formula for the unmerged form, so it is the
 // plain mixed-batch LoRA product above, per token with that token's top-k.
 //
-// Three launches per call, independent of the number of layers:
+// Four launches per call, independent of the number of layers:
 //   1. segments  stable sort of the (token, slot) pairs by expert (segments.cu);
-//   2. shrink    for every (linear, used expert): the expert's segment of tokens
-//                times A_e^T, gate-scaled, rounded to bf16 into
-//                S_l[T, U*r] (column block q = the q-th used expert);
-//   3. apply     one persistent tcgen05 kernel over all (linear, 128-row) units:
-//                D[128 x Npad] = W_tile x^T (d_in/64 swizzled K chunks) then
-//                + Bcat_tile S^T (the used experts' B rows, gathered by TMA),
-//                all into one fp32 TMEM accumulator, then y = bf16(D^T).
-// Every operand moves by TMA: W and the experts' B rows through the plan's
-// tensor maps, x and S through per-call maps that the host builds (and caches
-// by pointer set, T and workspace) before the launches.  W is streamed exactly
-// once per token tile; the x and S tiles come from L2.
+//                gives the U experts the batch uses;
+//   2. shrink    the used experts' stacked A rows times x_l^T on the tensor
+//                cores, in 1024-column K-slices, fp32 partials to the workspace;
+//   3. finalize  slices summed in order, times each token's gate on that
+//                expert, stored as a bf16 hi/lo pair S_l[T, 2 * Kext];
+//   4. apply     one persistent tcgen05 kernel over all (linear, row block)
+//                units: D[rows x Npad] = W_block x^T (d_in/64 swizzled K chunks)
+//                then + Bcat_block S^T (the used experts' B rows, gathered by
+//                TMA, against both halves of S), all into one fp32 TMEM
+//                accumulator, then y = bf16(D^T).  A unit covers 128, 256 or
+//                512 output rows (taller for smaller T), whose MMAs share each
+//                staged x chunk.
+// Every operand moves by TMA: W and the experts' A and B rows through the
+// plan's tensor maps, x and S through per-call maps that the host builds (and
+// caches by pointer set, T and workspace) before the launches.  W is streamed
+// exactly once per token tile; the x and S tiles come from L2.
 #include <cudaTypedefs.h>
 
 #include <algorithm>
@@ -36,8 +41,14 @@ namespace {
 struct WsLayout {
     size_t off_offsets, off_used, off_perm, off_S, off_P, total;
     int32_t Umax, Kext, Mt, Npad, n_tt;
+    int32_t shape, tile;    // apply units of 128 << shape rows; tokens per tile
     int64_t n_su;           // shrink units per token tile: Mt x total K-slices
 };
+
+// Unit height for a batch of T tokens.  A taller unit issues more MMAs per x
+// chunk it stages; its token tile (256 >> shape) must still cover T, or W is
+// streamed once per extra tile.
+int apply_shape(int64_t T) { return T <= 64 ? 2 : T <= 128 ? 1 : 0; }
 
 WsLayout ws_layout(const Plan* p, int64_t T, int32_t k)
 {
@@ -46,8 +57,10 @@ WsLayout ws_layout(const Plan* p, int64_t T, int32_t k)
     w.Umax = (int32_t)std::min<int64_t>(p->E, P);
     w.Kext = ((w.Umax * p->r + 63) / 64) * 64;
     w.Mt = (w.Umax * p->r + kTileM - 1) / kTileM;
-    w.Npad = (int32_t)std::min<int64_t>(kApplyMaxN, ((T + 15) / 16) * 16);
-    w.n_tt = (int32_t)((T + kApplyMaxN - 1) / kApplyMaxN);
+    w.shape = apply_shape(T);
+    w.tile = 256 >> w.shape;
+    w.Npad = (int32_t)std::min<int64_t>(w.tile, ((T + 15) / 16) * 16);
+    w.n_tt = (int32_t)((T + w.tile - 1) / w.tile);
     w.n_su = (int64_t)w.Mt * p->total_ks;
     auto up = [](size_t b) { return ((b + 255) / 256) * 256; };
     w.off_offsets = 0;
@@ -87,7 +100,7 @@ struct ShrinkArgs {
     float* P;
     int32_t* status;
     int64_t n_su;
-    int32_t n_lin, r, Npad, n_tt, total_ks;
+    int32_t n_lin, r, Npad, n_tt, total_ks, tile;
     int32_t ST, box_rows;
     uint32_t stage_bytes, off_bar, acc_stride, tmem_cols;
 };
@@ -180,7 +193,7 @@ __global__ void __launch_bounds__(kShrinkThreads, 1) shrink_tc_kernel(const __gr
                         const int qq = c / a.r, j0 = c - qq * a.r;
                         tma_load_3d(dst + (size_t)g * R * 128u, mA, &full[s], col, j0, s_used[1 + qq]);
                     }
-                    tma_load_2d(dst + kAChunkBytes, mX, &full[s], col, tt * kApplyMaxN);
+                    tma_load_2d(dst + kAChunkBytes, mX, &full[s], col, tt * a.tile);
                     issued = gc + 1;
                 }
             }
@@ -275,7 +288,8 @@ __global__ void __launch_bounds__(kShrinkThreads, 1) shrink_tc_kernel(const __gr
 __global__ void __launch_bounds__(128) shrink_finalize_kernel(const LinDesc* lins, const float* P, const int32_t* used,
                                                                const int32_t* idx, const float* gate, uint16_t* S,
                                                                int64_t T, int32_t k, int32_t r, int32_t Kext,
-                                                               int32_t Npad, int64_t n_su, int32_t total_ks)
+                                                               int32_t Npad, int32_t tile, int64_t n_su,
+                                                               int32_t total_ks)
 {
     __shared__ int s_used[kMaxE + 1];
     __shared__ int s_idx[kMaxSlots];
@@ -287,7 +301,7 @@ __global__ void __launch_bounds__(128) shrink_finalize_kernel(const LinDesc* lin
     __syncthreads();
     const int rows = s_used[0] * r;
     const int ks_base = __ldg(&lins[l].ks_base), n_ks = __ldg(&lins[l].n_ks);
-    const int tt = (int)(t / kApplyMaxN), tl = (int)(t - (int64_t)tt * kApplyMaxN);
+    const int tt = (int)(t / tile), tl = (int)(t - (int64_t)tt * tile);
     uint16_t* Srow = S + ((int64_t)l * T + t) * (2 * Kext);
     for (int c = threadIdx.x; c < Kext; c += blockDim.x) {
         float v = 0.f;
@@ -317,17 +331,19 @@ struct ApplyArgs {
     const CUtensorMap* xmaps;       // per call: x_l maps [n_lin], then the shrink-output map
     uint16_t* const* y_ptrs;        // per call, device table
     const int32_t* used;
-    const int2* order;              // units (linear, 128-row tile), longest first
+    const int2* order;              // units (linear, row block), longest first
     int32_t* sched;                 // [0] next unit, [1] CTAs finished (both back to 0 at exit)
     int32_t* status;
     int64_t T;
-    int32_t n_lin, r, Npad, n_tt, n_units, Kext;
+    int32_t n_lin, r, Npad, n_tt, n_units, Kext, tile;
     int32_t ST;
     uint32_t stage_bytes, off_bar, acc_stride, tmem_cols;
 };
 
-constexpr int kApplyThreads = 192;
-constexpr int kApplyEpiWarps = 4;
+template <int H> struct ApplyShape {
+    static constexpr int kEpiWarps = 4 * H;         // four per 128-row block
+    static constexpr int kThreads = 64 + 32 * kEpiWarps;
+};
 constexpr int kUnitRing = 4;
 
 // Last CTA out puts the work counters back to zero for the next launch.
@@ -342,15 +358,21 @@ __device__ __forceinline__ void release_counters(int32_t* sched)
 }
 
 // Warp roles: 0 = TMA producer and work fetcher, 1 = TMEM owner and MMA
-// issuer, 2-5 = epilogue.  Units are fetched from a global counter (longest
-// first), so SMs that stream faster take more of them; the producer passes
-// each unit id to the other roles through a small ring in shared memory.
-// Stage s holds a 128 x 64 A-operand chunk (W rows, or the used experts' B
-// rows) and an Npad x 64 B-operand chunk (x rows, or shrink-output rows), both
-// K-major; W and x use the 128-byte swizzle, B rows the plain core-matrix
-// layout.
-__global__ void __launch_bounds__(kApplyThreads, 1) apply_fused_kernel(const __grid_constant__ ApplyArgs a)
+// issuer, 2.. = epilogue (four warps per 128-row block).  Units are fetched
+// from a global counter (longest first), so SMs that stream faster take more of
+// them; the producer passes each unit id to the other roles through a small
+// ring in shared memory.  A unit covers H blocks of 128 output rows.  Stage s
+// holds H 128 x 64 A-operand chunks (W rows, or the used experts' B rows) and
+// one Npad x 64 B-operand chunk (x rows, or shrink-output rows) that the H
+// MMAs share, all K-major; W and x use the 128-byte swizzle, B rows the plain
+// core-matrix layout.  Block h accumulates in TMEM columns [h*Npad, (h+1)*Npad)
+// of the unit's accumulator.
+template <int H>
+__global__ void __launch_bounds__(ApplyShape<H>::kThreads, 1) apply_fused_kernel(const __grid_constant__ ApplyArgs a)
 {
+    constexpr int kApplyEpiWarps = ApplyShape<H>::kEpiWarps;
+    constexpr int kApplyThreads = ApplyShape<H>::kThreads;
+    constexpr int kApplyRows = kTileM * H;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* full = reinterpret_cast<uint64_t*>(base + a.off_bar);
@@ -377,7 +399,7 @@ __global__ void __launch_bounds__(kApplyThreads, 1) apply_fused_kernel(const __g
     if (threadIdx.x <= kMaxE) s_used[threadIdx.x] = a.used[threadIdx.x];
     // Zero the A regions: expert chunks load only the 8-column groups they use.
     for (int s = 0; s < a.ST; ++s)
-        for (uint32_t o = threadIdx.x * 16; o < kAChunkBytes; o += kApplyThreads * 16)
+        for (uint32_t o = threadIdx.x * 16; o < kAChunkBytes * H; o += kApplyThreads * 16)
             st_shared_v4(smem_u32(base + (size_t)s * a.stage_bytes + o), make_uint4(0, 0, 0, 0));
     fence_proxy_async_smem();
     __syncthreads();
@@ -414,8 +436,8 @@ __global__ void __launch_bounds__(kApplyThreads, 1) apply_fused_kernel(const __g
                 const int2 lm = a.order[u - tt * a.n_units];
                 const int l = lm.x;
                 const int nKb = (__ldg(&a.lins[l].d_in) + kChunkK - 1) / kChunkK;
-                const int m0 = lm.y * kTileM;
-                const int t0 = tt * kApplyMaxN;
+                const int m0 = lm.y * kApplyRows;
+                const int t0 = tt * a.tile;
                 const CUtensorMap* mW = a.maps + (size_t)l * kMapsPerLinear + kMapW;
                 const CUtensorMap* mB = a.maps + (size_t)l * kMapsPerLinear + kMapB;
                 const CUtensorMap* mX = a.xmaps + l;
@@ -425,9 +447,10 @@ __global__ void __launch_bounds__(kApplyThreads, 1) apply_fused_kernel(const __g
                     if (!mbar_wait(&empty[s], (uint32_t)((gc / a.ST) & 1) ^ 1u, abort_flag)) { stop = true; break; }
                     uint8_t* dst = base + (size_t)s * a.stage_bytes;
                     if (kc < nKb) {
-                        mbar_arrive_expect_tx(&full[s], kAChunkBytes + xbytes);
-                        tma_load_2d(dst, mW, &full[s], kc * kChunkK, m0);
-                        tma_load_2d(dst + kAChunkBytes, mX, &full[s], kc * kChunkK, t0);
+                        mbar_arrive_expect_tx(&full[s], kAChunkBytes * H + xbytes);
+                        for (int hh = 0; hh < H; ++hh)
+                            tma_load_2d(dst + hh * kAChunkBytes, mW, &full[s], kc * kChunkK, m0 + hh * kTileM);
+                        tma_load_2d(dst + kAChunkBytes * H, mX, &full[s], kc * kChunkK, t0);
                     } else {
                         // expand: the hi half of S, then the lo half, each
                         // against the same B rows of the used experts
@@ -436,13 +459,15 @@ __global__ void __launch_bounds__(kApplyThreads, 1) apply_fused_kernel(const __g
                         const int col0 = (ke - half * nKh) * kChunkK;
                         int ng = 0;
                         for (int g = 0; g < 8; ++g) if (col0 + g * 8 < U * a.r) ++ng;
-                        mbar_arrive_expect_tx(&full[s], (uint32_t)ng * 2048u + xbytes);
-                        for (int g = 0; g < ng; ++g) {
-                            const int c = col0 + g * 8;
-                            const int qq = c / a.r, j0 = c - qq * a.r;
-                            tma_load_3d(dst + (size_t)g * 2048u, mB, &full[s], j0, m0, s_used[1 + qq]);
-                        }
-                        tma_load_3d(dst + kAChunkBytes, mS, &full[s], half * a.Kext + col0, t0, l);
+                        mbar_arrive_expect_tx(&full[s], (uint32_t)(ng * H) * 2048u + xbytes);
+                        for (int hh = 0; hh < H; ++hh)
+                            for (int g = 0; g < ng; ++g) {
+                                const int c = col0 + g * 8;
+                                const int qq = c / a.r, j0 = c - qq * a.r;
+                                tma_load_3d(dst + hh * kAChunkBytes + (size_t)g * 2048u, mB, &full[s], j0,
+                                            m0 + hh * kTileM, s_used[1 + qq]);
+                            }
+                        tma_load_3d(dst + kAChunkBytes * H, mS, &full[s], half * a.Kext + col0, t0, l);
                     }
                     issued = gc + 1;
                 }
@@ -474,15 +499,19 @@ __global__ void __launch_bounds__(kApplyThreads, 1) apply_fused_kernel(const __g
                     const int s = (int)(gc % a.ST);
                     if (!mbar_wait(&full[s], (uint32_t)((gc / a.ST) & 1), abort_flag)) { stop = true; break; }
                     tc_fence_after();
-                    const uint32_t aaddr = smem_u32(base + (size_t)s * a.stage_bytes);
-                    const uint32_t baddr = aaddr + kAChunkBytes;
+                    const uint32_t abase = smem_u32(base + (size_t)s * a.stage_bytes);
+                    const uint32_t baddr = abase + kAChunkBytes * H;
 #pragma unroll
-                    for (int kk = 0; kk < kChunkK / 16; ++kk) {
-                        const uint64_t adesc = (kc < nKb)
-                            ? make_sdesc(aaddr + (uint32_t)kk * 32u, 16u, 1024u, kLayoutSw128)
-                            : make_sdesc(aaddr + (uint32_t)kk * 4096u, 2048u, 128u, kLayoutNone);
-                        const uint64_t bdesc = make_sdesc(baddr + (uint32_t)kk * 32u, 16u, 1024u, kLayoutSw128);
-                        tc_mma_bf16(d, adesc, bdesc, idesc, (kc | kk) ? 1u : 0u);
+                    for (int hh = 0; hh < H; ++hh) {
+                        const uint32_t aaddr = abase + hh * kAChunkBytes;
+#pragma unroll
+                        for (int kk = 0; kk < kChunkK / 16; ++kk) {
+                            const uint64_t adesc = (kc < nKb)
+                                ? make_sdesc(aaddr + (uint32_t)kk * 32u, 16u, 1024u, kLayoutSw128)
+                                : make_sdesc(aaddr + (uint32_t)kk * 4096u, 2048u, 128u, kLayoutNone);
+                            const uint64_t bdesc = make_sdesc(baddr + (uint32_t)kk * 32u, 16u, 1024u, kLayoutSw128);
+                            tc_mma_bf16(d + (uint32_t)(hh * a.Npad), adesc, bdesc, idesc, (kc | kk) ? 1u : 0u);
+                        }
                     }
                     tc_commit(&empty[s]);
                 }
@@ -496,6 +525,7 @@ __global__ void __launch_bounds__(kApplyThreads, 1) apply_fused_kernel(const __g
     } else {
         // ------------------------------------------------------------ epilogue
         const int q = warp & 3;        // TMEM lane quarter: warps 2,3,4,5 -> 2,3,0,1
+        const int hh = (warp - 2) >> 2;                        // which 128-row half
         for (int ui = 0;; ++ui) {
             const int j = ui & (kUnitRing - 1);
             bool ok = mbar_wait(&ufull[j], (uint32_t)((ui / kUnitRing) & 1), abort_flag);
@@ -513,8 +543,9 @@ __global__ void __launch_bounds__(kApplyThreads, 1) apply_fused_kernel(const __g
             const int d_out = __ldg(&a.lins[lm.x].d_out);
             uint16_t* y = a.y_ptrs[lm.x];
             const int64_t T = a.T;
-            const int row = lm.y * kTileM + q * 32 + lane;
-            const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)acc * a.acc_stride;
+            const int row = lm.y * kApplyRows + hh * kTileM + q * 32 + lane;
+            const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)acc * a.acc_stride +
+                                   (uint32_t)(hh * a.Npad);
             for (int c0 = 0; c0 < a.Npad; c0 += 32) {
                 uint32_t v[32];
                 if (a.Npad - c0 >= 32) {
@@ -527,7 +558,7 @@ __global__ void __launch_bounds__(kApplyThreads, 1) apply_fused_kernel(const __g
                 }
                 tc_wait_ld();
                 if (row < d_out) {
-                    const int64_t t0 = (int64_t)tt * kApplyMaxN + c0;
+                    const int64_t t0 = (int64_t)tt * a.tile + c0;
                     uint16_t* yp = y + t0 * d_out + row;
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
@@ -571,6 +602,110 @@ bool encode_tile_map(CUtensorMap* m, const void* ptr, int rank, const cuuint64_t
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+
+// The four launches of one apply call: segments, shrink, finalize, and the
+// fused base + expand kernel.  `xmaps` holds the call's x maps and then the
+// shrink-output map, `yp` is the device table of output pointers and `wsb` the
+// workspace laid out by `w`.
+template <int H>
+int launch_apply_fused(const ApplyArgs& a, uint32_t smem, int grid, cudaStream_t s)
+{
+    if (cudaFuncSetAttribute(apply_fused_kernel<H>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
+        return ADAFUSE_ERR_CUDA;
+    apply_fused_kernel<H><<<grid, ApplyShape<H>::kThreads, smem, s>>>(a);
+    return cuda_err(cudaGetLastError());
+}
+
+int launch_apply_kernels(Plan* p, const WsLayout& w, uint8_t* wsb, const CUtensorMap* xmaps, void* const* yp,
+                         const int32_t* idx, const float* gate, int64_t T, int32_t k, cudaStream_t s)
+{
+    int32_t* offsets = reinterpret_cast<int32_t*>(wsb + w.off_offsets);
+    int32_t* used = reinterpret_cast<int32_t*>(wsb + w.off_used);
+    int32_t* perm = reinterpret_cast<int32_t*>(wsb + w.off_perm);
+    uint16_t* S = reinterpret_cast<uint16_t*>(wsb + w.off_S);
+    float* P = reinterpret_cast<float*>(wsb + w.off_P);
+    const int32_t Npad = w.Npad;
+    const int H = 1 << w.shape;
+    const uint32_t kSmemMax = 232448u;
+
+    int rc = launch_segments(idx, T, k, p->E, offsets, perm, used, p->d_status, s);
+    if (rc != ADAFUSE_OK) return rc;
+
+    {
+        uint32_t accs = 32;
+        while (accs < (uint32_t)Npad) accs <<= 1;
+        const uint32_t stage_bytes = kAChunkBytes + (uint32_t)Npad * 128u;
+        const int ST = std::min(8, (int)((kSmemMax - 2048u) / stage_bytes));
+        if (ST < 2 || 2 * accs > 512) return ADAFUSE_ERR_UNSUPPORTED;
+        const uint32_t smem = (uint32_t)ST * stage_bytes + 1024u + 1024u;
+        ShrinkArgs sa{};
+        sa.lins = p->d_desc;
+        sa.maps = p->d_maps;
+        sa.xmaps = xmaps;
+        sa.used = used;
+        sa.P = P;
+        sa.status = p->d_status;
+        sa.n_su = w.n_su;
+        sa.n_lin = p->n_lin;
+        sa.r = p->r;
+        sa.Npad = Npad;
+        sa.n_tt = w.n_tt;
+        sa.total_ks = p->total_ks;
+        sa.tile = w.tile;
+        sa.ST = ST;
+        sa.box_rows = p->a_box_rows;
+        sa.stage_bytes = stage_bytes;
+        sa.off_bar = (uint32_t)ST * stage_bytes;
+        sa.acc_stride = accs;
+        sa.tmem_cols = 2 * accs;
+        if (cudaFuncSetAttribute(shrink_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+            cudaSuccess)
+            return ADAFUSE_ERR_CUDA;
+        shrink_tc_kernel<<<(int)std::min<int64_t>(p->num_sms, w.n_su * w.n_tt), kShrinkThreads, smem, s>>>(sa);
+        if (cudaGetLastError() != cudaSuccess) return ADAFUSE_ERR_CUDA;
+        shrink_finalize_kernel<<<dim3((unsigned)p->n_lin, (unsigned)T), 128, 0, s>>>(
+            p->d_desc, P, used, idx, gate, S, T, k, p->r, w.Kext, Npad, w.tile, w.n_su, p->total_ks);
+        if (cudaGetLastError() != cudaSuccess) return ADAFUSE_ERR_CUDA;
+    }
+
+    // Accumulators: two of H * Npad columns (Npad <= 256 / H).
+    uint32_t accs = 32;
+    while (accs < (uint32_t)(Npad * H)) accs <<= 1;
+    const uint32_t stage_bytes = kAChunkBytes * H + (uint32_t)Npad * 128u;
+    const int ST = std::min(8, (int)((kSmemMax - 2048u) / stage_bytes));
+    if (ST < 2 || 2 * accs > 512) return ADAFUSE_ERR_UNSUPPORTED;
+    const uint32_t smem = (uint32_t)ST * stage_bytes + 1024u + 1024u;
+    ApplyArgs a{};
+    a.lins = p->d_desc;
+    a.maps = p->d_maps;
+    a.xmaps = xmaps;
+    a.y_ptrs = reinterpret_cast<uint16_t* const*>(yp);
+    a.used = used;
+    a.order = p->d_apply_order[w.shape];
+    a.sched = p->d_sched;
+    a.n_units = (int32_t)p->apply_units[w.shape];
+    a.Kext = w.Kext;
+    a.tile = w.tile;
+    a.status = p->d_status;
+    a.T = T;
+    a.n_lin = p->n_lin;
+    a.r = p->r;
+    a.n_tt = w.n_tt;
+    a.Npad = Npad;
+    a.stage_bytes = stage_bytes;
+    a.acc_stride = accs;
+    a.tmem_cols = 2 * accs;
+    a.ST = ST;
+    a.off_bar = (uint32_t)ST * stage_bytes;
+    const int grid = (int)std::min<int64_t>(p->num_sms, (int64_t)a.n_units * a.n_tt);
+    p->last_launches = 4;
+    switch (H) {
+    case 1: return launch_apply_fused<1>(a, smem, grid, s);
+    case 2: return launch_apply_fused<2>(a, smem, grid, s);
+    default: return launch_apply_fused<4>(a, smem, grid, s);
+    }
+}
 }  // namespace
 
 size_t apply_workspace_bytes(const Plan* p, int64_t T, int32_t k)
@@ -594,9 +729,6 @@ int launch_apply(Plan* p, const void* const* x_ptrs, void* const* y_ptrs, int64_
             return ADAFUSE_ERR_UNSUPPORTED;
     }
     uint8_t* wsb = static_cast<uint8_t*>(ws);
-    int32_t* offsets = reinterpret_cast<int32_t*>(wsb + w.off_offsets);
-    int32_t* used = reinterpret_cast<int32_t*>(wsb + w.off_used);
-    int32_t* perm = reinterpret_cast<int32_t*>(wsb + w.off_perm);
     uint16_t* S = reinterpret_cast<uint16_t*>(wsb + w.off_S);
     const int32_t Npad = w.Npad;
 
@@ -637,74 +769,7 @@ int launch_apply(Plan* p, const void* const* x_ptrs, void* const* y_ptrs, int64_
         p->call_y.assign(y_ptrs, y_ptrs + p->n_lin);
     }
 
-    int rc = launch_segments(idx, T, k, p->E, offsets, perm, used, p->d_status, s);
-    if (rc != ADAFUSE_OK) return rc;
-
-    uint32_t accs = 32;
-    while (accs < (uint32_t)Npad) accs <<= 1;
-    const uint32_t stage_bytes = kAChunkBytes + (uint32_t)Npad * 128u;
-    const uint32_t kSmemMax = 232448u;
-    int ST = std::min(8, (int)((kSmemMax - 2048u) / stage_bytes));
-    if (ST < 2) return ADAFUSE_ERR_UNSUPPORTED;
-    const uint32_t smem = (uint32_t)ST * stage_bytes + 1024u + 1024u;
-
-    {
-        ShrinkArgs sa{};
-        sa.lins = p->d_desc;
-        sa.maps = p->d_maps;
-        sa.xmaps = d_maps;
-        sa.used = used;
-        sa.P = reinterpret_cast<float*>(wsb + w.off_P);
-        sa.status = p->d_status;
-        sa.n_su = w.n_su;
-        sa.n_lin = p->n_lin;
-        sa.r = p->r;
-        sa.Npad = Npad;
-        sa.n_tt = w.n_tt;
-        sa.total_ks = p->total_ks;
-        sa.ST = ST;
-        sa.box_rows = p->a_box_rows;
-        sa.stage_bytes = stage_bytes;
-        sa.off_bar = (uint32_t)ST * stage_bytes;
-        sa.acc_stride = accs;
-        sa.tmem_cols = 2 * accs;
-        if (cudaFuncSetAttribute(shrink_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-            return ADAFUSE_ERR_CUDA;
-        const int64_t units = w.n_su * w.n_tt;
-        const int grid = (int)std::min<int64_t>(p->num_sms, units);
-        shrink_tc_kernel<<<grid, kShrinkThreads, smem, s>>>(sa);
-        if (cudaGetLastError() != cudaSuccess) return ADAFUSE_ERR_CUDA;
-        shrink_finalize_kernel<<<dim3((unsigned)p->n_lin, (unsigned)T), 128, 0, s>>>(
-            p->d_desc, sa.P, used, idx, gate, S, T, k, p->r, w.Kext, Npad, w.n_su, p->total_ks);
-        if (cudaGetLastError() != cudaSuccess) return ADAFUSE_ERR_CUDA;
-    }
-
-    ApplyArgs a{};
-    a.lins = p->d_desc;
-    a.maps = p->d_maps;
-    a.xmaps = d_maps;
-    a.y_ptrs = reinterpret_cast<uint16_t* const*>(d_yp);
-    a.used = used;
-    a.order = p->d_apply_order;
-    a.sched = p->d_sched;
-    a.n_units = (int32_t)p->apply_units;
-    a.Kext = w.Kext;
-    a.status = p->d_status;
-    a.T = T;
-    a.n_lin = p->n_lin;
-    a.r = p->r;
-    a.n_tt = w.n_tt;
-    a.Npad = Npad;
-    a.stage_bytes = stage_bytes;
-    a.acc_stride = accs;
-    a.tmem_cols = 2 * accs;
-    a.ST = ST;
-    a.off_bar = (uint32_t)ST * stage_bytes;
-    if (cudaFuncSetAttribute(apply_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-        return ADAFUSE_ERR_CUDA;
-    apply_fused_kernel<<<(int)std::min<int64_t>(p->num_sms, (int64_t)a.n_units * a.n_tt), kApplyThreads, smem, s>>>(a);
-    p->last_launches = 4;
-    return cuda_err(cudaGetLastError());
+    return launch_apply_kernels(p, w, wsb, d_maps, d_yp, idx, gate, T, k, s);
 }
 
 }  // namespace af
@@ -770,11 +835,7 @@ int launch_apply_noalloc(Plan* p, const void* const* x_ptrs, void* const* y_ptrs
     CUtensorMap* d_maps = reinterpret_cast<CUtensorMap*>(d_desc);
     void* const* d_yp = reinterpret_cast<void* const*>(d_desc + (size_t)(p->n_lin + 1) * sizeof(CUtensorMap));
     uint8_t* wsb = d_desc + desc_bytes;
-    int32_t* offsets = reinterpret_cast<int32_t*>(wsb + w.off_offsets);
-    int32_t* used = reinterpret_cast<int32_t*>(wsb + w.off_used);
-    int32_t* perm = reinterpret_cast<int32_t*>(wsb + w.off_perm);
     uint16_t* S = reinterpret_cast<uint16_t*>(wsb + w.off_S);
-    float* P = reinterpret_cast<float*>(wsb + w.off_P);
     const int32_t Npad = w.Npad;
 
     // Descriptors for this call, staged in a static host buffer (no heap) under
@@ -801,70 +862,7 @@ int launch_apply_noalloc(Plan* p, const void* const* x_ptrs, void* const* y_ptrs
     if (cudaMemcpyAsync(d_desc, stage, map_bytes + sizeof(void*) * p->n_lin, cudaMemcpyHostToDevice, s) != cudaSuccess)
         return ADAFUSE_ERR_CUDA;
 
-    rc = launch_segments(idx, T, k, p->E, offsets, perm, used, p->d_status, s);
-    if (rc != ADAFUSE_OK) return rc;
-
-    uint32_t accs = 32;
-    while (accs < (uint32_t)Npad) accs <<= 1;
-    const uint32_t stage_bytes = kAChunkBytes + (uint32_t)Npad * 128u;
-    const uint32_t kSmemMax = 232448u;
-    const int ST = std::min(8, (int)((kSmemMax - 2048u) / stage_bytes));
-    if (ST < 2) return ADAFUSE_ERR_UNSUPPORTED;
-    const uint32_t smem = (uint32_t)ST * stage_bytes + 1024u + 1024u;
-
-    ShrinkArgs sa{};
-    sa.lins = p->d_desc;
-    sa.maps = p->d_maps;
-    sa.xmaps = d_maps;
-    sa.used = used;
-    sa.P = P;
-    sa.status = p->d_status;
-    sa.n_su = w.n_su;
-    sa.n_lin = p->n_lin;
-    sa.r = p->r;
-    sa.Npad = Npad;
-    sa.n_tt = w.n_tt;
-    sa.total_ks = p->total_ks;
-    sa.ST = ST;
-    sa.box_rows = p->a_box_rows;
-    sa.stage_bytes = stage_bytes;
-    sa.off_bar = (uint32_t)ST * stage_bytes;
-    sa.acc_stride = accs;
-    sa.tmem_cols = 2 * accs;
-    if (cudaFuncSetAttribute(shrink_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-        return ADAFUSE_ERR_CUDA;
-    shrink_tc_kernel<<<(int)std::min<int64_t>(p->num_sms, w.n_su * w.n_tt), kShrinkThreads, smem, s>>>(sa);
-    if (cudaGetLastError() != cudaSuccess) return ADAFUSE_ERR_CUDA;
-    shrink_finalize_kernel<<<dim3((unsigned)p->n_lin, (unsigned)T), 128, 0, s>>>(
-        p->d_desc, P, used, idx, gate, S, T, k, p->r, w.Kext, Npad, w.n_su, p->total_ks);
-    if (cudaGetLastError() != cudaSuccess) return ADAFUSE_ERR_CUDA;
-
-    ApplyArgs a{};
-    a.lins = p->d_desc;
-    a.maps = p->d_maps;
-    a.xmaps = d_maps;
-    a.y_ptrs = reinterpret_cast<uint16_t* const*>(d_yp);
-    a.used = used;
-    a.order = p->d_apply_order;
-    a.sched = p->d_sched;
-    a.n_units = (int32_t)p->apply_units;
-    a.Kext = w.Kext;
-    a.status = p->d_status;
-    a.T = T;
-    a.n_lin = p->n_lin;
-    a.r = p->r;
-    a.n_tt = w.n_tt;
-    a.Npad = Npad;
-    a.stage_bytes = stage_bytes;
-    a.acc_stride = accs;
-    a.tmem_cols = 2 * accs;
-    a.ST = ST;
-    a.off_bar = (uint32_t)ST * stage_bytes;
-    if (cudaFuncSetAttribute(apply_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-        return ADAFUSE_ERR_CUDA;
-    apply_fused_kernel<<<(int)std::min<int64_t>(p->num_sms, (int64_t)a.n_units * a.n_tt), kApplyThreads, smem, s>>>(a);
-    p->last_launches = 4;
-    return cuda_err(cudaGetLastError());
+    return launch_apply_kernels(p, w, wsb, d_maps, d_yp, idx, gate, T, k, s);
 }
 
 size_t apply_noalloc_limit_bytes() { return kNoAllocScratchBytes; }

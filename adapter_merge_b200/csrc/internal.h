@@ -42,7 +42,10 @@ constexpr int kChunkK = 64;      // apply: d_in per pipeline stage (one 128-byte
 constexpr int kMaxSlots = ADAFUSE_MAX_SLOTS;
 constexpr int kMaxKr = ADAFUSE_MAX_KR;
 constexpr int kMaxE = ADAFUSE_MAX_E;
-constexpr int kApplyMaxN = 256;  // tokens per apply tile (MMA N)
+// Apply units cover H = 1, 2 or 4 row blocks of 128 (the MMAs of a unit share
+// each x chunk); a unit of H blocks takes at most 256 / H tokens per tile, so
+// that its two accumulators fit the 512 TMEM columns.
+constexpr int kApplyShapes = 3;                   // H = 1 << shape
 
 struct Plan {
     int device = 0;
@@ -55,10 +58,10 @@ struct Plan {
     CUtensorMap* d_maps = nullptr;
     int32_t* d_status = nullptr;
     int64_t merge_tiles = 0;
-    int64_t apply_units = 0;
+    int64_t apply_units[kApplyShapes] = {};       // apply units for H = 1, 2, 4
     int32_t total_ks = 0;             // shrink K-slices over all linears
     int32_t a_box_rows = 8;           // rows per A-stack TMA box: largest power of two <= 128 dividing r
-    int2* d_apply_order = nullptr;      // apply units (linear, row tile), longest first
+    int2* d_apply_order[kApplyShapes] = {};      // apply units (linear, row block), longest first
     int32_t* d_sched = nullptr;         // work counters of the persistent kernels (zero between launches)
     int32_t last_launches = 0;
     // Per-call apply descriptors: TMA maps of every x_l and of the shrink

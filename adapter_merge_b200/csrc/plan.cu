@@ -73,7 +73,7 @@ void free_plan(Plan* p)
     if (p->d_desc) cudaFree(p->d_desc);
     if (p->d_maps) cudaFree(p->d_maps);
     if (p->d_status) cudaFree(p->d_status);
-    if (p->d_apply_order) cudaFree(p->d_apply_order);
+    for (int2* o : p->d_apply_order) if (o) cudaFree(o);
     if (p->d_sched) cudaFree(p->d_sched);
     if (p->d_call) cudaFree(p->d_call);
     delete static_cast<adafuse_plan*>(p);
@@ -154,28 +154,33 @@ extern "C" int adafuse_plan_create(adafuse_plan** out, const adafuse_linear* lin
     }
     if (units > 0x7fffffff) { free_plan(p); return ADAFUSE_ERR_UNSUPPORTED; }
     p->merge_tiles = tiles;
-    p->apply_units = units;
     p->total_ks = kslices;
 
-    // Apply units in decreasing order of the W bytes they stream (stable), so
-    // that dynamic scheduling ends with short units.
-    std::vector<int2> order;
-    order.reserve((size_t)units);
-    for (int l = 0; l < n_lin; ++l)
-        for (int m = 0; m < p->h_desc[l].n_rt; ++m) order.push_back(make_int2(l, m));
-    std::stable_sort(order.begin(), order.end(), [&](const int2& x, const int2& y) {
-        return p->h_desc[x.x].d_in > p->h_desc[y.x].d_in;
-    });
+    // Apply units, one list per unit height (H row blocks of 128), in
+    // decreasing order of the W bytes they stream (stable), so that dynamic
+    // scheduling ends with short units.
+    std::vector<int2> order[kApplyShapes];
+    for (int h = 0; h < kApplyShapes; ++h) {
+        const int rows = kTileM << h;
+        for (int l = 0; l < n_lin; ++l)
+            for (int m = 0; m < (p->h_desc[l].d_out + rows - 1) / rows; ++m) order[h].push_back(make_int2(l, m));
+        std::stable_sort(order[h].begin(), order[h].end(), [&](const int2& x, const int2& y) {
+            return p->h_desc[x.x].d_in > p->h_desc[y.x].d_in;
+        });
+        p->apply_units[h] = (int64_t)order[h].size();
+    }
 
     bool ok = cudaMalloc(&p->d_desc, sizeof(LinDesc) * n_lin) == cudaSuccess &&
               cudaMalloc(&p->d_maps, sizeof(CUtensorMap) * maps.size()) == cudaSuccess &&
               cudaMalloc(&p->d_status, sizeof(int32_t)) == cudaSuccess &&
-              cudaMalloc(&p->d_apply_order, sizeof(int2) * order.size()) == cudaSuccess &&
               cudaMalloc(&p->d_sched, sizeof(int32_t) * 8) == cudaSuccess &&
               cudaMalloc(&p->d_call, apply_call_bytes(n_lin)) == cudaSuccess;
+    for (int h = 0; h < kApplyShapes; ++h)
+        ok = ok && cudaMalloc(&p->d_apply_order[h], sizeof(int2) * order[h].size()) == cudaSuccess &&
+             cudaMemcpy(p->d_apply_order[h], order[h].data(), sizeof(int2) * order[h].size(),
+                        cudaMemcpyHostToDevice) == cudaSuccess;
     ok = ok && cudaMemcpy(p->d_desc, p->h_desc.data(), sizeof(LinDesc) * n_lin, cudaMemcpyHostToDevice) == cudaSuccess;
     ok = ok && cudaMemcpy(p->d_maps, maps.data(), sizeof(CUtensorMap) * maps.size(), cudaMemcpyHostToDevice) == cudaSuccess;
-    ok = ok && cudaMemcpy(p->d_apply_order, order.data(), sizeof(int2) * order.size(), cudaMemcpyHostToDevice) == cudaSuccess;
     ok = ok && cudaMemset(p->d_sched, 0, sizeof(int32_t) * 8) == cudaSuccess;
     ok = ok && cudaMemset(p->d_status, 0, sizeof(int32_t)) == cudaSuccess;
     ok = ok && cudaDeviceSynchronize() == cudaSuccess;

@@ -370,7 +370,7 @@ def main():
     mb = merge_bytes(cfg, cfg.k)
     traffic = None
     if cfg.name == "llama2-7b":
-        traffic = profiled_traffic(["merge.cu", "ptx.cuh", "internal.h"], "merge_fused_kernel_llama2-7b-2layer.md",
+        traffic = profiled_traffic(["merge.cu", "ptx.cuh", "internal.h"], "merge_rows_kernel_llama2-7b-2layer.md",
                                    "traffic_bytes_per_full_llama2_7b_launch")
     ab = apply_bytes(cfg, T, U)
     peak, peak_kind = read_peaks()
@@ -485,13 +485,13 @@ def main():
                       "gbs": round(apply_gbs, 2), "bytes": ab, "distinct_experts": U,
                       "frac_of_peak": round(apply_gbs / peak, 4),
                       "note": "call = segments + shrink + finalize + fused apply (4 launches)"},
-            "roofline": {"bound": "hbm", "kernel": "merge_fused_kernel", "achieved": round(kern_gbs, 2),
+            "roofline": {"bound": "hbm", "kernel": "merge_rows_kernel", "achieved": round(kern_gbs, 2),
                          "peak": peak, "unit": "GB/s", "frac": round(kern_gbs / peak, 4),
                          "peak_source": f"{peak_kind} hbm_gbs (burst copy)",
                          "algorithmic_bytes": mb,
                          "traffic": traffic,
                          "traffic_source": ("ncu dram bytes, 2-layer capture scaled by elements "
-                                            "(profiles/merge_fused_kernel_llama2-7b-2layer.md)") if traffic else None},
+                                            "(profiles/merge_rows_kernel_llama2-7b-2layer.md)") if traffic else None},
             "gpu_launches": 7 * args.steps,
             "clocks": clocks,
             "e2e": e2e,

@@ -212,8 +212,8 @@ ADAFUSE_API size_t adafuse_apply_workspace_bytes(const adafuse_plan* plan, int64
  * them (with the pointer tables) on `stream`; they are kept in the plan and
  * rebuilt only when the pointers, T or the workspace differ from the previous
  * call, so a serving loop that reuses its buffers does no host work beyond the
- * three launches.  Tokens are processed in tiles of 256; T larger than 256
- * streams W once per tile.  Each row of idx should hold distinct experts (as
+ * four launches.  Tokens are processed in tiles of 64 (T <= 64), 128
+ * (T <= 128) or 256 tokens; T larger than 256 streams W once per tile.  Each row of idx should hold distinct experts (as
  * pregate's does); a repeated expert adds its gates.
  * Errors: INVALID_ARG, WORKSPACE_TOO_SMALL, UNSUPPORTED (k < 1, k > E,
  * misaligned x_l).

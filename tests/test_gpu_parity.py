@@ -296,9 +296,11 @@ def test_apply_tiny_chain_with_pregate(am, cuda_device):
     assert m.plan.last_launches == 4
 
 
-@pytest.mark.parametrize("T", [1, 5, 16, 17, 64, 130, 256, 300])
+# T <= 64, 65..128 and > 128 take apply units of 512, 256 and 128 output rows;
+# d_out = 1000 leaves a last unit whose final 128-row block is all padding.
+@pytest.mark.parametrize("T", [1, 5, 16, 17, 64, 65, 128, 129, 130, 256, 300])
 def test_apply_token_counts(am, cuda_device, T):
-    cfg = synth.custom([(384, 520), (136, 72)], 6, 16, 2, T, name=f"aT{T}")
+    cfg = synth.custom([(384, 520), (136, 72), (1000, 264)], 6, 16, 2, T, name=f"aT{T}")
     m, xs, xs_dev, ys, xp, yp, idx, gate, ws = apply_setup(cfg, cuda_device, T)
     run_apply(m, xp, yp, T, idx, gate, ws, cuda_device)
     check_apply(m, xs, ys, idx.numpy(), gate.numpy().astype(np.float64), f"T={T}")
