@@ -182,8 +182,11 @@ def cpu_oracle_merge(cfg, target_s: float, nthreads: int):
     """(GB/s, seconds, sample) of the CPU oracle on about target_s of work."""
     smp = OracleMergeSample(cfg, nthreads)
     rows = smp.calibrate(target_s)
-    nb, dt = smp.run(rows)
-    return nb / dt / 1e9, dt, f"{rows} rows of each of q, gate, down (k=2, r=16)"
+    nb, dt, passes = 0, 0.0, 0
+    while passes == 0 or dt < target_s:
+        b, t = smp.run(rows)
+        nb, dt, passes = nb + b, dt + t, passes + 1
+    return nb / dt / 1e9, dt, f"{passes} x {rows} rows of each of q, gate, down (k=2, r=16)"
 
 
 def cpu_oracle_apply(cfg, target_s: float, nthreads: int):
@@ -200,17 +203,18 @@ def cpu_oracle_apply(cfg, target_s: float, nthreads: int):
     T = nthreads
     X, xs = synth.make_apply_inputs(sub, T, 0)
     idx, gate = synth.random_selection(T, cfg.E, cfg.k, 3)
-    t0 = time.perf_counter()
-    for i in range(len(picks)):
-        oracle.apply_linear(xs[i].view(torch.int16).numpy().view(np.uint16),
-                            w.W_views[i].view(torch.int16).numpy().view(np.uint16),
-                            w.A_views[i].view(torch.int16).numpy().view(np.uint16),
-                            w.B_views[i].view(torch.int16).numpy().view(np.uint16),
-                            idx.numpy(), gate.numpy().astype(np.float64), nthreads=nthreads)
-    dt = time.perf_counter() - t0
+    u = lambda t: t.view(torch.int16).numpy().view(np.uint16)
+    args = [(u(xs[i]), u(w.W_views[i]), u(w.A_views[i]), u(w.B_views[i])) for i in range(len(picks))]
+    dt, passes = 0.0, 0
+    while passes == 0 or dt < target_s:
+        t0 = time.perf_counter()
+        for a in args:
+            oracle.apply_linear(*a, idx.numpy(), gate.numpy().astype(np.float64), nthreads=nthreads)
+        dt += time.perf_counter() - t0
+        passes += 1
     # fraction of the model's weight elements the sample covered
     frac = sum(l.d_out * l.d_in for l in sub.linears) / cfg.n_elements
-    return T * frac / dt, dt, f"{T} tokens through q, gate, down"
+    return passes * T * frac / dt, dt, f"{passes} x {T} tokens through q, gate, down"
 
 
 def run_reference(args):
@@ -245,22 +249,142 @@ def run_reference(args):
     return 0
 
 
+def run_sweep(args):
+    """The single-linear 4096 x 4096 grid: E in {4, 8, 16, 32}, r in {8, 16,
+    32, 64}, k in {1, 2, 4}; merge per (E, r, k) and apply per T in {1, 16,
+    128}.  A 33.5 MB layer fits in the 126 MB L2, so every point rotates
+    through 8 independent copies (W, W', A, B and a plan each, 8 x 100+ MB
+    touched per cycle) and each launch finds its operands in HBM.  Per point:
+    the device time of one launch (CUDA events around it, median), the time
+    per launch when launches run back to back (launch gaps included), and the
+    host time of the API call (launch overhead)."""
+    import torch
+    import adapter_merge_b200 as am
+    from adapter_merge_b200 import build as ambuild
+    import synth
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    ambuild.build()
+    peak, peak_kind = read_peaks()
+    stream = torch.cuda.current_stream()
+    NC, R = 8, 5                          # copies, rounds over the copies
+    points = []
+    t_begin = time.perf_counter()
+    for E in (4, 8, 16, 32):
+        for r in (8, 16, 32, 64):
+            for k in (1, 2, 4):
+                if k > E or k * r > 256:
+                    continue
+                cfg = synth.sweep_point(E, r, k, 128)
+                lin = cfg.linears[0]
+                copies = []
+                for c in range(NC):
+                    w = synth.make_weights(cfg, 7000 + c, device=dev)
+                    Wo = torch.empty_like(w.W_views[0])
+                    plan = am.Plan([(w.W_views[0], Wo, w.A_views[0], w.B_views[0])], E, r)
+                    copies.append((w, Wo, plan))
+                # gates = softmax of N(0,1) logits, top-k: the router with an
+                # identity W_r makes its logits the synthetic input itself
+                xl = torch.zeros((1, 32), dtype=torch.bfloat16, device=dev)
+                xl[0, :E] = synth.normal((E,), 1.0, torch.bfloat16, 11, f"sweep-logits-E{E}-r{r}-k{k}").to(dev)
+                sel_i, sel_g = am.pregate(xl, torch.eye(E, 32, dtype=torch.float32, device=dev), k)
+                idx, gate = sel_i[0], sel_g[0]
+
+                def timed(fn):
+                    for c in range(NC):
+                        fn(c)
+                    torch.cuda.synchronize()
+                    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(NC * R)]
+                    for i in range(NC * R):
+                        ev[i][0].record(stream)
+                        fn(i % NC)
+                        ev[i][1].record(stream)
+                    torch.cuda.synchronize()
+                    dev_ms = statistics.median(a.elapsed_time(b) for a, b in ev)
+                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    e0.record(stream)
+                    h0 = time.perf_counter()
+                    for i in range(NC * R):
+                        fn(i % NC)
+                    h1 = time.perf_counter()
+                    e1.record(stream)
+                    torch.cuda.synchronize()
+                    return dev_ms, e0.elapsed_time(e1) / (NC * R), (h1 - h0) * 1e6 / (NC * R)
+
+                mb = merge_bytes(cfg, k)
+                m_dev, m_b2b, m_host = timed(lambda c: copies[c][2].merge(idx, gate))
+                pt = {"E": E, "r": r, "k": k,
+                      "merge": {"us": round(m_dev * 1e3, 2), "gbs": round(mb / (m_dev * 1e-3) / 1e9, 1),
+                                "frac_of_peak": round(mb / (m_dev * 1e-3) / 1e9 / peak, 3),
+                                "back_to_back_us": round(m_b2b * 1e3, 2), "host_us_per_call": round(m_host, 2),
+                                "bytes": mb},
+                      "apply": []}
+                for T in (1, 16, 128):
+                    X, xs = synth.make_apply_inputs(cfg, T, 5, device=dev)
+                    ys = [torch.empty((T, lin.d_out), dtype=torch.bfloat16, device=dev)]
+                    xp = am.PointerArrays(xs, ys)
+                    si, sg = synth.random_selection(T, E, k, 9, f"swa{E}{r}{k}{T}")
+                    si, sg = si.to(dev), sg.to(dev)
+                    U = int(torch.unique(si).numel())
+                    ws = torch.empty(copies[0][2].workspace_bytes(T, k), dtype=torch.uint8, device=dev)
+                    ab = apply_bytes(cfg, T, U)
+                    a_dev, a_b2b, a_host = timed(lambda c: copies[c][2].apply(xp, None, T, si, sg, ws))
+                    pt["apply"].append({"T": T, "U": U, "us": round(a_dev * 1e3, 2),
+                                        "gbs": round(ab / (a_dev * 1e-3) / 1e9, 1),
+                                        "frac_of_peak": round(ab / (a_dev * 1e-3) / 1e9 / peak, 3),
+                                        "tokens_per_s": round(T / (a_dev * 1e-3), 1),
+                                        "back_to_back_us": round(a_b2b * 1e3, 2),
+                                        "host_us_per_call": round(a_host, 2), "launches": 4, "bytes": ab})
+                for (_, _, plan) in copies:
+                    rc, st = plan.status()
+                    if rc != 0 or st != 0:
+                        raise RuntimeError(f"device status {st} at sweep point E={E} r={r} k={k}")
+                    plan.destroy()
+                points.append(pt)
+                del copies
+                torch.cuda.empty_cache()
+    if rank == 0:
+        fr = [p["merge"]["frac_of_peak"] for p in points]
+        line = {
+            "metric": "sweep: fused top-k LoRA merge GB/s per (E, r, k) and apply per T, one 4096x4096 linear",
+            "value": round(statistics.median(p["merge"]["gbs"] for p in points), 2), "unit": "GB/s",
+            "n_gpus": 1, "higher_is_better": True, "dtype": "bf16",
+            "data": "synthetic (seeded; gates = softmax of N(0,1) logits)",
+            "config": {"workload": "sweep 4096x4096, E in {4,8,16,32}, r in {8,16,32,64}, k in {1,2,4}, "
+                                   "T in {1,16,128}",
+                       "l2": f"{NC} rotated copies of every operand (no L2 reuse between launches)"},
+            "peak": peak, "peak_source": f"{peak_kind} hbm_gbs",
+            "merge_frac_of_peak": {"min": min(fr), "median": statistics.median(fr), "max": max(fr)},
+            "seconds": round(time.perf_counter() - t_begin, 1),
+            "points": points,
+        }
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--config", default="7b", choices=["7b", "13b"])
+    ap.add_argument("--config", default="7b", choices=["7b", "13b", "sweep"],
+                    help="sweep = the single-linear 4096^2 grid, measured per point (its own JSON line)")
     ap.add_argument("--layers", type=int, default=0,
                     help="use only the first N layers (small profiling case); 0 = the full model")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the switch / per-linear merge / pooled-router measurements")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
         return run_reference(args)
+    if args.config == "sweep":
+        return run_sweep(args)
 
     import torch
     import torch.distributed as dist
@@ -458,12 +582,59 @@ def main():
                        "x in and y out (weights resident)"}
         del h_W, h_A, h_B, h_Wout
 
+    # The NEXT rows on the same plan, outside the timed region: in-place switch
+    # between two selections (rank 2kr), the one-launch-per-linear merge, and
+    # the sequence-level router on the mean of the T first tokens.
+    extras = None
+    if not args.no_extras:
+        sel = [(torch.tensor(a, dtype=torch.int32, device=dev), torch.tensor(g, dtype=torch.float32, device=dev))
+               for a, g in (((1, 5), (0.4, 0.3)), ((6, 2), (0.5, 0.2)))]
+        if cfg.E < 7:
+            sel = sel[:1] + [(sel[0][0].flip(0), sel[0][1].flip(0))]
+        plan.merge(*sel[0])
+
+        def ev_mean(fn, n):
+            e = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n)]
+            fn(0)
+            torch.cuda.synchronize()
+            for i in range(n):
+                e[i][0].record(stream)
+                fn(i + 1)
+                e[i][1].record(stream)
+            torch.cuda.synchronize()
+            return mean([a.elapsed_time(b) for a, b in e])
+
+        def do_switch(i):
+            new, old = sel[(i + 1) % 2], sel[i % 2]
+            plan.switch(new[0], new[1], old[0], old[1])
+
+        n_sw = 10
+        sw_ms = ev_mean(do_switch, n_sw)
+        pl_ms = ev_mean(lambda i: plan.merge_per_linear(*sel[0]), 5)
+        pool_ms = ev_mean(lambda i: am.pregate(x_first, w.W_r, cfg.k, pool=True), 10)
+        sw_ms, pl_ms, pool_ms = max_over_ranks([sw_ms, pl_ms, pool_ms], dist, dev)
+        rc, st = plan.status()
+        if rc != 0 or st != 0:
+            raise RuntimeError(f"device status {st} after the extra measurements")
+        sb = merge_bytes(cfg, 2 * cfg.k)
+        extras = {
+            "switch": {"gbs": round(job_throughput(world, sb, sw_ms), 2), "ms": round(sw_ms, 4), "bytes": sb,
+                       "frac_of_peak": round(sb / (sw_ms * 1e-3) / 1e9 / read_peaks()[0], 4),
+                       "note": "W' <- W' - dW(old) + dW(new) in place, one launch, rank 2kr"},
+            "merge_per_linear": {"gbs": round(job_throughput(world, mb, pl_ms), 2), "ms": round(pl_ms, 4),
+                                 "launches": cfg.n_lin,
+                                 "vs_fused": round(pl_ms / m_kern, 3),
+                                 "note": "one CUDA-core launch per linear, no pipeline (ablation baseline)"},
+            "pregate_pooled": {"ms": round(pool_ms, 4), "tokens": T,
+                               "note": "one decision from the mean of the T router inputs"},
+        }
+
     cpu = None
     if rank == 0 and not args.no_cpu_baseline:
         import oracle
         cores = oracle.max_threads()
         gbs, dt, sample = cpu_oracle_merge(cfg, 10.0, cores)
-        tps, dta, sample_a = cpu_oracle_apply(cfg, 5.0, cores)
+        tps, dta, sample_a = cpu_oracle_apply(cfg, 10.0, cores)
         cpu = {"value": round(gbs, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
                "sample": f"{sample}; {dt:.1f} s",
                "apply_tokens_per_s": round(tps, 3), "apply_sample": f"{sample_a}; {dta:.1f} s"}
@@ -474,7 +645,7 @@ def main():
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded; Llama-2-7B shapes, random-init weights and adapters)",
-            "config": {"workload": f"{cfg.name}: full-model merge for one request (224 linears, E={cfg.E}, "
+            "config": {"workload": f"{cfg.name}: full-model merge for one request ({cfg.n_lin} linears, E={cfg.E}, "
                                    f"r={cfg.r}, top-{cfg.k}) + batched-decode apply (T={T})",
                        "linears": cfg.n_lin, "E": cfg.E, "r": cfg.r, "k": cfg.k, "apply_tokens": T,
                        "parallelism": f"replicas x{world} (independent requests, no collective)",
@@ -496,6 +667,7 @@ def main():
             "clocks": clocks,
             "e2e": e2e,
             "cpu_baseline": cpu,
+            "extras": extras,
         }
         print(json.dumps(line), flush=True)
     plan.destroy()
