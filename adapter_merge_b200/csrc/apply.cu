@@ -39,9 +39,11 @@ namespace {
 // ------------------------------------------------------------------ workspace
 
 struct WsLayout {
-    size_t off_offsets, off_used, off_perm, off_S, off_P, total;
+    size_t off_offsets, off_used, off_perm, off_S, off_P, off_Yp, off_cnt, total;
     int32_t Umax, Kext, Mt, Npad, n_tt;
     int32_t shape, tile;    // apply units of 128 << shape rows; tokens per tile
+    int32_t nsplit;         // K-splits per apply unit
+    int64_t n_grp;          // apply units (before splitting) over all token tiles
     int64_t n_su;           // shrink units per token tile: Mt x total K-slices
 };
 
@@ -50,6 +52,8 @@ struct WsLayout {
 // streamed once per extra tile.
 int apply_shape(int64_t T) { return T <= 64 ? 2 : T <= 128 ? 1 : 0; }
 
+int64_t token_tiles(int64_t T, int shape) { return (T + (256 >> shape) - 1) / (256 >> shape); }
+
 WsLayout ws_layout(const Plan* p, int64_t T, int32_t k)
 {
     WsLayout w{};
@@ -57,10 +61,21 @@ WsLayout ws_layout(const Plan* p, int64_t T, int32_t k)
     w.Umax = (int32_t)std::min<int64_t>(p->E, P);
     w.Kext = ((w.Umax * p->r + 63) / 64) * 64;
     w.Mt = (w.Umax * p->r + kTileM - 1) / kTileM;
+    // Taller units only while they still give every SM two units or more;
+    // below one unit per SM the units are split along K (base, then expand,
+    // chunks), at least four chunks of the longest linear per split.
     w.shape = apply_shape(T);
+    while (w.shape > 0 && p->apply_units[w.shape] * token_tiles(T, w.shape) < 2 * (int64_t)p->num_sms) --w.shape;
     w.tile = 256 >> w.shape;
     w.Npad = (int32_t)std::min<int64_t>(w.tile, ((T + 15) / 16) * 16);
-    w.n_tt = (int32_t)((T + w.tile - 1) / w.tile);
+    w.n_tt = (int32_t)token_tiles(T, w.shape);
+    w.n_grp = p->apply_units[w.shape] * w.n_tt;
+    int max_kb = 1;
+    for (const LinDesc& d : p->h_desc) max_kb = std::max(max_kb, (d.d_in + kChunkK - 1) / kChunkK);
+    w.nsplit = 1;
+    if (w.n_grp < p->num_sms)
+        w.nsplit = (int32_t)std::max<int64_t>(1, std::min<int64_t>({16, (p->num_sms + w.n_grp - 1) / w.n_grp,
+                                                                    max_kb / 4}));
     w.n_su = (int64_t)w.Mt * p->total_ks;
     auto up = [](size_t b) { return ((b + 255) / 256) * 256; };
     w.off_offsets = 0;
@@ -68,7 +83,11 @@ WsLayout ws_layout(const Plan* p, int64_t T, int32_t k)
     w.off_perm = 512;
     w.off_S = 512 + up((size_t)P * 4);
     w.off_P = w.off_S + up((size_t)p->n_lin * (size_t)T * (size_t)(2 * w.Kext) * 2);
-    w.total = w.off_P + up((size_t)w.n_tt * (size_t)w.n_su * (size_t)w.Npad * kTileM * 4);
+    w.off_Yp = w.off_P + up((size_t)w.n_tt * (size_t)w.n_su * (size_t)w.Npad * kTileM * 4);
+    const size_t rows_u = (size_t)kTileM << w.shape;
+    const bool split = w.nsplit > 1;
+    w.off_cnt = w.off_Yp + (split ? up((size_t)w.n_grp * w.nsplit * w.Npad * rows_u * 4) : 0);
+    w.total = w.off_cnt + (split ? up((size_t)w.n_grp * (rows_u / 32) * 4) : 0);
     return w;
 }
 
@@ -289,8 +308,11 @@ __global__ void __launch_bounds__(128) shrink_finalize_kernel(const LinDesc* lin
                                                                const int32_t* idx, const float* gate, uint16_t* S,
                                                                int64_t T, int32_t k, int32_t r, int32_t Kext,
                                                                int32_t Npad, int32_t tile, int64_t n_su,
-                                                               int32_t total_ks)
+                                                               int32_t total_ks, int32_t* cnt, int32_t n_cnt)
 {
+    // The apply kernel's split counters start from zero on every call.
+    if (blockIdx.x == 0 && blockIdx.y == 0)
+        for (int i = threadIdx.x; i < n_cnt; i += blockDim.x) cnt[i] = 0;
     __shared__ int s_used[kMaxE + 1];
     __shared__ int s_idx[kMaxSlots];
     __shared__ float s_gate[kMaxSlots];
@@ -336,9 +358,20 @@ struct ApplyArgs {
     int32_t* status;
     int64_t T;
     int32_t n_lin, r, Npad, n_tt, n_units, Kext, tile;
+    int32_t nsplit;                 // K-splits per unit (1: no split)
+    float* Yp;                      // split partials [groups][nsplit][Npad][128 H] fp32
+    int32_t* cnt;                   // [groups] splits finished (zeroed by the finalize kernel)
     int32_t ST;
     uint32_t stage_bytes, off_bar, acc_stride, tmem_cols;
 };
+
+// A unit's share of the chunk list of its linear: nKb base chunks, then nKe
+// expand chunks, split into nsplit contiguous ranges.
+__device__ __forceinline__ void split_range(int n, int nsplit, int s, int& c0, int& c1)
+{
+    c0 = (int)((int64_t)s * n / nsplit);
+    c1 = (int)((int64_t)(s + 1) * n / nsplit);
+}
 
 template <int H> struct ApplyShape {
     static constexpr int kEpiWarps = 4 * H;         // four per 128-row block
@@ -416,7 +449,7 @@ __global__ void __launch_bounds__(ApplyShape<H>::kThreads, 1) apply_fused_kernel
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
-    const int total = a.n_units * a.n_tt;
+    const int total = a.n_units * a.n_tt * a.nsplit;
     const uint32_t xbytes = (uint32_t)a.Npad * 128u;
 
     if (warp == 0) {
@@ -432,17 +465,20 @@ __global__ void __launch_bounds__(ApplyShape<H>::kThreads, 1) apply_fused_kernel
                 s_unit[j] = u;
                 mbar_arrive(&ufull[j]);
                 if (u < 0) break;
-                const int tt = u / a.n_units;
-                const int2 lm = a.order[u - tt * a.n_units];
+                const int g = u / a.nsplit, sp = u - g * a.nsplit;
+                const int tt = g / a.n_units;
+                const int2 lm = a.order[g - tt * a.n_units];
                 const int l = lm.x;
                 const int nKb = (__ldg(&a.lins[l].d_in) + kChunkK - 1) / kChunkK;
+                int c0, c1;
+                split_range(nKb + nKe, a.nsplit, sp, c0, c1);
                 const int m0 = lm.y * kApplyRows;
                 const int t0 = tt * a.tile;
                 const CUtensorMap* mW = a.maps + (size_t)l * kMapsPerLinear + kMapW;
                 const CUtensorMap* mB = a.maps + (size_t)l * kMapsPerLinear + kMapB;
                 const CUtensorMap* mX = a.xmaps + l;
                 bool stop = false;
-                for (int kc = 0; kc < nKb + nKe; ++kc, ++gc) {
+                for (int kc = c0; kc < c1; ++kc, ++gc) {
                     const int s = (int)(gc % a.ST);
                     if (!mbar_wait(&empty[s], (uint32_t)((gc / a.ST) & 1) ^ 1u, abort_flag)) { stop = true; break; }
                     uint8_t* dst = base + (size_t)s * a.stage_bytes;
@@ -489,13 +525,16 @@ __global__ void __launch_bounds__(ApplyShape<H>::kThreads, 1) apply_fused_kernel
                 const int u = s_unit[j];
                 mbar_arrive(&uempty[j]);
                 if (u < 0) break;
-                const int l = a.order[u % a.n_units].x;
+                const int g = u / a.nsplit, sp = u - g * a.nsplit;
+                const int l = a.order[g % a.n_units].x;
                 const int nKb = (__ldg(&a.lins[l].d_in) + kChunkK - 1) / kChunkK;
+                int c0, c1;
+                split_range(nKb + nKe, a.nsplit, sp, c0, c1);
                 const int acc = ui & 1;
                 if (!mbar_wait(&accempty[acc], (uint32_t)((ui >> 1) & 1) ^ 1u, abort_flag)) break;
                 tc_fence_after();
                 const uint32_t d = tmem_base + (uint32_t)acc * a.acc_stride;
-                for (int kc = 0; kc < nKb + nKe; ++kc, ++gc) {
+                for (int kc = c0; kc < c1; ++kc, ++gc) {
                     const int s = (int)(gc % a.ST);
                     if (!mbar_wait(&full[s], (uint32_t)((gc / a.ST) & 1), abort_flag)) { stop = true; break; }
                     tc_fence_after();
@@ -510,7 +549,8 @@ __global__ void __launch_bounds__(ApplyShape<H>::kThreads, 1) apply_fused_kernel
                                 ? make_sdesc(aaddr + (uint32_t)kk * 32u, 16u, 1024u, kLayoutSw128)
                                 : make_sdesc(aaddr + (uint32_t)kk * 4096u, 2048u, 128u, kLayoutNone);
                             const uint64_t bdesc = make_sdesc(baddr + (uint32_t)kk * 32u, 16u, 1024u, kLayoutSw128);
-                            tc_mma_bf16(d + (uint32_t)(hh * a.Npad), adesc, bdesc, idesc, (kc | kk) ? 1u : 0u);
+                            tc_mma_bf16(d + (uint32_t)(hh * a.Npad), adesc, bdesc, idesc,
+                                        (kc != c0 || kk) ? 1u : 0u);
                         }
                     }
                     tc_commit(&empty[s]);
@@ -524,8 +564,14 @@ __global__ void __launch_bounds__(ApplyShape<H>::kThreads, 1) apply_fused_kernel
         __syncwarp();
     } else {
         // ------------------------------------------------------------ epilogue
+        // Warp (hh, q) owns rows [hh*128 + q*32, +32) of the unit.  Without a
+        // K split it rounds its accumulator rows straight into y.  With one it
+        // stores them as an fp32 partial; the warp that finishes its rows last
+        // among the unit's splits adds the partials in split order (so the
+        // result does not depend on which split ends last) and writes y.
         const int q = warp & 3;        // TMEM lane quarter: warps 2,3,4,5 -> 2,3,0,1
-        const int hh = (warp - 2) >> 2;                        // which 128-row half
+        const int hh = (warp - 2) >> 2;                        // which 128-row block
+        const int rin = hh * kTileM + q * 32 + lane;           // row within the unit
         for (int ui = 0;; ++ui) {
             const int j = ui & (kUnitRing - 1);
             bool ok = mbar_wait(&ufull[j], (uint32_t)((ui / kUnitRing) & 1), abort_flag);
@@ -534,8 +580,9 @@ __global__ void __launch_bounds__(ApplyShape<H>::kThreads, 1) apply_fused_kernel
             __syncwarp();
             if (lane == 0) mbar_arrive(&uempty[j]);
             if (u < 0) break;
-            const int tt = u / a.n_units;
-            const int2 lm = a.order[u - tt * a.n_units];
+            const int g = u / a.nsplit, sp = u - g * a.nsplit;
+            const int tt = g / a.n_units;
+            const int2 lm = a.order[g - tt * a.n_units];
             const int acc = ui & 1;
             ok = mbar_wait(&accfull[acc], (uint32_t)((ui >> 1) & 1), abort_flag);
             if (!__all_sync(0xffffffffu, ok)) break;
@@ -543,26 +590,40 @@ __global__ void __launch_bounds__(ApplyShape<H>::kThreads, 1) apply_fused_kernel
             const int d_out = __ldg(&a.lins[lm.x].d_out);
             uint16_t* y = a.y_ptrs[lm.x];
             const int64_t T = a.T;
-            const int row = lm.y * kApplyRows + hh * kTileM + q * 32 + lane;
+            const int row = lm.y * kApplyRows + rin;
+            const int64_t tb = (int64_t)tt * a.tile;
             const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)acc * a.acc_stride +
                                    (uint32_t)(hh * a.Npad);
+            int kc0 = 0, kc1 = 1;
+            if (a.nsplit > 1) {
+                const int nKb = (__ldg(&a.lins[lm.x].d_in) + kChunkK - 1) / kChunkK;
+                split_range(nKb + nKe, a.nsplit, sp, kc0, kc1);
+            }
+            float* part = a.Yp + ((int64_t)u * a.Npad) * kApplyRows + rin;
             for (int c0 = 0; c0 < a.Npad; c0 += 32) {
                 uint32_t v[32];
-                if (a.Npad - c0 >= 32) {
+                if (kc0 == kc1) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) v[i] = 0;       // empty split: its share is zero
+                } else if (a.Npad - c0 >= 32) {
                     tc_ld_x32(tbase + (uint32_t)c0, v);
+                    tc_wait_ld();
                 } else {
                     uint32_t h[16];
                     tc_ld_x16(tbase + (uint32_t)c0, h);
+                    tc_wait_ld();
 #pragma unroll
                     for (int i = 0; i < 16; ++i) { v[i] = h[i]; v[16 + i] = 0; }
                 }
-                tc_wait_ld();
-                if (row < d_out) {
-                    const int64_t t0 = (int64_t)tt * a.tile + c0;
-                    uint16_t* yp = y + t0 * d_out + row;
+                if (a.nsplit > 1) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        if (c0 + i < a.Npad) part[(int64_t)(c0 + i) * kApplyRows] = __uint_as_float(v[i]);
+                } else if (row < d_out) {
+                    uint16_t* yp = y + (tb + c0) * d_out + row;
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
-                        if (c0 + i < a.Npad && t0 + i < T)
+                        if (c0 + i < a.Npad && tb + c0 + i < T)
                             yp[(int64_t)i * d_out] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[i])));
                     }
                 }
@@ -570,6 +631,41 @@ __global__ void __launch_bounds__(ApplyShape<H>::kThreads, 1) apply_fused_kernel
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&accempty[acc]);
+            if (a.nsplit > 1) {
+                __threadfence();
+                __syncwarp();
+                int last = 0;
+                if (lane == 0)
+                    last = atomicAdd(&a.cnt[(int64_t)g * kApplyEpiWarps + (warp - 2)], 1) == a.nsplit - 1;
+                last = __shfl_sync(0xffffffffu, last, 0);
+                if (last) {
+                    __threadfence();
+                    const float* p0 = a.Yp + ((int64_t)g * a.nsplit * a.Npad) * kApplyRows + rin;
+                    for (int c0 = 0; c0 < a.Npad; c0 += 32) {
+                        // 32 independent loads per split in flight; each sum
+                        // still runs over the splits in order
+                        float v[32];
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) v[i] = 0.f;
+                        for (int s2 = 0; s2 < a.nsplit; ++s2) {
+                            const float* ps = p0 + ((int64_t)s2 * a.Npad + c0) * kApplyRows;
+                            float t[32];
+#pragma unroll
+                            for (int i = 0; i < 32; ++i)
+                                t[i] = (c0 + i < a.Npad) ? __ldcg(ps + (int64_t)i * kApplyRows) : 0.f;
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) v[i] += t[i];
+                        }
+                        if (row < d_out) {
+                            uint16_t* yp = y + (tb + c0) * d_out + row;
+#pragma unroll
+                            for (int i = 0; i < 32; ++i)
+                                if (c0 + i < a.Npad && tb + c0 + i < T)
+                                    yp[(int64_t)i * d_out] = __bfloat16_as_ushort(__float2bfloat16_rn(v[i]));
+                        }
+                    }
+                }
+            }
         }
     }
 
@@ -627,6 +723,8 @@ int launch_apply_kernels(Plan* p, const WsLayout& w, uint8_t* wsb, const CUtenso
     float* P = reinterpret_cast<float*>(wsb + w.off_P);
     const int32_t Npad = w.Npad;
     const int H = 1 << w.shape;
+    int32_t* cnt = w.nsplit > 1 ? reinterpret_cast<int32_t*>(wsb + w.off_cnt) : nullptr;
+    const int32_t n_cnt = w.nsplit > 1 ? (int32_t)(w.n_grp * 4 * H) : 0;
     const uint32_t kSmemMax = 232448u;
 
     int rc = launch_segments(idx, T, k, p->E, offsets, perm, used, p->d_status, s);
@@ -665,7 +763,7 @@ int launch_apply_kernels(Plan* p, const WsLayout& w, uint8_t* wsb, const CUtenso
         shrink_tc_kernel<<<(int)std::min<int64_t>(p->num_sms, w.n_su * w.n_tt), kShrinkThreads, smem, s>>>(sa);
         if (cudaGetLastError() != cudaSuccess) return ADAFUSE_ERR_CUDA;
         shrink_finalize_kernel<<<dim3((unsigned)p->n_lin, (unsigned)T), 128, 0, s>>>(
-            p->d_desc, P, used, idx, gate, S, T, k, p->r, w.Kext, Npad, w.tile, w.n_su, p->total_ks);
+            p->d_desc, P, used, idx, gate, S, T, k, p->r, w.Kext, Npad, w.tile, w.n_su, p->total_ks, cnt, n_cnt);
         if (cudaGetLastError() != cudaSuccess) return ADAFUSE_ERR_CUDA;
     }
 
@@ -687,6 +785,9 @@ int launch_apply_kernels(Plan* p, const WsLayout& w, uint8_t* wsb, const CUtenso
     a.n_units = (int32_t)p->apply_units[w.shape];
     a.Kext = w.Kext;
     a.tile = w.tile;
+    a.nsplit = w.nsplit;
+    a.Yp = w.nsplit > 1 ? reinterpret_cast<float*>(wsb + w.off_Yp) : nullptr;
+    a.cnt = cnt;
     a.status = p->d_status;
     a.T = T;
     a.n_lin = p->n_lin;
@@ -698,7 +799,7 @@ int launch_apply_kernels(Plan* p, const WsLayout& w, uint8_t* wsb, const CUtenso
     a.tmem_cols = 2 * accs;
     a.ST = ST;
     a.off_bar = (uint32_t)ST * stage_bytes;
-    const int grid = (int)std::min<int64_t>(p->num_sms, (int64_t)a.n_units * a.n_tt);
+    const int grid = (int)std::min<int64_t>(p->num_sms, w.n_grp * w.nsplit);
     p->last_launches = 4;
     switch (H) {
     case 1: return launch_apply_fused<1>(a, smem, grid, s);

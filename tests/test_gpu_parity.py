@@ -314,6 +314,33 @@ def test_apply_ranks(am, cuda_device, E, r, k, T):
     check_apply(m, xs, ys, idx.numpy(), gate.numpy().astype(np.float64), f"E{E} r{r} k{k} T{T}")
 
 
+# On a 148-SM B200 a plan this small gives 8 units of 128 rows, so every unit
+# is split along K into 16 ranges of its chunk list (base, then expand); the
+# (128, 72) linear has about 6 chunks, so most of its splits are empty.
+@pytest.mark.parametrize("T", [1, 16, 64, 100, 200])
+def test_apply_split_k_with_empty_splits(am, cuda_device, T):
+    cfg = synth.custom([(256, 4096), (128, 72), (520, 1032)], 6, 16, 2, T, name=f"asplit{T}")
+    m, xs, xs_dev, ys, xp, yp, idx, gate, ws = apply_setup(cfg, cuda_device, T)
+    for rep in range(2):                 # the split counters must start from zero on every call
+        for y in ys:
+            y.fill_(float("nan"))
+        run_apply(m, xp, yp, T, idx, gate, ws, cuda_device)
+        check_apply(m, xs, ys, idx.numpy(), gate.numpy().astype(np.float64), f"split T={T} call {rep}")
+    assert m.plan.status() == (0, 0)
+
+
+# 152 linears of 1024 x 128: 304, 608 and 1216 units of 512, 256 and 128 rows,
+# enough for every unit height to run unsplit (T = 48, 100, 200).
+@pytest.mark.parametrize("T", [48, 100, 200])
+def test_apply_unit_heights_unsplit(am, cuda_device, T):
+    cfg = synth.custom([(1024, 128)] * 152, 4, 8, 2, T, name=f"aheights{T}")
+    m, xs, xs_dev, ys, xp, yp, idx, gate, ws = apply_setup(cfg, cuda_device, T)
+    run_apply(m, xp, yp, T, idx, gate, ws, cuda_device)
+    check_apply(m, xs, ys, idx.numpy(), gate.numpy().astype(np.float64), f"heights T={T}",
+                lins=range(0, 152, 7))
+    assert m.plan.status() == (0, 0)
+
+
 def test_apply_zero_gates_poison_bad_and_duplicate(am, cuda_device):
     T = 24
     cfg = synth.custom([(264, 392)], 6, 16, 2, T, name="aedge")
