@@ -120,7 +120,7 @@ struct ShrinkArgs {
     int32_t* status;
     int64_t n_su;
     int32_t n_lin, r, Npad, n_tt, total_ks, tile;
-    int32_t ST, box_rows;
+    int32_t ST, box_rows, run_max;
     uint32_t stage_bytes, off_bar, acc_stride, tmem_cols;
 };
 
@@ -157,6 +157,7 @@ __global__ void __launch_bounds__(kShrinkThreads, 1) shrink_tc_kernel(const __gr
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(donebar + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     int* s_used = reinterpret_cast<int*>(tmem_slot + 4);     // [1 + kMaxE]
+    int* s_loads = s_used + 1 + kMaxE;                        // [kTileM / 8]: A loads of the current unit
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
@@ -201,16 +202,42 @@ __global__ void __launch_bounds__(kShrinkThreads, 1) shrink_tc_kernel(const __gr
                 const int R = a.box_rows;               // A rows per box (divides r and 128)
                 int ng = 0;
                 for (int g = 0; g < kTileM / R; ++g) if (su.mq * kTileM + g * R < rows) ++ng;
+                // One box per expert (R == r): a run of consecutive expert ids
+                // is loaded in pieces of 2^i whole experts.  Entry: expert |
+                // map << 8 | tile position << 16.
+                int nload = 0;
+                if (a.run_max > 1) {
+                    const int q0 = su.mq * (kTileM / R), q1 = q0 + ng;
+                    for (int q = q0; q < q1;) {
+                        int e = s_used[1 + q], L = 1;
+                        while (q + L < q1 && s_used[1 + q + L] == e + L) ++L;
+                        while (L > 0) {
+                            int D = 1, mi = -1;
+                            while (2 * D <= L && 2 * D <= a.run_max) { D *= 2; ++mi; }
+                            s_loads[nload++] = e | ((mi < 0 ? kMapA : kMapARun + mi) << 8) | ((q - q0) << 16);
+                            q += D; e += D; L -= D;
+                        }
+                    }
+                }
                 for (int kc = 0; kc < su.nK; ++kc, ++gc) {
                     const int s = (int)(gc % a.ST);
                     if (!mbar_wait(&empty[s], (uint32_t)((gc / a.ST) & 1) ^ 1u, abort_flag)) { stop = true; break; }
                     uint8_t* dst = base + (size_t)s * a.stage_bytes;
                     const int col = su.k0 + kc * kChunkK;
                     mbar_arrive_expect_tx(&full[s], (uint32_t)(ng * R) * 128u + xbytes);
-                    for (int g = 0; g < ng; ++g) {
-                        const int c = su.mq * kTileM + g * R;
-                        const int qq = c / a.r, j0 = c - qq * a.r;
-                        tma_load_3d(dst + (size_t)g * R * 128u, mA, &full[s], col, j0, s_used[1 + qq]);
+                    if (a.run_max > 1) {
+                        for (int i = 0; i < nload; ++i) {
+                            const int v = s_loads[i];
+                            tma_load_3d(dst + (size_t)(v >> 16) * R * 128u,
+                                        a.maps + (size_t)su.l * kMapsPerLinear + ((v >> 8) & 0xff), &full[s], col, 0,
+                                        v & 0xff);
+                        }
+                    } else {
+                        for (int g = 0; g < ng; ++g) {
+                            const int c = su.mq * kTileM + g * R;
+                            const int qq = c / a.r, j0 = c - qq * a.r;
+                            tma_load_3d(dst + (size_t)g * R * 128u, mA, &full[s], col, j0, s_used[1 + qq]);
+                        }
                     }
                     tma_load_2d(dst + kAChunkBytes, mX, &full[s], col, tt * a.tile);
                     issued = gc + 1;
@@ -753,6 +780,7 @@ int launch_apply_kernels(Plan* p, const WsLayout& w, uint8_t* wsb, const CUtenso
         sa.tile = w.tile;
         sa.ST = ST;
         sa.box_rows = p->a_box_rows;
+        sa.run_max = p->a_run_max;
         sa.stage_bytes = stage_bytes;
         sa.off_bar = (uint32_t)ST * stage_bytes;
         sa.acc_stride = accs;

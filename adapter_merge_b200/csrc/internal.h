@@ -31,9 +31,12 @@ struct LinDesc {
 // Tensor maps kept per linear: W (load, 64x128 boxes), W_out (load, 64x128
 // boxes), B (3-D stack, 8x128x1 boxes), W_out store (64x32 boxes: one per
 // merge epilogue warp), A (3-D stack, 64 x a_box_rows x 1 boxes, 128-byte
-// swizzle).
-constexpr int kMapsPerLinear = 5;
-constexpr int kMapW = 0, kMapWout = 1, kMapB = 2, kMapWoutStore = 3, kMapA = 4;
+// swizzle) and, where a_box_rows == r, the A stack again in boxes of 2, 4, 8
+// and 16 whole experts (kMapARun + i holds 2 << i experts), so that a run of
+// consecutive experts moves in one load.
+constexpr int kMapsPerLinear = 9;
+constexpr int kMapW = 0, kMapWout = 1, kMapB = 2, kMapWoutStore = 3, kMapA = 4, kMapARun = 5;
+constexpr int kARunMaps = 4;
 constexpr int kShrinkKS = 1024;  // d_in columns per shrink work unit
 
 constexpr int kTileM = 128;      // output rows per tile (MMA M, TMEM lanes)
@@ -61,6 +64,7 @@ struct Plan {
     int64_t apply_units[kApplyShapes] = {};       // apply units for H = 1, 2, 4
     int32_t total_ks = 0;             // shrink K-slices over all linears
     int32_t a_box_rows = 8;           // rows per A-stack TMA box: largest power of two <= 128 dividing r
+    int32_t a_run_max = 1;            // most experts one A-stack load may carry (1: no run maps)
     int2* d_apply_order[kApplyShapes] = {};      // apply units (linear, row block), longest first
     int32_t* d_sched = nullptr;         // work counters of the persistent kernels (zero between launches)
     int32_t last_launches = 0;

@@ -43,11 +43,11 @@ bool encode_w(CUtensorMap* m, const void* ptr, int rows, int cols, int box_rows 
 
 // A stack: 3-D [E, r, d_in] bf16, box 64 (d_in) x rows x 1 (expert), 128-byte
 // swizzle: a box is rows/8 whole 1 KB swizzle atoms of A rows.
-bool encode_a(CUtensorMap* m, const void* ptr, int E, int r, int d_in, int64_t a_es, int rows)
+bool encode_a(CUtensorMap* m, const void* ptr, int E, int r, int d_in, int64_t a_es, int rows, int experts = 1)
 {
     cuuint64_t dims[3] = {(cuuint64_t)d_in, (cuuint64_t)r, (cuuint64_t)E};
     cuuint64_t strides[2] = {(cuuint64_t)d_in * 2, (cuuint64_t)a_es * 2};
-    cuuint32_t box[3] = {64, (cuuint32_t)rows, 1};
+    cuuint32_t box[3] = {64, (cuuint32_t)rows, (cuuint32_t)experts};
     cuuint32_t estr[3] = {1, 1, 1};
     return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -121,6 +121,10 @@ extern "C" int adafuse_plan_create(adafuse_plan** out, const adafuse_linear* lin
     std::vector<CUtensorMap> maps((size_t)n_lin * kMapsPerLinear);
     p->a_box_rows = 8;
     while (p->a_box_rows < 128 && r % (2 * p->a_box_rows) == 0) p->a_box_rows *= 2;
+    if (p->a_box_rows == r)
+        while (2 * p->a_run_max <= E && 2 * p->a_run_max * r <= kTileM &&
+               2 * p->a_run_max <= (2 << (kARunMaps - 1)))
+            p->a_run_max *= 2;
     int64_t tiles = 0, units = 0;
     int32_t kslices = 0;
     for (int l = 0; l < n_lin; ++l) {
@@ -151,6 +155,12 @@ extern "C" int adafuse_plan_create(adafuse_plan** out, const adafuse_linear* lin
             free_plan(p);
             return ADAFUSE_ERR_UNSUPPORTED;
         }
+        for (int i = 0; i < kARunMaps && (2 << i) <= p->a_run_max; ++i)
+            if (!encode_a(&maps[(size_t)l * kMapsPerLinear + kMapARun + i], L.A, E, r, L.d_in, L.a_expert_stride,
+                          p->a_box_rows, 2 << i)) {
+                free_plan(p);
+                return ADAFUSE_ERR_UNSUPPORTED;
+            }
     }
     if (units > 0x7fffffff) { free_plan(p); return ADAFUSE_ERR_UNSUPPORTED; }
     p->merge_tiles = tiles;
