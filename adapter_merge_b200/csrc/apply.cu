@@ -42,6 +42,7 @@ struct WsLayout {
     size_t off_offsets, off_used, off_perm, off_S, off_P, off_Yp, off_cnt, total;
     int32_t Umax, Kext, Mt, Npad, n_tt;
     int32_t shape, tile;    // apply units of 128 << shape rows; tokens per tile
+    int32_t ksg, total_ks;  // shrink K-slice width shrink_ks(ksg); slices over all linears
     int32_t nsplit;         // K-splits per apply unit
     int64_t n_grp;          // apply units (before splitting) over all token tiles
     int64_t n_su;           // shrink units per token tile: Mt x total K-slices
@@ -70,13 +71,23 @@ WsLayout ws_layout(const Plan* p, int64_t T, int32_t k)
     w.Npad = (int32_t)std::min<int64_t>(w.tile, ((T + 15) / 16) * 16);
     w.n_tt = (int32_t)token_tiles(T, w.shape);
     w.n_grp = p->apply_units[w.shape] * w.n_tt;
+    // Split count: the fewest waves of equal units over the SMs, each split
+    // charged a fixed 0.15 of a whole unit (pipeline fill, partial exchange).
     int max_kb = 1;
     for (const LinDesc& d : p->h_desc) max_kb = std::max(max_kb, (d.d_in + kChunkK - 1) / kChunkK);
     w.nsplit = 1;
-    if (w.n_grp < p->num_sms)
-        w.nsplit = (int32_t)std::max<int64_t>(1, std::min<int64_t>({16, (p->num_sms + w.n_grp - 1) / w.n_grp,
-                                                                    max_kb / 4}));
-    w.n_su = (int64_t)w.Mt * p->total_ks;
+    if (w.n_grp < p->num_sms) {
+        double best = 1e30;
+        for (int sp = 1; sp <= std::min(16, std::max(1, max_kb / 4)); ++sp) {
+            const int64_t waves = (w.n_grp * sp + p->num_sms - 1) / p->num_sms;
+            const double cost = (double)waves * (1.0 / sp + 0.15);
+            if (cost < best - 1e-9) { best = cost; w.nsplit = sp; }
+        }
+    }
+    // Narrow shrink slices only when the wide ones leave SMs without a unit.
+    w.ksg = (int64_t)w.Mt * p->total_ks[0] * token_tiles(T, w.shape) < p->num_sms ? 1 : 0;
+    w.total_ks = p->total_ks[w.ksg];
+    w.n_su = (int64_t)w.Mt * w.total_ks;
     auto up = [](size_t b) { return ((b + 255) / 256) * 256; };
     w.off_offsets = 0;
     w.off_used = 256;
@@ -119,7 +130,7 @@ struct ShrinkArgs {
     float* P;
     int32_t* status;
     int64_t n_su;
-    int32_t n_lin, r, Npad, n_tt, total_ks, tile;
+    int32_t n_lin, r, Npad, n_tt, total_ks, tile, ksg;
     int32_t ST, box_rows, run_max;
     uint32_t stage_bytes, off_bar, acc_stride, tmem_cols;
 };
@@ -128,19 +139,20 @@ constexpr int kShrinkThreads = 192;
 
 struct ShrinkUnit {
     int l, mq, ks, k0, nK;
-    __device__ void at(const LinDesc* lins, int n_lin, int total_ks, int64_t u)
+    __device__ void at(const LinDesc* lins, int n_lin, int total_ks, int ksg, int64_t u)
     {
         mq = (int)(u / total_ks);
         const int g = (int)(u - (int64_t)mq * total_ks);
         int lo = 0, hi = n_lin - 1;
         while (lo < hi) {
             int mid = (lo + hi + 1) >> 1;
-            if (__ldg(&lins[mid].ks_base) <= g) lo = mid; else hi = mid - 1;
+            if (__ldg(&lins[mid].ks_base[ksg]) <= g) lo = mid; else hi = mid - 1;
         }
         l = lo;
-        ks = g - __ldg(&lins[l].ks_base);
-        k0 = ks * kShrinkKS;
-        const int k1 = min(__ldg(&lins[l].d_in), k0 + kShrinkKS);
+        ks = g - __ldg(&lins[l].ks_base[ksg]);
+        const int width = shrink_ks(ksg);
+        k0 = ks * width;
+        const int k1 = min(__ldg(&lins[l].d_in), k0 + width);
         nK = (k1 - k0 + kChunkK - 1) / kChunkK;
     }
 };
@@ -195,7 +207,7 @@ __global__ void __launch_bounds__(kShrinkThreads, 1) shrink_tc_kernel(const __gr
             for (int64_t ua = u_begin; ua < u_end && !stop; ++ua) {
                 const int tt = (int)(ua / a.n_su);
                 ShrinkUnit su;
-                su.at(a.lins, a.n_lin, a.total_ks, ua - (int64_t)tt * a.n_su);
+                su.at(a.lins, a.n_lin, a.total_ks, a.ksg, ua - (int64_t)tt * a.n_su);
                 if (su.mq * kTileM >= rows) continue;
                 const CUtensorMap* mA = a.maps + (size_t)su.l * kMapsPerLinear + kMapA;
                 const CUtensorMap* mX = a.xmaps + su.l;
@@ -254,7 +266,7 @@ __global__ void __launch_bounds__(kShrinkThreads, 1) shrink_tc_kernel(const __gr
             for (int64_t ua = u_begin; ua < u_end && !stop; ++ua) {
                 const int tt = (int)(ua / a.n_su);
                 ShrinkUnit su;
-                su.at(a.lins, a.n_lin, a.total_ks, ua - (int64_t)tt * a.n_su);
+                su.at(a.lins, a.n_lin, a.total_ks, a.ksg, ua - (int64_t)tt * a.n_su);
                 if (su.mq * kTileM >= rows) continue;
                 const int acc = (int)(uc & 1);
                 if (!mbar_wait(&accempty[acc], (uint32_t)((uc >> 1) & 1) ^ 1u, abort_flag)) break;
@@ -287,7 +299,7 @@ __global__ void __launch_bounds__(kShrinkThreads, 1) shrink_tc_kernel(const __gr
             const int tt = (int)(ua / a.n_su);
             const int64_t u = ua - (int64_t)tt * a.n_su;
             ShrinkUnit su;
-            su.at(a.lins, a.n_lin, a.total_ks, u);
+            su.at(a.lins, a.n_lin, a.total_ks, a.ksg, u);
             if (su.mq * kTileM >= rows) continue;
             const int acc = (int)(uc & 1);
             bool ok = mbar_wait(&accfull[acc], (uint32_t)((uc >> 1) & 1), abort_flag);
@@ -335,7 +347,8 @@ __global__ void __launch_bounds__(128) shrink_finalize_kernel(const LinDesc* lin
                                                                const int32_t* idx, const float* gate, uint16_t* S,
                                                                int64_t T, int32_t k, int32_t r, int32_t Kext,
                                                                int32_t Npad, int32_t tile, int64_t n_su,
-                                                               int32_t total_ks, int32_t* cnt, int32_t n_cnt)
+                                                               int32_t total_ks, int32_t ksg, int32_t* cnt,
+                                                               int32_t n_cnt)
 {
     // The apply kernel's split counters start from zero on every call.
     if (blockIdx.x == 0 && blockIdx.y == 0)
@@ -349,7 +362,7 @@ __global__ void __launch_bounds__(128) shrink_finalize_kernel(const LinDesc* lin
     if (threadIdx.x < k) { s_idx[threadIdx.x] = idx[t * k + threadIdx.x]; s_gate[threadIdx.x] = gate[t * k + threadIdx.x]; }
     __syncthreads();
     const int rows = s_used[0] * r;
-    const int ks_base = __ldg(&lins[l].ks_base), n_ks = __ldg(&lins[l].n_ks);
+    const int ks_base = __ldg(&lins[l].ks_base[ksg]), n_ks = __ldg(&lins[l].n_ks[ksg]);
     const int tt = (int)(t / tile), tl = (int)(t - (int64_t)tt * tile);
     uint16_t* Srow = S + ((int64_t)l * T + t) * (2 * Kext);
     for (int c = threadIdx.x; c < Kext; c += blockDim.x) {
@@ -776,7 +789,8 @@ int launch_apply_kernels(Plan* p, const WsLayout& w, uint8_t* wsb, const CUtenso
         sa.r = p->r;
         sa.Npad = Npad;
         sa.n_tt = w.n_tt;
-        sa.total_ks = p->total_ks;
+        sa.total_ks = w.total_ks;
+        sa.ksg = w.ksg;
         sa.tile = w.tile;
         sa.ST = ST;
         sa.box_rows = p->a_box_rows;
@@ -791,7 +805,8 @@ int launch_apply_kernels(Plan* p, const WsLayout& w, uint8_t* wsb, const CUtenso
         shrink_tc_kernel<<<(int)std::min<int64_t>(p->num_sms, w.n_su * w.n_tt), kShrinkThreads, smem, s>>>(sa);
         if (cudaGetLastError() != cudaSuccess) return ADAFUSE_ERR_CUDA;
         shrink_finalize_kernel<<<dim3((unsigned)p->n_lin, (unsigned)T), 128, 0, s>>>(
-            p->d_desc, P, used, idx, gate, S, T, k, p->r, w.Kext, Npad, w.tile, w.n_su, p->total_ks, cnt, n_cnt);
+            p->d_desc, P, used, idx, gate, S, T, k, p->r, w.Kext, Npad, w.tile, w.n_su, w.total_ks, w.ksg, cnt,
+            n_cnt);
         if (cudaGetLastError() != cudaSuccess) return ADAFUSE_ERR_CUDA;
     }
 

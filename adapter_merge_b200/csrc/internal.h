@@ -24,8 +24,8 @@ struct LinDesc {
     int32_t d_out, d_in;
     int32_t n_rt;          // ceil(d_out / 128)
     int32_t n_strips;      // ceil(d_in / 128)
-    int32_t ks_base;       // first shrink K-slice (kShrinkKS columns) of this linear
-    int32_t n_ks;          // ceil(d_in / kShrinkKS)
+    int32_t ks_base[2];    // first shrink K-slice of this linear, slices of shrink_ks(g) columns
+    int32_t n_ks[2];       // ceil(d_in / shrink_ks(g))
 };
 
 // Tensor maps kept per linear: W (load, 64x128 boxes), W_out (load, 64x128
@@ -37,7 +37,9 @@ struct LinDesc {
 constexpr int kMapsPerLinear = 9;
 constexpr int kMapW = 0, kMapWout = 1, kMapB = 2, kMapWoutStore = 3, kMapA = 4, kMapARun = 5;
 constexpr int kARunMaps = 4;
-constexpr int kShrinkKS = 1024;  // d_in columns per shrink work unit
+// d_in columns per shrink work unit: g = 0 normally, g = 1 when the wide
+// slices leave SMs idle
+__host__ __device__ constexpr int shrink_ks(int g) { return g ? 256 : 1024; }
 
 constexpr int kTileM = 128;      // output rows per tile (MMA M, TMEM lanes)
 constexpr int kTileN = 128;      // merge: d_in columns per tile (MMA N)
@@ -62,7 +64,7 @@ struct Plan {
     int32_t* d_status = nullptr;
     int64_t merge_tiles = 0;
     int64_t apply_units[kApplyShapes] = {};       // apply units for H = 1, 2, 4
-    int32_t total_ks = 0;             // shrink K-slices over all linears
+    int32_t total_ks[2] = {};         // shrink K-slices over all linears, per slice width
     int32_t a_box_rows = 8;           // rows per A-stack TMA box: largest power of two <= 128 dividing r
     int32_t a_run_max = 1;            // most experts one A-stack load may carry (1: no run maps)
     int2* d_apply_order[kApplyShapes] = {};      // apply units (linear, row block), longest first

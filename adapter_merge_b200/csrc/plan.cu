@@ -126,7 +126,7 @@ extern "C" int adafuse_plan_create(adafuse_plan** out, const adafuse_linear* lin
                2 * p->a_run_max <= (2 << (kARunMaps - 1)))
             p->a_run_max *= 2;
     int64_t tiles = 0, units = 0;
-    int32_t kslices = 0;
+    int32_t kslices[2] = {0, 0};
     for (int l = 0; l < n_lin; ++l) {
         const adafuse_linear& L = lins[l];
         LinDesc& d = p->h_desc[l];
@@ -142,9 +142,11 @@ extern "C" int adafuse_plan_create(adafuse_plan** out, const adafuse_linear* lin
         d.n_strips = (L.d_in + kTileN - 1) / kTileN;
         d.tile_base = tiles;
         d.unit_base = units;
-        d.n_ks = (L.d_in + kShrinkKS - 1) / kShrinkKS;
-        d.ks_base = kslices;
-        kslices += d.n_ks;
+        for (int g = 0; g < 2; ++g) {
+            d.n_ks[g] = (L.d_in + shrink_ks(g) - 1) / shrink_ks(g);
+            d.ks_base[g] = kslices[g];
+            kslices[g] += d.n_ks[g];
+        }
         tiles += (int64_t)d.n_rt * d.n_strips;
         units += d.n_rt;
         if (!encode_w(&maps[(size_t)l * kMapsPerLinear + kMapW], L.W, L.d_out, L.d_in) ||
@@ -164,7 +166,8 @@ extern "C" int adafuse_plan_create(adafuse_plan** out, const adafuse_linear* lin
     }
     if (units > 0x7fffffff) { free_plan(p); return ADAFUSE_ERR_UNSUPPORTED; }
     p->merge_tiles = tiles;
-    p->total_ks = kslices;
+    p->total_ks[0] = kslices[0];
+    p->total_ks[1] = kslices[1];
 
     // Apply units, one list per unit height (H row blocks of 128), in
     // decreasing order of the W bytes they stream (stable), so that dynamic
