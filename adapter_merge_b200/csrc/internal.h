@@ -20,7 +20,6 @@ struct LinDesc {
     int64_t a_es;          // expert stride of A, elements
     int64_t b_es;          // expert stride of B, elements
     int64_t tile_base;     // first merge tile (128 x 128) of this linear
-    int64_t unit_base;     // first apply unit (128 output rows) of this linear
     int32_t d_out, d_in;
     int32_t n_rt;          // ceil(d_out / 128)
     int32_t n_strips;      // ceil(d_in / 128)

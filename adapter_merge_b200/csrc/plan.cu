@@ -141,7 +141,6 @@ extern "C" int adafuse_plan_create(adafuse_plan** out, const adafuse_linear* lin
         d.n_rt = (L.d_out + kTileM - 1) / kTileM;
         d.n_strips = (L.d_in + kTileN - 1) / kTileN;
         d.tile_base = tiles;
-        d.unit_base = units;
         for (int g = 0; g < 2; ++g) {
             d.n_ks[g] = (L.d_in + shrink_ks(g) - 1) / shrink_ks(g);
             d.ks_base[g] = kslices[g];
