@@ -48,7 +48,8 @@ struct MergeArgs {
     int32_t Kp;         // ns*r rounded up to 16
     int32_t mode;       // 0: merge W -> W_out; 1: switch, W_out in place
     int32_t stall;      // test hook: CTA 0 withholds its first W stage
-    int32_t SW, SB, NA; // W stages, B stages, A buffers (row-order kernel: SB unused)
+    int32_t SW, SB, NA; // W stages, B stages, A buffers (row-order kernel: SB unused, NA = Bcat row blocks)
+    int32_t NAR;        // row-order kernel: A tile slots
     int32_t box_rows;   // rows per A-stack TMA box (row-order kernel)
     uint32_t off_B, off_A, off_bar, stage_bytes;
 };
@@ -395,17 +396,23 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_fused_kernel(const __g
 
 // ------------------------------------------------------------------ row order
 
-// Row-order variant (k*r <= 128): tiles are walked along the rows of each
-// 128-row block, so consecutive tiles of a CTA continue the same rows of W
-// (longer contiguous DRAM runs; ~4 % more streaming bandwidth than walking
-// down column strips in a copy-only measurement of this pipeline).  The gate
-// moves to the B side: warps 2-3 build the gate-scaled Bcat (128 rows x Kp,
-// K-major core matrices) once per row block, and warp 0 loads the raw A rows
-// of the tile's 128 columns by TMA (MN-major, 128-byte swizzle) into the same
-// stage as the W tile.  A stage is released by the MMA (A consumed) and the
-// eight epilogue stores (W' read).
-struct RowTileIt {
-    int l, strip, rt, n_rt, n_strips;
+// Row-order variant (k*r <= 128).  Tiles are walked along the rows of W in
+// pairs of 128-row blocks, the two blocks interleaved column block by column
+// block: (rows 0-127, cols 0-127), (rows 128-255, cols 0-127), (rows 0-127,
+// cols 128-255), ...  Consecutive tiles of a CTA continue the same rows of W
+// (long contiguous DRAM runs), and the raw A rows of a 128-column block
+// (Kp x 128, MN-major, 128-byte swizzle, loaded by TMA into a ring of their
+// own) serve both blocks of the pair: half the A traffic of walking one block
+// at a time, where those loads cost 12 % of the launch.  The gate sits on the
+// B side: warps 2-3 build the gate-scaled Bcat of both row blocks (128 rows x
+// Kp each, K-major core matrices) once per pair.  A W stage is released by
+// the MMA and the eight epilogue stores (W' read), an A slot by the MMA of
+// its column block's last tile, a Bcat pair slot by the MMA of the pair's
+// last tile.
+struct PairTileIt {
+    int l, rp, strip, b, nb, n_rt, n_strips;
+    __device__ int rt() const { return 2 * rp + b; }
+    __device__ void set_nb() { nb = min(2, n_rt - 2 * rp); }
     __device__ void init(const LinDesc* lins, int n_lin, int64_t g)
     {
         int lo = 0, hi = n_lin - 1;
@@ -417,35 +424,55 @@ struct RowTileIt {
         n_rt = lins[l].n_rt;
         n_strips = lins[l].n_strips;
         const int64_t local = g - lins[l].tile_base;
-        rt = (int)(local / n_strips);
-        strip = (int)(local - (int64_t)rt * n_strips);
+        const int64_t pair_tiles = 2 * (int64_t)n_strips;
+        const int full_pairs = n_rt / 2;
+        if (local < (int64_t)full_pairs * pair_tiles) {
+            rp = (int)(local / pair_tiles);
+            const int rem = (int)(local - (int64_t)rp * pair_tiles);
+            strip = rem >> 1;
+            b = rem & 1;
+        } else {                                   // the single block left when n_rt is odd
+            rp = full_pairs;
+            strip = (int)(local - (int64_t)full_pairs * pair_tiles);
+            b = 0;
+        }
+        set_nb();
     }
     __device__ void next(const LinDesc* lins, int n_lin)
     {
-        if (++strip == n_strips) {
-            strip = 0;
-            if (++rt == n_rt) {
-                rt = 0;
-                if (++l < n_lin) {
-                    n_rt = lins[l].n_rt;
-                    n_strips = lins[l].n_strips;
-                }
-            }
+        if (++b < nb) return;
+        b = 0;
+        if (++strip < n_strips) return;
+        strip = 0;
+        if (2 * ++rp < n_rt) { set_nb(); return; }
+        rp = 0;
+        if (++l < n_lin) {
+            n_rt = lins[l].n_rt;
+            n_strips = lins[l].n_strips;
+            set_nb();
         }
     }
+    __device__ bool col_first() const { return b == 0; }
+    __device__ bool col_last() const { return b == nb - 1; }
+    __device__ bool pair_first() const { return b == 0 && strip == 0; }
+    __device__ bool pair_last() const { return b == nb - 1 && strip == n_strips - 1; }
 };
 
 __global__ void __launch_bounds__(kMergeThreads, 1) merge_rows_kernel(const __grid_constant__ MergeArgs a)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* sStage = base;                       // SW x [W tile 32 KB | A tile Kp x 128]
-    uint8_t* sBcat = base + a.off_B;              // NA x [128 x Kp] gate-scaled B rows
+    uint8_t* sStage = base;                       // SW x W tile (32 KB)
+    uint8_t* sA = base + a.off_A;                 // NAR x A tile [Kp x 128], MN-major, 128-byte swizzle
+    uint8_t* sBcat = base + a.off_B;              // NA x [128 x Kp] gate-scaled B rows, two per pair slot
+    const int NP = a.NA / 2;                      // Bcat pair slots
     uint64_t* full = reinterpret_cast<uint64_t*>(base + a.off_bar);
     uint64_t* empty = full + a.SW;
-    uint64_t* bcfull = empty + a.SW;
-    uint64_t* bcempty = bcfull + a.NA;
-    uint64_t* accfull = bcempty + a.NA;
+    uint64_t* afull = empty + a.SW;
+    uint64_t* aempty = afull + a.NAR;
+    uint64_t* bcfull = aempty + a.NAR;
+    uint64_t* bcempty = bcfull + NP;
+    uint64_t* accfull = bcempty + NP;
     uint64_t* accempty = accfull + 2;
     uint64_t* donebar = accempty + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(donebar + 1);
@@ -461,7 +488,8 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_rows_kernel(const __gr
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < a.SW; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], kEpiWarps + 1); }
-        for (int i = 0; i < a.NA; ++i) { mbar_init(&bcfull[i], 2); mbar_init(&bcempty[i], 1); }
+        for (int i = 0; i < a.NAR; ++i) { mbar_init(&afull[i], 1); mbar_init(&aempty[i], 1); }
+        for (int i = 0; i < NP; ++i) { mbar_init(&bcfull[i], 2); mbar_init(&bcempty[i], 1); }
         for (int i = 0; i < 2; ++i) { mbar_init(&accfull[i], 1); mbar_init(&accempty[i], kEpiWarps); }
         mbar_init(donebar, 1);
         *abort_flag = 0;
@@ -486,11 +514,11 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_rows_kernel(const __gr
         if (bad && blockIdx.x == 0) atomicOr(a.status, ADAFUSE_STATUS_BAD_INDEX);
         fence_mbar_init();
     }
-    // Zero the A part of every stage: the K padding rows and the rows of
-    // skipped slots are never loaded and must read as finite zeros.
-    for (int st = 0; st < a.SW; ++st)
+    // Zero every A slot: the K padding rows and the rows of skipped slots are
+    // never loaded and must read as finite zeros.
+    for (int st = 0; st < a.NAR; ++st)
         for (uint32_t o = threadIdx.x * 16; o < ATile; o += kMergeThreads * 16)
-            st_shared_v4(smem_u32(sStage + (size_t)st * a.stage_bytes + kWTileBytes + o), make_uint4(0, 0, 0, 0));
+            st_shared_v4(smem_u32(sA + (size_t)st * ATile + o), make_uint4(0, 0, 0, 0));
     fence_proxy_async_smem();
     __syncthreads();
     if (*s_skip) return;       // switch between identical selections: nothing to do
@@ -513,61 +541,76 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_rows_kernel(const __gr
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (lane == 0 && count > 0) {
-            RowTileIt it;
+            PairTileIt it;
             it.init(a.lins, a.n_lin, t_begin);
             int nvalid = 0;
             for (int s = 0; s < a.ns; ++s) if (s_e[s] >= 0) ++nvalid;
             const uint32_t abytes = (uint32_t)nvalid * (uint32_t)a.r * 256u;    // 2 halves x r rows x 128 B
             const int R = a.box_rows;
-            int64_t issued = 0;
+            int64_t issued = 0, aseq = -1, a_issued = 0;
             for (int64_t i = 0; i < count; ++i) {
                 const int sw = (int)(i % a.SW);
                 if (!mbar_wait(&empty[sw], (uint32_t)((i / a.SW) & 1) ^ 1u, abort_flag)) break;
                 const CUtensorMap* mW = a.maps + (size_t)it.l * kMapsPerLinear + kmap_in;
-                const CUtensorMap* mA = a.maps + (size_t)it.l * kMapsPerLinear + kMapA;
-                const int n0 = it.strip * kTileN, m0 = it.rt * kTileM;
+                const int n0 = it.strip * kTileN, m0 = it.rt() * kTileM;
                 uint8_t* dst = sStage + (size_t)sw * a.stage_bytes;
                 if (!(a.stall && blockIdx.x == 0 && i == 0)) {
-                    mbar_arrive_expect_tx(&full[sw], kWTileBytes + abytes);
+                    mbar_arrive_expect_tx(&full[sw], kWTileBytes);
                     tma_load_2d(dst, mW, &full[sw], n0, m0);
                     tma_load_2d(dst + kWBoxBytes, mW, &full[sw], n0 + 64, m0);
+                    issued = i + 1;
+                }
+                if (i == 0 || it.col_first()) {
+                    // the A rows of this column block, for both tiles of the pair
+                    const int as = (int)(++aseq % a.NAR);
+                    if (!mbar_wait(&aempty[as], (uint32_t)((aseq / a.NAR) & 1) ^ 1u, abort_flag)) break;
+                    const CUtensorMap* mA = a.maps + (size_t)it.l * kMapsPerLinear + kMapA;
+                    uint8_t* adst = sA + (size_t)as * ATile;
+                    mbar_arrive_expect_tx(&afull[as], abytes);
                     for (int s = 0; s < a.ns; ++s) {
                         const int e = s_e[s];
                         if (e < 0) continue;
                         for (int h = 0; h < 2; ++h)
                             for (int j0 = 0; j0 < a.r; j0 += R)
-                                tma_load_3d(dst + kWTileBytes + (size_t)h * a.Kp * 128u + (size_t)((s * a.r + j0) / 8) * 1024u,
-                                            mA, &full[sw], n0 + 64 * h, j0, e);
+                                tma_load_3d(adst + (size_t)h * a.Kp * 128u + (size_t)((s * a.r + j0) / 8) * 1024u,
+                                            mA, &afull[as], n0 + 64 * h, j0, e);
                     }
-                    issued = i + 1;
+                    a_issued = aseq + 1;
                 }
                 if (i + 1 < count) it.next(a.lins, a.n_lin);
             }
+            // Drain the TMA loads still in flight before the CTA may exit.
             for (int64_t j = std::max<int64_t>(0, issued - a.SW); j < issued; ++j)
                 mbar_wait_drain(&full[j % a.SW], (uint32_t)((j / a.SW) & 1));
+            for (int64_t j = std::max<int64_t>(0, a_issued - a.NAR); j < a_issued; ++j)
+                mbar_wait_drain(&afull[j % a.NAR], (uint32_t)((j / a.NAR) & 1));
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0 && count > 0) {
-            RowTileIt it;
+            PairTileIt it;
             it.init(a.lins, a.n_lin, t_begin);
             const uint32_t idesc = make_idesc_bf16(kTileM, kTileN, 0u, 1u);
             const uint32_t lbo_a = (uint32_t)a.Kp * 128u;       // 64-column blocks of the A tile
-            int64_t blk_seq = -1;
+            int64_t pseq = -1, aseq = -1;
             for (int64_t i = 0; i < count; ++i) {
-                const bool first = (i == 0) || (it.strip == 0);
-                const bool last = (i + 1 == count) || (it.strip == it.n_strips - 1);
-                if (first) ++blk_seq;
-                const int bb = (int)(blk_seq % a.NA);
+                const bool pfirst = (i == 0) || it.pair_first();
+                const bool plast = (i + 1 == count) || it.pair_last();
+                const bool cfirst = (i == 0) || it.col_first();
+                const bool clast = (i + 1 == count) || it.col_last();
+                if (pfirst) ++pseq;
+                if (cfirst) ++aseq;
+                const int ps = (int)(pseq % NP), as = (int)(aseq % a.NAR);
                 const int sw = (int)(i % a.SW);
                 const int acc = (int)(i & 1);
                 if (!mbar_wait(&full[sw], (uint32_t)((i / a.SW) & 1), abort_flag)) break;
-                if (first && !mbar_wait(&bcfull[bb], (uint32_t)((blk_seq / a.NA) & 1), abort_flag)) break;
+                if (cfirst && !mbar_wait(&afull[as], (uint32_t)((aseq / a.NAR) & 1), abort_flag)) break;
+                if (pfirst && !mbar_wait(&bcfull[ps], (uint32_t)((pseq / NP) & 1), abort_flag)) break;
                 if (!mbar_wait(&accempty[acc], (uint32_t)((i >> 1) & 1) ^ 1u, abort_flag)) break;
                 tc_fence_after();
                 const uint32_t d = tmem_base + (uint32_t)acc * kTileN;
-                const uint32_t bcaddr = smem_u32(sBcat + (size_t)bb * BcBytes);
-                const uint32_t aaddr = smem_u32(sStage + (size_t)sw * a.stage_bytes + kWTileBytes);
+                const uint32_t bcaddr = smem_u32(sBcat + (size_t)(ps * 2 + it.b) * BcBytes);
+                const uint32_t aaddr = smem_u32(sA + (size_t)as * ATile);
                 for (int kk = 0; kk < a.Kp / 16; ++kk) {
                     const uint64_t adesc = make_sdesc(bcaddr + (uint32_t)kk * 4096u, 2048u, 128u, kLayoutNone);
                     const uint64_t bdesc = make_sdesc(aaddr + (uint32_t)kk * 2048u, lbo_a, 1024u, kLayoutSw128);
@@ -575,7 +618,8 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_rows_kernel(const __gr
                 }
                 tc_commit(&accfull[acc]);
                 tc_commit(&empty[sw]);
-                if (last) tc_commit(&bcempty[bb]);
+                if (clast) tc_commit(&aempty[as]);
+                if (plast) tc_commit(&bcempty[ps]);
                 if (i + 1 < count) it.next(a.lins, a.n_lin);
             }
             tc_commit(donebar);
@@ -586,53 +630,55 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_rows_kernel(const __gr
         // ------------------------------------------------------------ Bcat builder
         if (count > 0) {
             const int tb = (warp - 2) * 32 + lane;
-            RowTileIt it;
+            PairTileIt it;
             it.init(a.lins, a.n_lin, t_begin);
-            int64_t blk_seq = -1;
+            int64_t pseq = -1;
             for (int64_t i = 0; i < count; ++i) {
-                if (i == 0 || it.strip == 0) {
-                    ++blk_seq;
-                    const int bb = (int)(blk_seq % a.NA);
-                    bool ok = mbar_wait(&bcempty[bb], (uint32_t)((blk_seq / a.NA) & 1) ^ 1u, abort_flag);
+                if (i == 0 || it.pair_first()) {
+                    ++pseq;
+                    const int ps = (int)(pseq % NP);
+                    bool ok = mbar_wait(&bcempty[ps], (uint32_t)((pseq / NP) & 1) ^ 1u, abort_flag);
                     ok = __all_sync(0xffffffffu, ok);
                     if (!ok) break;
                     const LinDesc L = a.lins[it.l];
-                    const int m0 = it.rt * kTileM;
-                    const uint32_t bbase = smem_u32(sBcat + (size_t)bb * BcBytes);
-                    const int groups = a.Kp / 8;
-                    const int total = kTileM * groups;         // (row, 8-column group) pairs
-                    for (int id0 = 0; id0 < total; id0 += 64 * 8) {
-                        uint4 v[8];
-                        float gs[8];
+                    for (int bq = 0; bq < it.nb; ++bq) {         // both row blocks of the pair
+                        const int m0 = (2 * it.rp + bq) * kTileM;
+                        const uint32_t bbase = smem_u32(sBcat + (size_t)(ps * 2 + bq) * BcBytes);
+                        const int groups = a.Kp / 8;
+                        const int total = kTileM * groups;         // (row, 8-column group) pairs
+                        for (int id0 = 0; id0 < total; id0 += 64 * 8) {
+                            uint4 v[8];
+                            float gs[8];
 #pragma unroll
-                        for (int u = 0; u < 8; ++u) {
-                            const int id = id0 + u * 64 + tb;
-                            v[u] = make_uint4(0, 0, 0, 0);
-                            gs[u] = 0.f;
-                            if (id < total) {
-                                const int row = id / groups, cg = id - row * groups;
-                                const int c = cg * 8;
-                                const int s = c / a.r, j = c - s * a.r;
-                                const int o = m0 + row;
-                                if (s < a.ns && s_e[s] >= 0 && o < L.d_out) {
-                                    v[u] = ld_global_nc_v4(L.B + (int64_t)s_e[s] * L.b_es + (int64_t)o * a.r + j);
-                                    gs[u] = s_g[s];
+                            for (int u = 0; u < 8; ++u) {
+                                const int id = id0 + u * 64 + tb;
+                                v[u] = make_uint4(0, 0, 0, 0);
+                                gs[u] = 0.f;
+                                if (id < total) {
+                                    const int row = id / groups, cg = id - row * groups;
+                                    const int c = cg * 8;
+                                    const int s = c / a.r, j = c - s * a.r;
+                                    const int o = m0 + row;
+                                    if (s < a.ns && s_e[s] >= 0 && o < L.d_out) {
+                                        v[u] = ld_global_nc_v4(L.B + (int64_t)s_e[s] * L.b_es + (int64_t)o * a.r + j);
+                                        gs[u] = s_g[s];
+                                    }
                                 }
                             }
-                        }
 #pragma unroll
-                        for (int u = 0; u < 8; ++u) {
-                            const int id = id0 + u * 64 + tb;
-                            if (id < total) {
-                                const int row = id / groups, cg = id - row * groups;
-                                st_shared_v4(bbase + (uint32_t)(row >> 3) * 128u + (uint32_t)cg * 2048u + (uint32_t)(row & 7) * 16u,
-                                             scale_bf16x8(v[u], gs[u]));
+                            for (int u = 0; u < 8; ++u) {
+                                const int id = id0 + u * 64 + tb;
+                                if (id < total) {
+                                    const int row = id / groups, cg = id - row * groups;
+                                    st_shared_v4(bbase + (uint32_t)(row >> 3) * 128u + (uint32_t)cg * 2048u + (uint32_t)(row & 7) * 16u,
+                                                 scale_bf16x8(v[u], gs[u]));
+                                }
                             }
                         }
                     }
                     fence_proxy_async_smem();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&bcfull[bb]);
+                    if (lane == 0) mbar_arrive(&bcfull[ps]);
                 }
                 if (i + 1 < count) it.next(a.lins, a.n_lin);
             }
@@ -643,7 +689,7 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_rows_kernel(const __gr
         const int q = warp & 3;
         const int h = ew >> 2;
         const int row = q * 32 + lane;
-        RowTileIt it;
+        PairTileIt it;
         if (count > 0) it.init(a.lins, a.n_lin, t_begin);
         int64_t stored = 0;
         for (int64_t i = 0; i < count; ++i) {
@@ -680,7 +726,7 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_rows_kernel(const __gr
             __syncwarp();
             if (lane == 0) {
                 const CUtensorMap* mO = a.maps + (size_t)it.l * kMapsPerLinear + kMapWoutStore;
-                tma_store_2d(mO, slice, it.strip * kTileN + h * 64, it.rt * kTileM + q * 32);
+                tma_store_2d(mO, slice, it.strip * kTileN + h * 64, it.rt() * kTileM + q * 32);
                 bulk_commit_group();
                 bulk_wait_group_read<1>();
                 if (i > 0) mbar_arrive(&empty[(i - 1) % a.SW]);
@@ -775,16 +821,22 @@ int launch_merge_fused(Plan* p, const int32_t* idx0, const float* gate0, const i
     a.stall = (p->flags & ADAFUSE_PLAN_TEST_STALL) ? 1 : 0;
     a.box_rows = p->a_box_rows;
     if (a.Kp <= 128) {
-        // Row-order kernel: stages of [W tile | A tile], two Bcat buffers.
-        const uint32_t stage = kWTileBytes + (uint32_t)a.Kp * 256u;
-        const uint32_t bc = (uint32_t)a.Kp * 256u;
-        int SW = std::min(4, (int)((kSmemMax - 2048u - 2u * bc) / stage));
+        // Row-order kernel: W stages, a ring of A tiles, and the Bcat of one
+        // or two row-block pairs; the most W stages (up to four) that fit.
+        const uint32_t at = (uint32_t)a.Kp * 256u, bc = at;
+        int SW = 0, NA = 0, NAR = 0;
+        for (int na : {4, 2})
+            for (int nar : {3, 2}) {
+                const int64_t room = (int64_t)kSmemMax - 2048 - (int64_t)na * bc - (int64_t)nar * at;
+                const int sw = room > 0 ? (int)std::min<int64_t>(4, room / kWTileBytes) : 0;
+                if (sw > SW) { SW = sw; NA = na; NAR = nar; }
+            }
         if (SW >= 2) {
-            a.SW = SW; a.SB = 0; a.NA = 2;
-            a.stage_bytes = stage;
-            a.off_B = (uint32_t)SW * stage;
-            a.off_A = a.off_B;
-            a.off_bar = a.off_B + 2u * bc;
+            a.SW = SW; a.SB = 0; a.NA = NA; a.NAR = NAR;
+            a.stage_bytes = kWTileBytes;
+            a.off_A = (uint32_t)SW * kWTileBytes;
+            a.off_B = a.off_A + (uint32_t)NAR * at;
+            a.off_bar = a.off_B + (uint32_t)NA * bc;
             const uint32_t smem = a.off_bar + 1024u + 1024u;
             if (cudaFuncSetAttribute(merge_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
                 return ADAFUSE_ERR_CUDA;

@@ -10,9 +10,12 @@
 // One CTA per decision.  Warp 0 lane e owns expert e: its logit is the fp32 sum
 // of the products x_j * W_r[e, j] in ascending j (products rounded before the
 // add), so the decision is a fixed function of the inputs.  W_r streams
-// through a 4-stage cp.async ring (three 256-column chunks ahead) and warps
-// 1-3 stage the next chunk of x while warp 0 consumes the current one.  Softmax and top-k are warp shuffles over the
-// lanes (ties to the lower index, NaN ranked last).
+// through a 4-stage cp.async ring (three 256-column chunks ahead).  The whole
+// x row is staged in shared memory before the chain starts when it fits (one
+// round of loads instead of one per chunk); otherwise, and for the pooled
+// mean, warps 1-3 stage the next chunk of x while warp 0 consumes the current
+// one.  Softmax and top-k are warp shuffles over the lanes (ties to the lower
+// index, NaN ranked last).
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -48,7 +51,7 @@ __host__ __device__ constexpr int stage_floats(int E) { return E * kRowPad + kCh
 __global__ void __launch_bounds__(kRouterThreads) pregate_kernel(const uint16_t* x, int64_t T, int32_t H,
                                                                   int64_t ldx, const float* Wr, const float* br,
                                                                   int32_t E, int32_t k, uint32_t flags,
-                                                                  int32_t* idx, float* gate)
+                                                                  int32_t* idx, float* gate, int xfull)
 {
     extern __shared__ float rsm[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -90,8 +93,14 @@ __global__ void __launch_bounds__(kRouterThreads) pregate_kernel(const uint16_t*
         }
     };
 
+    float* xall = rsm + kStages * SF;          // [H] when xfull
     for (int c = 0; c < kStages - 1; ++c) issue_w(c);
-    load_x(0, tid, kRouterThreads);
+    if (xfull) {
+#pragma unroll 8
+        for (int j = tid; j < H; j += kRouterThreads) xall[j] = bf16_at(x + t * ldx + j);
+    } else {
+        load_x(0, tid, kRouterThreads);
+    }
     float z = 0.f;
     for (int c = 0; c < nchunks; ++c) {
         issue_w(c + kStages - 1);
@@ -100,7 +109,7 @@ __global__ void __launch_bounds__(kRouterThreads) pregate_kernel(const uint16_t*
         if (warp == 0) {
             if (lane < E) {
                 const float* ws = rsm + (c % kStages) * SF + lane * kRowPad;
-                const float* xs = rsm + (c % kStages) * SF + E * kRowPad;
+                const float* xs = xfull ? xall + c * kChunk : rsm + (c % kStages) * SF + E * kRowPad;
                 const int n = min(kChunk, H - c * kChunk);
                 const int n4 = n & ~15;
                 // Same order as the scalar loop: one product, one add, ascending j.
@@ -121,7 +130,7 @@ __global__ void __launch_bounds__(kRouterThreads) pregate_kernel(const uint16_t*
                 }
                 for (int jj = n4; jj < n; ++jj) z = __fadd_rn(z, __fmul_rn(xs[jj], ws[jj]));
             }
-        } else if (c + 1 < nchunks) {
+        } else if (!xfull && c + 1 < nchunks) {
             load_x(c + 1, tid - 32, kRouterThreads - 32);
         }
         __syncthreads();                       // stage c % kStages may be refilled
@@ -178,11 +187,14 @@ extern "C" int adafuse_pregate(const void* x, int64_t T, int32_t H, int64_t x_ro
     const bool pool = (flags & ADAFUSE_POOL_MEAN) != 0;
     if (!pool && T > 0x7fffffff) return ADAFUSE_ERR_UNSUPPORTED;
     const unsigned grid = pool ? 1u : (unsigned)T;
-    const size_t smem = sizeof(float) * af::kStages * af::stage_floats(E);
+    size_t smem = sizeof(float) * af::kStages * af::stage_floats(E);
+    const size_t smem_x = smem + sizeof(float) * (size_t)H;
+    const int xfull = (!pool && smem_x <= 200 * 1024) ? 1 : 0;
+    if (xfull) smem = smem_x;
     if (smem > 48 * 1024 &&
         cudaFuncSetAttribute(af::pregate_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return ADAFUSE_ERR_CUDA;
     af::pregate_kernel<<<grid, af::kRouterThreads, smem, (cudaStream_t)stream>>>(
-        static_cast<const uint16_t*>(x), T, H, x_row_stride, W_r, b_r, E, k, flags, idx, gate);
+        static_cast<const uint16_t*>(x), T, H, x_row_stride, W_r, b_r, E, k, flags, idx, gate, xfull);
     return af::cuda_err(cudaGetLastError());
 }
