@@ -50,6 +50,7 @@ struct MergeArgs {
     int32_t stall;      // test hook: CTA 0 withholds its first W stage
     int32_t SW, SB, NA; // W stages, B stages, A buffers (row-order kernel: SB unused, NA = Bcat row blocks)
     int32_t NAR;        // row-order kernel: A tile slots
+    int32_t G;          // row-order kernel: 128-row blocks per group
     int32_t box_rows;   // rows per A-stack TMA box (row-order kernel)
     uint32_t off_B, off_A, off_bar, stage_bytes;
 };
@@ -397,24 +398,25 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_fused_kernel(const __g
 // ------------------------------------------------------------------ row order
 
 // Row-order variant (k*r <= 128).  Tiles are walked along the rows of W in
-// pairs of 128-row blocks, the two blocks interleaved column block by column
-// block: (rows 0-127, cols 0-127), (rows 128-255, cols 0-127), (rows 0-127,
-// cols 128-255), ...  Consecutive tiles of a CTA continue the same rows of W
-// (long contiguous DRAM runs), and the raw A rows of a 128-column block
-// (Kp x 128, MN-major, 128-byte swizzle, loaded by TMA into a ring of their
-// own) serve both blocks of the pair: half the A traffic of walking one block
-// at a time, where those loads cost 12 % of the launch.  The gate sits on the
-// B side: warps 2-3 build the gate-scaled Bcat of both row blocks (128 rows x
-// Kp each, K-major core matrices) once per pair.  A W stage is released by
-// the MMA and the eight epilogue stores (W' read), an A slot by the MMA of
-// its column block's last tile, a Bcat pair slot by the MMA of the pair's
-// last tile.
-struct PairTileIt {
-    int l, rp, strip, b, nb, n_rt, n_strips;
-    __device__ int rt() const { return 2 * rp + b; }
-    __device__ void set_nb() { nb = min(2, n_rt - 2 * rp); }
-    __device__ void init(const LinDesc* lins, int n_lin, int64_t g)
+// groups of G (2 or 4) 128-row blocks, the blocks of a group interleaved
+// column block by column block: (block 0, cols 0-127), (block 1, cols 0-127),
+// ..., (block 0, cols 128-255), ...  Consecutive tiles of a CTA continue the
+// same rows of W (long contiguous DRAM runs), and the raw A rows of a
+// 128-column block (Kp x 128, MN-major, 128-byte swizzle, loaded by TMA into
+// a ring of their own) serve all G blocks of the group: 1/G of the A traffic
+// of walking one block at a time, where those loads cost 12 % of the launch.
+// The gate sits on the B side: warps 2-3 build the gate-scaled Bcat of the
+// group's blocks (128 rows x Kp each, K-major core matrices) once per group.
+// A W stage is released by the MMA and the eight epilogue stores (W' read),
+// an A slot by the MMA of its column block's last tile, a Bcat group slot by
+// the MMA of the group's last tile.
+struct GroupTileIt {
+    int l, gi, strip, b, nb, n_rt, n_strips, G;
+    __device__ int rt() const { return G * gi + b; }
+    __device__ void set_nb() { nb = min(G, n_rt - G * gi); }
+    __device__ void init(const LinDesc* lins, int n_lin, int64_t g, int group)
     {
+        G = group;
         int lo = 0, hi = n_lin - 1;
         while (lo < hi) {
             int mid = (lo + hi + 1) >> 1;
@@ -424,17 +426,19 @@ struct PairTileIt {
         n_rt = lins[l].n_rt;
         n_strips = lins[l].n_strips;
         const int64_t local = g - lins[l].tile_base;
-        const int64_t pair_tiles = 2 * (int64_t)n_strips;
-        const int full_pairs = n_rt / 2;
-        if (local < (int64_t)full_pairs * pair_tiles) {
-            rp = (int)(local / pair_tiles);
-            const int rem = (int)(local - (int64_t)rp * pair_tiles);
-            strip = rem >> 1;
-            b = rem & 1;
-        } else {                                   // the single block left when n_rt is odd
-            rp = full_pairs;
-            strip = (int)(local - (int64_t)full_pairs * pair_tiles);
-            b = 0;
+        const int64_t group_tiles = (int64_t)G * n_strips;
+        const int full_groups = n_rt / G;
+        if (local < (int64_t)full_groups * group_tiles) {
+            gi = (int)(local / group_tiles);
+            const int rem = (int)(local - (int64_t)gi * group_tiles);
+            strip = rem / G;
+            b = rem - strip * G;
+        } else {                                   // the blocks left when G does not divide n_rt
+            gi = full_groups;
+            const int left = n_rt - full_groups * G;
+            const int rem = (int)(local - (int64_t)full_groups * group_tiles);
+            strip = rem / left;
+            b = rem - strip * left;
         }
         set_nb();
     }
@@ -444,8 +448,8 @@ struct PairTileIt {
         b = 0;
         if (++strip < n_strips) return;
         strip = 0;
-        if (2 * ++rp < n_rt) { set_nb(); return; }
-        rp = 0;
+        if (G * ++gi < n_rt) { set_nb(); return; }
+        gi = 0;
         if (++l < n_lin) {
             n_rt = lins[l].n_rt;
             n_strips = lins[l].n_strips;
@@ -454,8 +458,8 @@ struct PairTileIt {
     }
     __device__ bool col_first() const { return b == 0; }
     __device__ bool col_last() const { return b == nb - 1; }
-    __device__ bool pair_first() const { return b == 0 && strip == 0; }
-    __device__ bool pair_last() const { return b == nb - 1 && strip == n_strips - 1; }
+    __device__ bool group_first() const { return b == 0 && strip == 0; }
+    __device__ bool group_last() const { return b == nb - 1 && strip == n_strips - 1; }
 };
 
 __global__ void __launch_bounds__(kMergeThreads, 1) merge_rows_kernel(const __grid_constant__ MergeArgs a)
@@ -464,8 +468,8 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_rows_kernel(const __gr
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sStage = base;                       // SW x W tile (32 KB)
     uint8_t* sA = base + a.off_A;                 // NAR x A tile [Kp x 128], MN-major, 128-byte swizzle
-    uint8_t* sBcat = base + a.off_B;              // NA x [128 x Kp] gate-scaled B rows, two per pair slot
-    const int NP = a.NA / 2;                      // Bcat pair slots
+    uint8_t* sBcat = base + a.off_B;              // NA x [128 x Kp] gate-scaled B rows, G per group slot
+    const int NP = a.NA / a.G;                    // Bcat group slots
     uint64_t* full = reinterpret_cast<uint64_t*>(base + a.off_bar);
     uint64_t* empty = full + a.SW;
     uint64_t* afull = empty + a.SW;
@@ -541,8 +545,8 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_rows_kernel(const __gr
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (lane == 0 && count > 0) {
-            PairTileIt it;
-            it.init(a.lins, a.n_lin, t_begin);
+            GroupTileIt it;
+            it.init(a.lins, a.n_lin, t_begin, a.G);
             int nvalid = 0;
             for (int s = 0; s < a.ns; ++s) if (s_e[s] >= 0) ++nvalid;
             const uint32_t abytes = (uint32_t)nvalid * (uint32_t)a.r * 256u;    // 2 halves x r rows x 128 B
@@ -561,7 +565,7 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_rows_kernel(const __gr
                     issued = i + 1;
                 }
                 if (i == 0 || it.col_first()) {
-                    // the A rows of this column block, for both tiles of the pair
+                    // the A rows of this column block, for every tile of the group
                     const int as = (int)(++aseq % a.NAR);
                     if (!mbar_wait(&aempty[as], (uint32_t)((aseq / a.NAR) & 1) ^ 1u, abort_flag)) break;
                     const CUtensorMap* mA = a.maps + (size_t)it.l * kMapsPerLinear + kMapA;
@@ -588,14 +592,14 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_rows_kernel(const __gr
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0 && count > 0) {
-            PairTileIt it;
-            it.init(a.lins, a.n_lin, t_begin);
+            GroupTileIt it;
+            it.init(a.lins, a.n_lin, t_begin, a.G);
             const uint32_t idesc = make_idesc_bf16(kTileM, kTileN, 0u, 1u);
             const uint32_t lbo_a = (uint32_t)a.Kp * 128u;       // 64-column blocks of the A tile
             int64_t pseq = -1, aseq = -1;
             for (int64_t i = 0; i < count; ++i) {
-                const bool pfirst = (i == 0) || it.pair_first();
-                const bool plast = (i + 1 == count) || it.pair_last();
+                const bool pfirst = (i == 0) || it.group_first();
+                const bool plast = (i + 1 == count) || it.group_last();
                 const bool cfirst = (i == 0) || it.col_first();
                 const bool clast = (i + 1 == count) || it.col_last();
                 if (pfirst) ++pseq;
@@ -609,7 +613,7 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_rows_kernel(const __gr
                 if (!mbar_wait(&accempty[acc], (uint32_t)((i >> 1) & 1) ^ 1u, abort_flag)) break;
                 tc_fence_after();
                 const uint32_t d = tmem_base + (uint32_t)acc * kTileN;
-                const uint32_t bcaddr = smem_u32(sBcat + (size_t)(ps * 2 + it.b) * BcBytes);
+                const uint32_t bcaddr = smem_u32(sBcat + (size_t)(ps * a.G + it.b) * BcBytes);
                 const uint32_t aaddr = smem_u32(sA + (size_t)as * ATile);
                 for (int kk = 0; kk < a.Kp / 16; ++kk) {
                     const uint64_t adesc = make_sdesc(bcaddr + (uint32_t)kk * 4096u, 2048u, 128u, kLayoutNone);
@@ -630,20 +634,20 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_rows_kernel(const __gr
         // ------------------------------------------------------------ Bcat builder
         if (count > 0) {
             const int tb = (warp - 2) * 32 + lane;
-            PairTileIt it;
-            it.init(a.lins, a.n_lin, t_begin);
+            GroupTileIt it;
+            it.init(a.lins, a.n_lin, t_begin, a.G);
             int64_t pseq = -1;
             for (int64_t i = 0; i < count; ++i) {
-                if (i == 0 || it.pair_first()) {
+                if (i == 0 || it.group_first()) {
                     ++pseq;
                     const int ps = (int)(pseq % NP);
                     bool ok = mbar_wait(&bcempty[ps], (uint32_t)((pseq / NP) & 1) ^ 1u, abort_flag);
                     ok = __all_sync(0xffffffffu, ok);
                     if (!ok) break;
                     const LinDesc L = a.lins[it.l];
-                    for (int bq = 0; bq < it.nb; ++bq) {         // both row blocks of the pair
-                        const int m0 = (2 * it.rp + bq) * kTileM;
-                        const uint32_t bbase = smem_u32(sBcat + (size_t)(ps * 2 + bq) * BcBytes);
+                    for (int bq = 0; bq < it.nb; ++bq) {         // every row block of the group
+                        const int m0 = (a.G * it.gi + bq) * kTileM;
+                        const uint32_t bbase = smem_u32(sBcat + (size_t)(ps * a.G + bq) * BcBytes);
                         const int groups = a.Kp / 8;
                         const int total = kTileM * groups;         // (row, 8-column group) pairs
                         for (int id0 = 0; id0 < total; id0 += 64 * 8) {
@@ -689,8 +693,8 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_rows_kernel(const __gr
         const int q = warp & 3;
         const int h = ew >> 2;
         const int row = q * 32 + lane;
-        PairTileIt it;
-        if (count > 0) it.init(a.lins, a.n_lin, t_begin);
+        GroupTileIt it;
+        if (count > 0) it.init(a.lins, a.n_lin, t_begin, a.G);
         int64_t stored = 0;
         for (int64_t i = 0; i < count; ++i) {
             const int acc = (int)(i & 1);
@@ -821,18 +825,25 @@ int launch_merge_fused(Plan* p, const int32_t* idx0, const float* gate0, const i
     a.stall = (p->flags & ADAFUSE_PLAN_TEST_STALL) ? 1 : 0;
     a.box_rows = p->a_box_rows;
     if (a.Kp <= 128) {
-        // Row-order kernel: W stages, a ring of A tiles, and the Bcat of one
-        // or two row-block pairs; the most W stages (up to four) that fit.
+        // Row-order kernel: W stages (up to four), a ring of A tiles, and the
+        // Bcat of one or two groups of G row blocks.  Preference: W stages,
+        // then the group size (less A traffic), then a second group slot (the
+        // next group's Bcat built ahead), then A slots.  Groups of four only
+        // where a CTA walks enough tiles to amortise building four blocks.
         const uint32_t at = (uint32_t)a.Kp * 256u, bc = at;
-        int SW = 0, NA = 0, NAR = 0;
-        for (int na : {4, 2})
-            for (int nar : {3, 2}) {
-                const int64_t room = (int64_t)kSmemMax - 2048 - (int64_t)na * bc - (int64_t)nar * at;
-                const int sw = room > 0 ? (int)std::min<int64_t>(4, room / kWTileBytes) : 0;
-                if (sw > SW) { SW = sw; NA = na; NAR = nar; }
-            }
+        const bool long_walk = p->merge_tiles >= 256 * (int64_t)p->num_sms;
+        int SW = 0, NA = 0, NAR = 0, G = 0;
+        for (int g : {4, 2}) {
+            if (g == 4 && !long_walk) continue;
+            for (int np : {2, 1})
+                for (int nar : {3, 2}) {
+                    const int64_t room = (int64_t)kSmemMax - 2048 - (int64_t)np * g * bc - (int64_t)nar * at;
+                    const int sw = room > 0 ? (int)std::min<int64_t>(4, room / kWTileBytes) : 0;
+                    if (sw > SW) { SW = sw; NA = np * g; NAR = nar; G = g; }
+                }
+        }
         if (SW >= 2) {
-            a.SW = SW; a.SB = 0; a.NA = NA; a.NAR = NAR;
+            a.SW = SW; a.SB = 0; a.NA = NA; a.NAR = NAR; a.G = G;
             a.stage_bytes = kWTileBytes;
             a.off_A = (uint32_t)SW * kWTileBytes;
             a.off_B = a.off_A + (uint32_t)NAR * at;
