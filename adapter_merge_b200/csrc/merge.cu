@@ -476,7 +476,8 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_rows_kernel(const __gr
     uint64_t* aempty = afull + a.NAR;
     uint64_t* bcfull = aempty + a.NAR;
     uint64_t* bcempty = bcfull + NP;
-    uint64_t* accfull = bcempty + NP;
+    uint64_t* bcload = bcempty + NP;              // raw B rows of a group slot landed (TMA)
+    uint64_t* accfull = bcload + NP;
     uint64_t* accempty = accfull + 2;
     uint64_t* donebar = accempty + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(donebar + 1);
@@ -493,7 +494,7 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_rows_kernel(const __gr
     if (threadIdx.x == 0) {
         for (int i = 0; i < a.SW; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], kEpiWarps + 1); }
         for (int i = 0; i < a.NAR; ++i) { mbar_init(&afull[i], 1); mbar_init(&aempty[i], 1); }
-        for (int i = 0; i < NP; ++i) { mbar_init(&bcfull[i], 2); mbar_init(&bcempty[i], 1); }
+        for (int i = 0; i < NP; ++i) { mbar_init(&bcfull[i], 2); mbar_init(&bcempty[i], 1); mbar_init(&bcload[i], 1); }
         for (int i = 0; i < 2; ++i) { mbar_init(&accfull[i], 1); mbar_init(&accempty[i], kEpiWarps); }
         mbar_init(donebar, 1);
         *abort_flag = 0;
@@ -636,7 +637,7 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_rows_kernel(const __gr
             const int tb = (warp - 2) * 32 + lane;
             GroupTileIt it;
             it.init(a.lins, a.n_lin, t_begin, a.G);
-            int64_t pseq = -1;
+            int64_t pseq = -1, loaded = -1;
             for (int64_t i = 0; i < count; ++i) {
                 if (i == 0 || it.group_first()) {
                     ++pseq;
@@ -644,41 +645,39 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_rows_kernel(const __gr
                     bool ok = mbar_wait(&bcempty[ps], (uint32_t)((pseq / NP) & 1) ^ 1u, abort_flag);
                     ok = __all_sync(0xffffffffu, ok);
                     if (!ok) break;
-                    const LinDesc L = a.lins[it.l];
-                    for (int bq = 0; bq < it.nb; ++bq) {         // every row block of the group
-                        const int m0 = (a.G * it.gi + bq) * kTileM;
-                        const uint32_t bbase = smem_u32(sBcat + (size_t)(ps * a.G + bq) * BcBytes);
-                        const int groups = a.Kp / 8;
-                        const int total = kTileM * groups;         // (row, 8-column group) pairs
-                        for (int id0 = 0; id0 < total; id0 += 64 * 8) {
-                            uint4 v[8];
-                            float gs[8];
-#pragma unroll
-                            for (int u = 0; u < 8; ++u) {
-                                const int id = id0 + u * 64 + tb;
-                                v[u] = make_uint4(0, 0, 0, 0);
-                                gs[u] = 0.f;
-                                if (id < total) {
-                                    const int row = id / groups, cg = id - row * groups;
-                                    const int c = cg * 8;
-                                    const int s = c / a.r, j = c - s * a.r;
-                                    const int o = m0 + row;
-                                    if (s < a.ns && s_e[s] >= 0 && o < L.d_out) {
-                                        v[u] = ld_global_nc_v4(L.B + (int64_t)s_e[s] * L.b_es + (int64_t)o * a.r + j);
-                                        gs[u] = s_g[s];
-                                    }
-                                }
+                    // The raw B rows of every block of the group come by TMA
+                    // (one 128-row x 8-column box per expert column group,
+                    // already in the K-major core-matrix layout), then both
+                    // warps scale them by their slot's gate in place; slots
+                    // without an expert and the K padding become zeros.
+                    uint8_t* gbase = sBcat + (size_t)ps * a.G * BcBytes;
+                    if (warp == 2 && lane == 0) {
+                        int nvalid = 0;
+                        for (int s2 = 0; s2 < a.ns; ++s2) if (s_e[s2] >= 0) ++nvalid;
+                        const CUtensorMap* mB = a.maps + (size_t)it.l * kMapsPerLinear + kMapB;
+                        mbar_arrive_expect_tx(&bcload[ps], (uint32_t)(it.nb * nvalid * a.r) * 256u);
+                        for (int bq = 0; bq < it.nb; ++bq)
+                            for (int s2 = 0; s2 < a.ns; ++s2) {
+                                const int e = s_e[s2];
+                                if (e < 0) continue;
+                                for (int j0 = 0; j0 < a.r; j0 += 8)
+                                    tma_load_3d(gbase + (size_t)bq * BcBytes + (size_t)((s2 * a.r + j0) / 8) * 2048u, mB,
+                                                &bcload[ps], j0, (a.G * it.gi + bq) * kTileM, e);
                             }
-#pragma unroll
-                            for (int u = 0; u < 8; ++u) {
-                                const int id = id0 + u * 64 + tb;
-                                if (id < total) {
-                                    const int row = id / groups, cg = id - row * groups;
-                                    st_shared_v4(bbase + (uint32_t)(row >> 3) * 128u + (uint32_t)cg * 2048u + (uint32_t)(row & 7) * 16u,
-                                                 scale_bf16x8(v[u], gs[u]));
-                                }
-                            }
-                        }
+                        loaded = pseq;
+                    }
+                    ok = mbar_wait(&bcload[ps], (uint32_t)((pseq / NP) & 1), abort_flag);
+                    ok = __all_sync(0xffffffffu, ok);
+                    if (!ok) break;
+                    const int groups = a.Kp / 8;
+                    const int chunks = it.nb * groups * kTileM;      // 16-byte chunks: (block, column group, row)
+                    for (int id = tb; id < chunks; id += 64) {
+                        const int cg = (id / kTileM) % groups;
+                        const int s2 = (cg * 8) / a.r;
+                        const uint32_t addr = smem_u32(gbase) + (uint32_t)id * 16u;   // = block*BcBytes + cg*2048 + row*16
+                        uint4 v = make_uint4(0, 0, 0, 0);
+                        if (s2 < a.ns && s_e[s2] >= 0) v = scale_bf16x8(ld_shared_v4(addr), s_g[s2]);
+                        st_shared_v4(addr, v);
                     }
                     fence_proxy_async_smem();
                     __syncwarp();
@@ -686,6 +685,9 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_rows_kernel(const __gr
                 }
                 if (i + 1 < count) it.next(a.lins, a.n_lin);
             }
+            // After an abort the last B loads may still be in flight.
+            if (warp == 2 && lane == 0 && loaded >= 0)
+                mbar_wait_drain(&bcload[loaded % NP], (uint32_t)((loaded / NP) & 1));
         }
     } else {
         // ------------------------------------------------------------ epilogue

@@ -434,6 +434,27 @@ def test_full_size_merge_sampled(am, cuda_device, cfg_fn):
             assert_delta_frobenius(got, W[rr[0]:rr[1]], ref, dz, f"{cfg.name} linear {l} rows {rr}")
     assert m.plan.status() == (0, 0)
 
+    # In-place switch to another selection at full size (rank 2kr, the same
+    # launch configuration as the benchmark's switch): sampled rows against
+    # the oracle's switch of the oracle's own merged rows.
+    new_i = np.array([(int(idx_ref[0][s]) + 1 + s) % cfg.E for s in range(cfg.k)], dtype=np.int32)
+    if len(set(new_i.tolist())) < cfg.k:
+        new_i = np.arange(cfg.k, dtype=np.int32)
+    new_g = np.linspace(0.5, 0.2, cfg.k).astype(np.float32)
+    d = lambda a_, t: torch.as_tensor(a_.astype(t)).to(cuda_device)
+    m.plan.switch(d(new_i, np.int32), d(new_g, np.float32), idx[0], gate[0])
+    torch.cuda.synchronize()
+    for l in picks[:4]:
+        lin = cfg.linears[l]
+        W, A, B = u16(m.w.W_views[l]), u16(m.w.A_views[l]), u16(m.w.B_views[l])
+        for rr in sampled_rows(lin)[:2]:
+            cur = oracle.merge_linear(W, A, B, idx_ref[0], g, rows=rr)
+            Bs = np.ascontiguousarray(B[:, rr[0]:rr[1], :])           # the same rows of the B stack
+            ref = oracle.merge_linear(cur, A, Bs, list(new_i) + list(idx_ref[0]),
+                                      list(new_g.astype(np.float64)) + list(-g))
+            assert_close_bf16(u16(m.W_out[l][rr[0]:rr[1]]), ref, f"{cfg.name} switch linear {l} rows {rr}")
+    assert m.plan.status() == (0, 0)
+
 
 @pytest.mark.parametrize("cfg_fn", [synth.llama7b, synth.llama13b])
 def test_full_size_apply_sampled(am, cuda_device, cfg_fn):
