@@ -398,7 +398,7 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_fused_kernel(const __g
 // ------------------------------------------------------------------ row order
 
 // Row-order variant (k*r <= 128).  Tiles are walked along the rows of W in
-// groups of G (2 or 4) 128-row blocks, the blocks of a group interleaved
+// groups of G (2, 4 or 8) 128-row blocks, the blocks of a group interleaved
 // column block by column block: (block 0, cols 0-127), (block 1, cols 0-127),
 // ..., (block 0, cols 128-255), ...  Consecutive tiles of a CTA continue the
 // same rows of W (long contiguous DRAM runs), and the raw A rows of a
@@ -830,13 +830,13 @@ int launch_merge_fused(Plan* p, const int32_t* idx0, const float* gate0, const i
         // Row-order kernel: W stages (up to four), a ring of A tiles, and the
         // Bcat of one or two groups of G row blocks.  Preference: W stages,
         // then the group size (less A traffic), then a second group slot (the
-        // next group's Bcat built ahead), then A slots.  Groups of four only
-        // where a CTA walks enough tiles to amortise building four blocks.
+        // next group's Bcat built ahead), then A slots.  Groups of four or
+        // eight only where a CTA walks enough tiles to amortise their builds.
         const uint32_t at = (uint32_t)a.Kp * 256u, bc = at;
         const bool long_walk = p->merge_tiles >= 256 * (int64_t)p->num_sms;
         int SW = 0, NA = 0, NAR = 0, G = 0;
-        for (int g : {4, 2}) {
-            if (g == 4 && !long_walk) continue;
+        for (int g : {8, 4, 2}) {
+            if (g >= 4 && !long_walk) continue;
             for (int np : {2, 1})
                 for (int nar : {3, 2}) {
                     const int64_t room = (int64_t)kSmemMax - 2048 - (int64_t)np * g * bc - (int64_t)nar * at;
