@@ -833,7 +833,7 @@ int launch_merge_fused(Plan* p, const int32_t* idx0, const float* gate0, const i
         // next group's Bcat built ahead), then A slots.  Groups of four or
         // eight only where a CTA walks enough tiles to amortise their builds.
         const uint32_t at = (uint32_t)a.Kp * 256u, bc = at;
-        const bool long_walk = p->merge_tiles >= 256 * (int64_t)p->num_sms;
+        const bool long_walk = p->merge_tiles >= 128 * (int64_t)p->num_sms;
         int SW = 0, NA = 0, NAR = 0, G = 0;
         for (int g : {8, 4, 2}) {
             if (g >= 4 && !long_walk) continue;
