@@ -11,7 +11,8 @@
 //   2. shrink    the used experts' stacked A rows times x_l^T on the tensor
 //                cores, in 1024-column K-slices, fp32 partials to the workspace;
 //   3. finalize  slices summed in order, times each token's gate on that
-//                expert, stored as a bf16 hi/lo pair S_l[T, 2 * Kext];
+//                expert, stored as a bf16 hi/lo pair S_l[T, 2 * Kext]
+//                (hi and lo interleaved by groups of 32 columns);
 //   4. apply     one persistent tcgen05 kernel over all (linear, row block)
 //                units: D[rows x Npad] = W_block x^T (d_in/64 swizzled K chunks)
 //                then + Bcat_block S^T (the used experts' B rows, gathered by
@@ -339,10 +340,12 @@ __global__ void __launch_bounds__(kShrinkThreads, 1) shrink_tc_kernel(const __gr
 // s = coef(t, c) * (sum over the K-slices of linear l of the partials), for
 // c < U*r (zero for the padding columns up to Kext); coef(t, c) is the sum of
 // token t's gates on expert used[1 + c/r] (zero if t did not pick it).  s is
-// stored as two bf16 values, S[l, t, c] = bf16(s) and S[l, t, Kext + c] =
-// bf16(s - bf16(s)), whose sum carries s to about 2^-17 relative: the expand
-// multiplies both halves by the same B rows, so the LoRA term keeps close to
-// fp32 precision even where it cancels most of the base product.
+// stored as two bf16 values, hi = bf16(s) and lo = bf16(s - hi), whose sum
+// carries s to about 2^-17 relative: the expand multiplies both halves by the
+// same B rows, so the LoRA term keeps close to fp32 precision even where it
+// cancels most of the base product.  Row layout of S_l[t]: for each group of
+// 32 columns, its 32 hi values then its 32 lo values, so that one 64-column
+// box of S feeds both halves of an expand chunk.
 __global__ void __launch_bounds__(128) shrink_finalize_kernel(const LinDesc* lins, const float* P, const int32_t* used,
                                                                const int32_t* idx, const float* gate, uint16_t* S,
                                                                int64_t T, int32_t k, int32_t r, int32_t Kext,
@@ -380,8 +383,9 @@ __global__ void __launch_bounds__(128) shrink_finalize_kernel(const LinDesc* lin
             }
         }
         const __nv_bfloat16 hi = __float2bfloat16_rn(v);
-        Srow[c] = __bfloat16_as_ushort(hi);
-        Srow[Kext + c] = __bfloat16_as_ushort(__float2bfloat16_rn(v - __bfloat162float(hi)));
+        const int o = 64 * (c >> 5) + (c & 31);              // [hi 32 | lo 32] per 32-column group
+        Srow[o] = __bfloat16_as_ushort(hi);
+        Srow[o + 32] = __bfloat16_as_ushort(__float2bfloat16_rn(v - __bfloat162float(hi)));
     }
 }
 
@@ -477,8 +481,7 @@ __global__ void __launch_bounds__(ApplyShape<H>::kThreads, 1) apply_fused_kernel
     fence_proxy_async_smem();
     __syncthreads();
     const int U = s_used[0];
-    const int nKh = (U * a.r + kChunkK - 1) / kChunkK;     // expand chunks per half (hi, lo)
-    const int nKe = 2 * nKh;
+    const int nKe = (U * a.r + 31) / 32;                    // expand chunks: 32 columns of Bcat each
 
     if (warp == 1) {
         tmem_alloc(tmem_slot, a.tmem_cols);
@@ -528,13 +531,14 @@ __global__ void __launch_bounds__(ApplyShape<H>::kThreads, 1) apply_fused_kernel
                             tma_load_2d(dst + hh * kAChunkBytes, mW, &full[s], kc * kChunkK, m0 + hh * kTileM);
                         tma_load_2d(dst + kAChunkBytes * H, mX, &full[s], kc * kChunkK, t0);
                     } else {
-                        // expand: the hi half of S, then the lo half, each
-                        // against the same B rows of the used experts
+                        // expand: 32 columns of Bcat (the used experts' B
+                        // rows) against the hi and the lo half of S for
+                        // those columns, which sit side by side in one
+                        // 64-column box of S
                         const int ke = kc - nKb;
-                        const int half = ke >= nKh ? 1 : 0;
-                        const int col0 = (ke - half * nKh) * kChunkK;
+                        const int col0 = ke * 32;
                         int ng = 0;
-                        for (int g = 0; g < 8; ++g) if (col0 + g * 8 < U * a.r) ++ng;
+                        for (int g = 0; g < 4; ++g) if (col0 + g * 8 < U * a.r) ++ng;
                         mbar_arrive_expect_tx(&full[s], (uint32_t)(ng * H) * 2048u + xbytes);
                         for (int hh = 0; hh < H; ++hh)
                             for (int g = 0; g < ng; ++g) {
@@ -543,7 +547,7 @@ __global__ void __launch_bounds__(ApplyShape<H>::kThreads, 1) apply_fused_kernel
                                 tma_load_3d(dst + hh * kAChunkBytes + (size_t)g * 2048u, mB, &full[s], j0,
                                             m0 + hh * kTileM, s_used[1 + qq]);
                             }
-                        tma_load_3d(dst + kAChunkBytes * H, mS, &full[s], half * a.Kext + col0, t0, l);
+                        tma_load_3d(dst + kAChunkBytes * H, mS, &full[s], 2 * col0, t0, l);
                     }
                     issued = gc + 1;
                 }
@@ -583,14 +587,21 @@ __global__ void __launch_bounds__(ApplyShape<H>::kThreads, 1) apply_fused_kernel
 #pragma unroll
                     for (int hh = 0; hh < H; ++hh) {
                         const uint32_t aaddr = abase + hh * kAChunkBytes;
+                        const uint32_t d_h = d + (uint32_t)(hh * a.Npad);
+                        if (kc < nKb) {
 #pragma unroll
-                        for (int kk = 0; kk < kChunkK / 16; ++kk) {
-                            const uint64_t adesc = (kc < nKb)
-                                ? make_sdesc(aaddr + (uint32_t)kk * 32u, 16u, 1024u, kLayoutSw128)
-                                : make_sdesc(aaddr + (uint32_t)kk * 4096u, 2048u, 128u, kLayoutNone);
-                            const uint64_t bdesc = make_sdesc(baddr + (uint32_t)kk * 32u, 16u, 1024u, kLayoutSw128);
-                            tc_mma_bf16(d + (uint32_t)(hh * a.Npad), adesc, bdesc, idesc,
-                                        (kc != c0 || kk) ? 1u : 0u);
+                            for (int kk = 0; kk < kChunkK / 16; ++kk)
+                                tc_mma_bf16(d_h, make_sdesc(aaddr + (uint32_t)kk * 32u, 16u, 1024u, kLayoutSw128),
+                                            make_sdesc(baddr + (uint32_t)kk * 32u, 16u, 1024u, kLayoutSw128), idesc,
+                                            (kc != c0 || kk) ? 1u : 0u);
+                        } else {
+                            // K steps 0-1 of the S chunk hold the hi half, 2-3 the
+                            // lo half; both multiply the same 32 Bcat columns
+#pragma unroll
+                            for (int kk = 0; kk < 4; ++kk)
+                                tc_mma_bf16(d_h, make_sdesc(aaddr + (uint32_t)(kk & 1) * 4096u, 2048u, 128u, kLayoutNone),
+                                            make_sdesc(baddr + (uint32_t)kk * 32u, 16u, 1024u, kLayoutSw128), idesc,
+                                            (kc != c0 || kk) ? 1u : 0u);
                         }
                     }
                     tc_commit(&empty[s]);
