@@ -403,6 +403,7 @@ struct ApplyArgs {
     int64_t T;
     int32_t n_lin, r, Npad, n_tt, n_units, Kext, tile;
     int32_t nsplit;                 // K-splits per unit (1: no split)
+    int32_t bcols;                  // columns per B-row box of the expand: 8, 16 or 32
     float* Yp;                      // split partials [groups][nsplit][Npad][128 H] fp32
     int32_t* cnt;                   // [groups] splits finished (zeroed by the finalize kernel)
     int32_t ST;
@@ -519,6 +520,8 @@ __global__ void __launch_bounds__(ApplyShape<H>::kThreads, 1) apply_fused_kernel
                 const int t0 = tt * a.tile;
                 const CUtensorMap* mW = a.maps + (size_t)l * kMapsPerLinear + kMapW;
                 const CUtensorMap* mB = a.maps + (size_t)l * kMapsPerLinear + kMapB;
+                const CUtensorMap* mB16 = a.maps + (size_t)l * kMapsPerLinear + kMapB16;
+                const CUtensorMap* mB32 = a.maps + (size_t)l * kMapsPerLinear + kMapB32;
                 const CUtensorMap* mX = a.xmaps + l;
                 bool stop = false;
                 for (int kc = c0; kc < c1; ++kc, ++gc) {
@@ -535,16 +538,20 @@ __global__ void __launch_bounds__(ApplyShape<H>::kThreads, 1) apply_fused_kernel
                         // rows) against the hi and the lo half of S for
                         // those columns, which sit side by side in one
                         // 64-column box of S
+                        // B rows in boxes of bcols columns (one expert each:
+                        // bcols divides r), at bcols * 256 bytes per box
                         const int ke = kc - nKb;
                         const int col0 = ke * 32;
+                        const int bc = a.bcols;
+                        const CUtensorMap* mBx = bc == 32 ? mB32 : bc == 16 ? mB16 : mB;
                         int ng = 0;
-                        for (int g = 0; g < 4; ++g) if (col0 + g * 8 < U * a.r) ++ng;
-                        mbar_arrive_expect_tx(&full[s], (uint32_t)(ng * H) * 2048u + xbytes);
+                        for (int g = 0; g < 32 / bc; ++g) if (col0 + g * bc < U * a.r) ++ng;
+                        mbar_arrive_expect_tx(&full[s], (uint32_t)(ng * H * bc) * 256u + xbytes);
                         for (int hh = 0; hh < H; ++hh)
                             for (int g = 0; g < ng; ++g) {
-                                const int c = col0 + g * 8;
+                                const int c = col0 + g * bc;
                                 const int qq = c / a.r, j0 = c - qq * a.r;
-                                tma_load_3d(dst + hh * kAChunkBytes + (size_t)g * 2048u, mB, &full[s], j0,
+                                tma_load_3d(dst + hh * kAChunkBytes + (size_t)g * bc * 256u, mBx, &full[s], j0,
                                             m0 + hh * kTileM, s_used[1 + qq]);
                             }
                         tma_load_3d(dst + kAChunkBytes * H, mS, &full[s], 2 * col0, t0, l);
@@ -561,6 +568,7 @@ __global__ void __launch_bounds__(ApplyShape<H>::kThreads, 1) apply_fused_kernel
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             const uint32_t idesc = make_idesc_bf16(kTileM, (uint32_t)a.Npad, 0u, 0u);
+            const int bmode = a.bcols == 32 ? 2 : a.bcols == 16 ? 1 : 0;
             int64_t gc = 0;
             bool stop = false;
             for (int ui = 0; !stop; ++ui) {
@@ -596,12 +604,21 @@ __global__ void __launch_bounds__(ApplyShape<H>::kThreads, 1) apply_fused_kernel
                                             (kc != c0 || kk) ? 1u : 0u);
                         } else {
                             // K steps 0-1 of the S chunk hold the hi half, 2-3 the
-                            // lo half; both multiply the same 32 Bcat columns
+                            // lo half; both multiply the same 32 Bcat columns,
+                            // whose 16-column K steps sit in: two 8-column
+                            // core-matrix groups (no swizzle), one 16-column
+                            // box (32-byte swizzle) or half of a 32-column box
+                            // (64-byte swizzle)
 #pragma unroll
-                            for (int kk = 0; kk < 4; ++kk)
-                                tc_mma_bf16(d_h, make_sdesc(aaddr + (uint32_t)(kk & 1) * 4096u, 2048u, 128u, kLayoutNone),
-                                            make_sdesc(baddr + (uint32_t)kk * 32u, 16u, 1024u, kLayoutSw128), idesc,
-                                            (kc != c0 || kk) ? 1u : 0u);
+                            for (int kk = 0; kk < 4; ++kk) {
+                                const uint32_t k2 = (uint32_t)(kk & 1);
+                                const uint64_t adesc =
+                                    bmode == 0 ? make_sdesc(aaddr + k2 * 4096u, 2048u, 128u, kLayoutNone)
+                                    : bmode == 1 ? make_sdesc(aaddr + k2 * 4096u, 16u, 256u, kLayoutSw32)
+                                                 : make_sdesc(aaddr + k2 * 32u, 16u, 512u, kLayoutSw64);
+                                tc_mma_bf16(d_h, adesc, make_sdesc(baddr + (uint32_t)kk * 32u, 16u, 1024u, kLayoutSw128),
+                                            idesc, (kc != c0 || kk) ? 1u : 0u);
+                            }
                         }
                     }
                     tc_commit(&empty[s]);
@@ -840,6 +857,7 @@ int launch_apply_kernels(Plan* p, const WsLayout& w, uint8_t* wsb, const CUtenso
     a.Kext = w.Kext;
     a.tile = w.tile;
     a.nsplit = w.nsplit;
+    a.bcols = p->b_box_cols;
     a.Yp = w.nsplit > 1 ? reinterpret_cast<float*>(wsb + w.off_Yp) : nullptr;
     a.cnt = cnt;
     a.status = p->d_status;

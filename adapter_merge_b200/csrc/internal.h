@@ -32,9 +32,12 @@ struct LinDesc {
 // merge epilogue warp), A (3-D stack, 64 x a_box_rows x 1 boxes, 128-byte
 // swizzle) and, where a_box_rows == r, the A stack again in boxes of 2, 4, 8
 // and 16 whole experts (kMapARun + i holds 2 << i experts), so that a run of
-// consecutive experts moves in one load.
-constexpr int kMapsPerLinear = 9;
+// consecutive experts moves in one load; where 16 (32) divides r, the B
+// stack again in 16 x 128 boxes with 32-byte swizzle (32 x 128, 64-byte
+// swizzle) for the apply's expand.
+constexpr int kMapsPerLinear = 11;
 constexpr int kMapW = 0, kMapWout = 1, kMapB = 2, kMapWoutStore = 3, kMapA = 4, kMapARun = 5;
+constexpr int kMapB16 = 9, kMapB32 = 10;
 constexpr int kARunMaps = 4;
 // d_in columns per shrink work unit: g = 0 normally, g = 1 when the wide
 // slices leave SMs idle
@@ -66,6 +69,7 @@ struct Plan {
     int32_t total_ks[2] = {};         // shrink K-slices over all linears, per slice width
     int32_t a_box_rows = 8;           // rows per A-stack TMA box: largest power of two <= 128 dividing r
     int32_t a_run_max = 1;            // most experts one A-stack load may carry (1: no run maps)
+    int32_t b_box_cols = 8;           // columns per B-stack box of the apply's expand: 8, 16 or 32
     int2* d_apply_order[kApplyShapes] = {};      // apply units (linear, row block), longest first
     int32_t* d_sched = nullptr;         // work counters of the persistent kernels (zero between launches)
     int32_t last_launches = 0;

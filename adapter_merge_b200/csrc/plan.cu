@@ -56,14 +56,16 @@ bool encode_a(CUtensorMap* m, const void* ptr, int E, int r, int d_in, int64_t a
 
 // B stack: 3-D [E, d_out, r] bf16, box 8 (r) x 128 (rows) x 1 (expert), no swizzle:
 // one box is 16 stacked 8x8 core matrices (2 KB).
-bool encode_b(CUtensorMap* m, const void* ptr, int E, int d_out, int r, int64_t b_es)
+bool encode_b(CUtensorMap* m, const void* ptr, int E, int d_out, int r, int64_t b_es, int cols = 8)
 {
     cuuint64_t dims[3] = {(cuuint64_t)r, (cuuint64_t)d_out, (cuuint64_t)E};
     cuuint64_t strides[2] = {(cuuint64_t)r * 2, (cuuint64_t)b_es * 2};
-    cuuint32_t box[3] = {8, 128, 1};
+    cuuint32_t box[3] = {(cuuint32_t)cols, 128, 1};
     cuuint32_t estr[3] = {1, 1, 1};
+    const CUtensorMapSwizzle sw = cols == 32 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                : cols == 16 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_NONE;
     return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
-                       CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                       CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -121,6 +123,7 @@ extern "C" int adafuse_plan_create(adafuse_plan** out, const adafuse_linear* lin
     std::vector<CUtensorMap> maps((size_t)n_lin * kMapsPerLinear);
     p->a_box_rows = 8;
     while (p->a_box_rows < 128 && r % (2 * p->a_box_rows) == 0) p->a_box_rows *= 2;
+    p->b_box_cols = r % 32 == 0 ? 32 : r % 16 == 0 ? 16 : 8;
     if (p->a_box_rows == r)
         while (2 * p->a_run_max <= E && 2 * p->a_run_max * r <= kTileM &&
                2 * p->a_run_max <= (2 << (kARunMaps - 1)))
@@ -153,6 +156,13 @@ extern "C" int adafuse_plan_create(adafuse_plan** out, const adafuse_linear* lin
             !encode_w(&maps[(size_t)l * kMapsPerLinear + kMapWoutStore], L.W_out, L.d_out, L.d_in, 32) ||
             !encode_b(&maps[(size_t)l * kMapsPerLinear + kMapB], L.B, E, L.d_out, r, L.b_expert_stride) ||
             !encode_a(&maps[(size_t)l * kMapsPerLinear + kMapA], L.A, E, r, L.d_in, L.a_expert_stride, p->a_box_rows)) {
+            free_plan(p);
+            return ADAFUSE_ERR_UNSUPPORTED;
+        }
+        if ((r % 16 == 0 && !encode_b(&maps[(size_t)l * kMapsPerLinear + kMapB16], L.B, E, L.d_out, r,
+                                      L.b_expert_stride, 16)) ||
+            (r % 32 == 0 && !encode_b(&maps[(size_t)l * kMapsPerLinear + kMapB32], L.B, E, L.d_out, r,
+                                      L.b_expert_stride, 32))) {
             free_plan(p);
             return ADAFUSE_ERR_UNSUPPORTED;
         }

@@ -243,8 +243,13 @@ __device__ __forceinline__ void tc_ld_x16(uint32_t taddr, uint32_t (&v)[16])
 //             core matrices along K, sbo = along M/N.
 //   layout 2: 128-byte swizzle, K-major -- rows of 128 bytes, 8-row atoms of
 //             1024 bytes; sbo = stride between atoms, lbo unused (16).
+//   layout 4: 64-byte swizzle, K-major -- rows of 64 bytes, 8-row atoms of 512
+//             bytes; layout 6: 32-byte swizzle, rows of 32 bytes, 8-row atoms
+//             of 256 bytes (same sbo / lbo use).
 constexpr uint32_t kLayoutNone = 0;
 constexpr uint32_t kLayoutSw128 = 2;
+constexpr uint32_t kLayoutSw64 = 4;
+constexpr uint32_t kLayoutSw32 = 6;
 
 __device__ __forceinline__ uint64_t make_sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo, uint32_t layout)
 {
