@@ -198,7 +198,7 @@ ADAFUSE_API size_t adafuse_apply_workspace_bytes(const adafuse_plan* plan, int64
  * with fp32 accumulation.  Four launches, whatever the number of linears:
  * segment build (stable sort of the pairs by expert; gives the U experts the
  * batch uses), shrink (the used experts' A rows times x^T on the tensor cores,
- * split over 1024-column K-slices), finalize (slices summed in order, gates
+ * split over 1024-column K-slices, 256 for small plans), finalize (slices summed in order, gates
  * applied, kept as a pair of bf16 values whose sum is the fp32 result), then
  * one tensor-core kernel over all linears that streams W once and adds the
  * expand (the used experts' B rows against both halves of the shrink) into
@@ -212,9 +212,12 @@ ADAFUSE_API size_t adafuse_apply_workspace_bytes(const adafuse_plan* plan, int64
  * them (with the pointer tables) on `stream`; they are kept in the plan and
  * rebuilt only when the pointers, T or the workspace differ from the previous
  * call, so a serving loop that reuses its buffers does no host work beyond the
- * four launches.  Tokens are processed in tiles of 64 (T <= 64), 128
- * (T <= 128) or 256 tokens; T larger than 256 streams W once per tile.  Each row of idx should hold distinct experts (as
- * pregate's does); a repeated expert adds its gates.
+ * four launches.  The apply kernel's work units cover 512, 256 or 128 output
+ * rows with token tiles of 64, 128 or 256 (taller units for smaller T, as long
+ * as the plan has two units per SM; with fewer than one per SM, units are
+ * split along K and their fp32 partials added in a fixed order); T larger
+ * than 256 streams W once per tile.  Each row of idx should hold distinct
+ * experts (as pregate's does); a repeated expert adds its gates.
  * Errors: INVALID_ARG, WORKSPACE_TOO_SMALL, UNSUPPORTED (k < 1, k > E,
  * misaligned x_l).
  */
