@@ -158,7 +158,8 @@ def test_merge_tiny_chain_with_pregate(am, cuda_device):
 SHAPES = [(640, 392), (8, 8), (136, 1000), (256, 256), (1000, 72), (128, 136)]
 
 
-@pytest.mark.parametrize("E,r,k", [(5, 16, 2), (4, 8, 1), (8, 64, 4), (6, 32, 3), (32, 8, 2)])
+@pytest.mark.parametrize("E,r,k", [(5, 16, 2), (4, 8, 1), (8, 64, 4), (6, 32, 3), (32, 8, 2), (32, 16, 8),
+                                   (12, 48, 2)])
 def test_merge_shapes_and_ranks(am, cuda_device, E, r, k):
     cfg = synth.custom(SHAPES, E, r, k, 1, name=f"mshape{E}{r}{k}")
     m = Model(cfg, cuda_device)
@@ -298,7 +299,7 @@ def test_apply_tiny_chain_with_pregate(am, cuda_device):
 
 # T <= 64, 65..128 and > 128 take apply units of 512, 256 and 128 output rows;
 # d_out = 1000 leaves a last unit whose final 128-row block is all padding.
-@pytest.mark.parametrize("T", [1, 5, 16, 17, 64, 65, 128, 129, 130, 256, 300])
+@pytest.mark.parametrize("T", [1, 5, 16, 17, 64, 65, 128, 129, 130, 256, 300, 1000])
 def test_apply_token_counts(am, cuda_device, T):
     cfg = synth.custom([(384, 520), (136, 72), (1000, 264)], 6, 16, 2, T, name=f"aT{T}")
     m, xs, xs_dev, ys, xp, yp, idx, gate, ws = apply_setup(cfg, cuda_device, T)
@@ -306,7 +307,8 @@ def test_apply_token_counts(am, cuda_device, T):
     check_apply(m, xs, ys, idx.numpy(), gate.numpy().astype(np.float64), f"T={T}")
 
 
-@pytest.mark.parametrize("E,r,k,T", [(4, 8, 1, 16), (8, 16, 2, 64), (32, 64, 4, 128), (16, 32, 2, 32), (3, 24, 3, 9)])
+@pytest.mark.parametrize("E,r,k,T", [(4, 8, 1, 16), (8, 16, 2, 64), (32, 64, 4, 128), (16, 32, 2, 32), (3, 24, 3, 9),
+                                     (32, 16, 8, 64), (12, 48, 2, 40)])
 def test_apply_ranks(am, cuda_device, E, r, k, T):
     cfg = synth.custom([(256, 392), (520, 136)], E, r, k, T, name=f"aR{E}{r}{k}{T}")
     m, xs, xs_dev, ys, xp, yp, idx, gate, ws = apply_setup(cfg, cuda_device, T)
