@@ -404,6 +404,7 @@ struct ApplyArgs {
     int32_t n_lin, r, Npad, n_tt, n_units, Kext, tile;
     int32_t nsplit;                 // K-splits per unit (1: no split)
     int32_t bcols;                  // columns per B-row box of the expand: 8, 16 or 32
+    int32_t stall;                  // test hook: CTA 0 withholds its first stage
     float* Yp;                      // split partials [groups][nsplit][Npad][128 H] fp32
     int32_t* cnt;                   // [groups] splits finished (zeroed by the finalize kernel)
     int32_t ST;
@@ -528,7 +529,10 @@ __global__ void __launch_bounds__(ApplyShape<H>::kThreads, 1) apply_fused_kernel
                     const int s = (int)(gc % a.ST);
                     if (!mbar_wait(&empty[s], (uint32_t)((gc / a.ST) & 1) ^ 1u, abort_flag)) { stop = true; break; }
                     uint8_t* dst = base + (size_t)s * a.stage_bytes;
-                    if (kc < nKb) {
+                    if (a.stall && blockIdx.x == 0 && gc == 0) {
+                        // test hook: CTA 0 never loads its first stage, so the
+                        // MMA warp's wait on it runs out
+                    } else if (kc < nKb) {
                         mbar_arrive_expect_tx(&full[s], kAChunkBytes * H + xbytes);
                         for (int hh = 0; hh < H; ++hh)
                             tma_load_2d(dst + hh * kAChunkBytes, mW, &full[s], kc * kChunkK, m0 + hh * kTileM);
@@ -858,6 +862,7 @@ int launch_apply_kernels(Plan* p, const WsLayout& w, uint8_t* wsb, const CUtenso
     a.tile = w.tile;
     a.nsplit = w.nsplit;
     a.bcols = p->b_box_cols;
+    a.stall = (p->flags & ADAFUSE_PLAN_TEST_STALL) ? 1 : 0;
     a.Yp = w.nsplit > 1 ? reinterpret_cast<float*>(wsb + w.off_Yp) : nullptr;
     a.cnt = cnt;
     a.status = p->d_status;

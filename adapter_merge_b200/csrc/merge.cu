@@ -8,19 +8,24 @@
 // with the large product split into GEMM tiles assigned to thread blocks and a
 // prefetch buffer hiding global->shared latency.
 //
-// B200 design (one persistent CTA per SM, warp-specialised):
-//   warp 0      TMA producer: W tile (128 rows x 128 cols, two 64-column boxes,
-//               128-byte swizzle) into a W ring; the selected experts' B rows
-//               (128 x k*r, no swizzle) into a B ring.
-//   warp 1      allocates TMEM (2 x 128 fp32 columns) and issues tcgen05.mma:
-//               dW tile = Bcat[128 x Kp] * Acat[Kp x 128] into TMEM, K = k*r.
-//   warps 2-3   build Acat for a 128-column strip once per strip: gate-scaled
-//               A rows (fp32 multiply, bf16 round) in the MN-major core-matrix
-//               layout; double-buffered, reused by every row tile of the strip.
-//   warps 4-11  epilogue: each warp takes a 32-row x 64-column slice: dW from
-//               TMEM (tcgen05.ld), W from the swizzled smem tile, W + dW
-//               rounded to bf16 in place, and a TMA store of the slice.  The
-//               stage is released once all eight stores have read it.
+// B200 design: one persistent CTA per SM, warp-specialised, two variants.
+//   merge_rows_kernel (k*r <= 128, every model configuration): 128 x 128
+//     tiles walked along the rows of W in groups of 2, 4 or 8 row blocks
+//     interleaved column by column.  Warp 0 loads W tiles by TMA (two
+//     64-column boxes, 128-byte swizzle) and, once per column block of a
+//     group, the raw A rows of the selected experts (MN-major, 128-byte
+//     swizzle) that all the group's tiles share; warps 2-3 load the selected
+//     experts' B rows of the group's blocks by TMA and scale them by the
+//     gates in place (Bcat, K-major core matrices); warp 1 issues tcgen05.mma
+//     (dW = Bcat[128 x Kp] * Acat[Kp x 128], K = k*r) into one of two TMEM
+//     accumulators of 128 columns.
+//   merge_fused_kernel (k*r up to 256): tiles walked down 128-column strips;
+//     warps 2-3 build the gate-scaled A strip once per strip, the B rows of
+//     each tile come by TMA.
+//   In both, warps 4-11 are the epilogue: each warp takes a 32-row x 64-column
+//   slice: dW from TMEM (tcgen05.ld), W from the swizzled smem tile, W + dW
+//   rounded to bf16 in place, and a TMA store of the slice.  A W stage is
+//   released once the MMA and all eight stores have read it.
 // HBM traffic is W read + W' write (4 bytes per element) plus the selected
 // adapters; the tensor cores carry the rank-(k*r) contraction (16*k*r/4 FLOP/B).
 #include <algorithm>

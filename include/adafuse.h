@@ -67,12 +67,12 @@ typedef struct CUstream_st* adafuse_stream_t;   /* same type as cudaStream_t */
 #define ADAFUSE_POOL_MEAN  (1u << 1)   /* pregate: one decision for the mean of the T rows */
 
 /* ---- plan flags ---- */
-/* Test hook for the failure path: every fused merge or switch on a plan
- * created with this flag withholds the first shared-memory stage of CTA 0, so
- * that CTA's pipeline wait runs out (after about 1.5 s) instead of the data
- * arriving.  The launch then completes with ADAFUSE_STATUS_TIMEOUT set and
- * W_out incomplete, while the GPU context stays usable.  Never set it outside
- * tests. */
+/* Test hook for the failure path: every fused merge, switch or apply on a
+ * plan created with this flag withholds the first shared-memory stage of CTA 0
+ * of the merge or of the fused apply kernel, so that CTA's pipeline wait runs
+ * out (after about 1.5 s) instead of the data arriving.  The launch then
+ * completes with ADAFUSE_STATUS_TIMEOUT set and W_out (or y) incomplete, while
+ * the GPU context stays usable.  Never set it outside tests. */
 #define ADAFUSE_PLAN_TEST_STALL  (1u << 31)
 
 /* ---- device status bits (adafuse_plan_status) ---- */

@@ -1,6 +1,6 @@
 """Failure detection on the GPU without a fault: a plan created with the
 ADAFUSE_PLAN_TEST_STALL hook withholds one shared-memory stage in CTA 0 of the
-fused merge, so that a pipeline wait runs out.  The kernel must give up after
+fused merge (or of the fused apply), so that a pipeline wait runs out.  The kernel must give up after
 its bounded wait, free its resources, report ADAFUSE_STATUS_TIMEOUT through the
 status word, and leave the context usable for the next (normal) launch."""
 import time
@@ -50,3 +50,36 @@ def test_stalled_merge_times_out_and_reports(am, cuda_device):
     for l in range(cfg.n_lin):
         ref = oracle.merge_linear(u16(w.W_views[l]), u16(w.A_views[l]), u16(w.B_views[l]), [1, 3], [0.5, 0.25])
         assert_close_bf16(u16(m.W_out[l]), ref, f"after timeout, linear {l}")
+
+
+def test_stalled_apply_times_out_and_reports(am, cuda_device):
+    T = 24
+    cfg = synth.custom([(512, 384), (256, 136)], 4, 16, 2, T, name="stall-apply")
+    w = synth.make_weights(cfg, 1, device=cuda_device)
+    W_out = [torch.zeros_like(t) for t in w.W_views]
+    X, xs = synth.make_apply_inputs(cfg, T, 2, device=cuda_device)
+    ys = [torch.zeros((T, l.d_out), dtype=torch.bfloat16, device=cuda_device) for l in cfg.linears]
+    idx, gate = synth.random_selection(T, cfg.E, cfg.k, 3, "stall-apply")
+    idx, gate = idx.to(cuda_device), gate.to(cuda_device)
+    plan = am.Plan(list(zip(w.W_views, W_out, w.A_views, w.B_views)), cfg.E, cfg.r, flags=am.PLAN_TEST_STALL)
+    ws = torch.empty(plan.workspace_bytes(T, cfg.k), dtype=torch.uint8, device=cuda_device)
+    t0 = time.time()
+    plan.apply(xs, ys, T, idx, gate, ws)
+    rc, st = plan.status()                     # synchronises
+    elapsed = time.time() - t0
+    assert rc == am.ERR_TIMEOUT
+    assert st & am.STATUS_TIMEOUT
+    assert elapsed < 60
+    assert plan.status() == (0, 0)
+    plan.destroy()
+
+    # the context and the shared work counters are still usable: a normal
+    # plan's apply on the same workspace matches the oracle
+    m = Model(cfg, cuda_device, weights=w)
+    m.plan.apply(xs, ys, T, idx, gate, ws)
+    torch.cuda.synchronize()
+    assert m.plan.status() == (0, 0)
+    for l in range(cfg.n_lin):
+        ref = oracle.apply_linear(u16(xs[l]), u16(w.W_views[l]), u16(w.A_views[l]), u16(w.B_views[l]),
+                                  idx.cpu().numpy(), gate.cpu().numpy().astype(np.float64))
+        assert_close_bf16(u16(ys[l]), ref, f"after apply timeout, linear {l}")
