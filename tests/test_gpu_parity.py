@@ -159,7 +159,7 @@ SHAPES = [(640, 392), (8, 8), (136, 1000), (256, 256), (1000, 72), (128, 136)]
 
 
 @pytest.mark.parametrize("E,r,k", [(5, 16, 2), (4, 8, 1), (8, 64, 4), (6, 32, 3), (32, 8, 2), (32, 16, 8),
-                                   (12, 48, 2)])
+                                   (12, 48, 2), (1, 16, 1), (4, 256, 1)])
 def test_merge_shapes_and_ranks(am, cuda_device, E, r, k):
     cfg = synth.custom(SHAPES, E, r, k, 1, name=f"mshape{E}{r}{k}")
     m = Model(cfg, cuda_device)
@@ -308,7 +308,7 @@ def test_apply_token_counts(am, cuda_device, T):
 
 
 @pytest.mark.parametrize("E,r,k,T", [(4, 8, 1, 16), (8, 16, 2, 64), (32, 64, 4, 128), (16, 32, 2, 32), (3, 24, 3, 9),
-                                     (32, 16, 8, 64), (12, 48, 2, 40)])
+                                     (32, 16, 8, 64), (12, 48, 2, 40), (1, 16, 1, 7), (4, 256, 1, 20)])
 def test_apply_ranks(am, cuda_device, E, r, k, T):
     cfg = synth.custom([(256, 392), (520, 136)], E, r, k, T, name=f"aR{E}{r}{k}{T}")
     m, xs, xs_dev, ys, xp, yp, idx, gate, ws = apply_setup(cfg, cuda_device, T)
