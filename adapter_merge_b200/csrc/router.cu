@@ -34,6 +34,11 @@ __device__ __forceinline__ void cp_async_4(uint32_t dst, const void* src)
     asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
 }
 
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+
 // Is (c1, z1, e1) ranked before (c0, z0, e0)?  Class 0 = finite or infinite
 // logit, 1 = NaN, 2 = no expert / already taken.
 __device__ __forceinline__ bool ranks_before(int c1, float z1, int e1, int c0, float z0, int e0)
@@ -51,7 +56,7 @@ __host__ __device__ constexpr int stage_floats(int E) { return E * kRowPad + kCh
 __global__ void __launch_bounds__(kRouterThreads) pregate_kernel(const uint16_t* x, int64_t T, int32_t H,
                                                                   int64_t ldx, const float* Wr, const float* br,
                                                                   int32_t E, int32_t k, uint32_t flags,
-                                                                  int32_t* idx, float* gate, int xfull)
+                                                                  int32_t* idx, float* gate, int xfull, int w16)
 {
     extern __shared__ float rsm[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -66,9 +71,17 @@ __global__ void __launch_bounds__(kRouterThreads) pregate_kernel(const uint16_t*
             float* ws = rsm + (c % kStages) * SF;
             const int j0 = c * kChunk;
             const int n = min(kChunk, H - j0);
-            for (int id = tid; id < E * kChunk; id += kRouterThreads) {
-                const int e = id / kChunk, jj = id - e * kChunk;
-                if (jj < n) cp_async_4(smem_u32(ws + e * kRowPad + jj), Wr + (int64_t)e * H + j0 + jj);
+            if (w16) {
+                // 16-byte copies: W_r rows start on 16-byte boundaries (H % 4 == 0)
+                for (int id = tid; id < E * (kChunk / 4); id += kRouterThreads) {
+                    const int e = id / (kChunk / 4), jj = (id - e * (kChunk / 4)) * 4;
+                    if (jj < n) cp_async_16(smem_u32(ws + e * kRowPad + jj), Wr + (int64_t)e * H + j0 + jj);
+                }
+            } else {
+                for (int id = tid; id < E * kChunk; id += kRouterThreads) {
+                    const int e = id / kChunk, jj = id - e * kChunk;
+                    if (jj < n) cp_async_4(smem_u32(ws + e * kRowPad + jj), Wr + (int64_t)e * H + j0 + jj);
+                }
             }
         }
         asm volatile("cp.async.commit_group;" ::: "memory");
@@ -195,6 +208,7 @@ extern "C" int adafuse_pregate(const void* x, int64_t T, int32_t H, int64_t x_ro
         cudaFuncSetAttribute(af::pregate_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return ADAFUSE_ERR_CUDA;
     af::pregate_kernel<<<grid, af::kRouterThreads, smem, (cudaStream_t)stream>>>(
-        static_cast<const uint16_t*>(x), T, H, x_row_stride, W_r, b_r, E, k, flags, idx, gate, xfull);
+        static_cast<const uint16_t*>(x), T, H, x_row_stride, W_r, b_r, E, k, flags, idx, gate, xfull,
+        (H % 4 == 0 && (reinterpret_cast<uintptr_t>(W_r) & 15u) == 0) ? 1 : 0);
     return af::cuda_err(cudaGetLastError());
 }
