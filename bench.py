@@ -514,13 +514,25 @@ def main():
     # selection crossing PCIe.
     e2e = None
     if not args.no_e2e:
-        h_W = torch.empty(w.W.shape, dtype=w.W.dtype, pin_memory=True)
-        h_W.copy_(w.W)
-        h_A = torch.empty(w.A.shape, dtype=w.A.dtype, pin_memory=True)
-        h_A.copy_(w.A)
-        h_B = torch.empty(w.B.shape, dtype=w.B.dtype, pin_memory=True)
-        h_B.copy_(w.B)
-        h_Wout = torch.empty(W_out.shape, dtype=W_out.dtype, pin_memory=True)
+        # The full-weight form pins a host copy of W, A, B and W' per rank;
+        # every rank takes the same decision (collectives stay in step).
+        need = (w.W.numel() + w.A.numel() + w.B.numel() + W_out.numel()) * 2
+        local_world = int(os.environ.get("LOCAL_WORLD_SIZE", str(world)))
+        try:
+            import psutil
+            avail = psutil.virtual_memory().available
+        except Exception:
+            avail = None
+        fits = 1.0 if avail is None or avail > 1.25 * need * local_world else 0.0
+        full = -max_over_ranks([-fits], dist, dev)[0] > 0.5
+        if full:
+            h_W = torch.empty(w.W.shape, dtype=w.W.dtype, pin_memory=True)
+            h_W.copy_(w.W)
+            h_A = torch.empty(w.A.shape, dtype=w.A.dtype, pin_memory=True)
+            h_A.copy_(w.A)
+            h_B = torch.empty(w.B.shape, dtype=w.B.dtype, pin_memory=True)
+            h_B.copy_(w.B)
+            h_Wout = torch.empty(W_out.shape, dtype=W_out.dtype, pin_memory=True)
         h_xreq = x_req.cpu().pin_memory()
         h_first = x_first.cpu().pin_memory()
         h_X = X.cpu().pin_memory()
@@ -564,12 +576,16 @@ def main():
             torch.cuda.synchronize()
             return mean([e[0].elapsed_time(e[1]) for e in evs_])
 
-        em_m, em_a, em_r = max_over_ranks([timed(e2e_merge, ne, False), timed(e2e_apply, 10),
-                                           timed(e2e_merge, 10, True)], dist, dev)
+        em_m = timed(e2e_merge, ne, False) if full else 0.0
+        em_m, em_a, em_r = max_over_ranks([em_m, timed(e2e_apply, 10), timed(e2e_merge, 10, True)], dist, dev)
         h2d_m = (w.W.numel() + w.A.numel() + w.B.numel() + x_req.numel()) * 2
         d2h_m = W_out.numel() * 2 + 2 * cfg.k * 4
         h2d_a = (x_first.numel() + X.numel()) * 2
         d2h_a = Y.numel() * 2 + cfg.k * 4
+        if not full:        # host memory too small for a pinned model copy per rank
+            em_m = em_r
+            h2d_m = x_req.numel() * 2
+            d2h_m = 2 * cfg.k * 4
         e2e = {"value": round(job_throughput(world, mb, em_m), 3), "unit": "GB/s",
                "h2d_bytes_per_step": h2d_m + h2d_a, "d2h_bytes_per_step": d2h_m + d2h_a,
                "merge_ms": round(em_m, 3), "merge_h2d_bytes": h2d_m, "merge_d2h_bytes": d2h_m,
@@ -578,9 +594,12 @@ def main():
                "resident": {"value": round(job_throughput(world, mb, em_r), 2), "unit": "GB/s",
                             "h2d_bytes_per_step": x_req.numel() * 2, "d2h_bytes_per_step": 2 * cfg.k * 4,
                             "note": "weights and adapters resident; only the router input and the selection cross"},
-               "note": "merge with W, A, B in and W' out through pinned host buffers each step; apply with "
-                       "x in and y out (weights resident)"}
-        del h_W, h_A, h_B, h_Wout
+               "note": ("merge with W, A, B in and W' out through pinned host buffers each step; apply with "
+                        "x in and y out (weights resident)") if full else
+                       ("host memory holds no pinned model copy per rank: merge with the router input in and "
+                        "the selection out (weights resident); apply with x in and y out")}
+        if full:
+            del h_W, h_A, h_B, h_Wout
 
     # The NEXT rows on the same plan, outside the timed region: in-place switch
     # between two selections (rank 2kr), the one-launch-per-linear merge, and
