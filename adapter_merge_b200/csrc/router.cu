@@ -58,6 +58,8 @@ __global__ void __launch_bounds__(kRouterThreads) pregate_kernel(const uint16_t*
                                                                   int32_t E, int32_t k, uint32_t flags,
                                                                   int32_t* idx, float* gate, int xfull, int w16)
 {
+    // xfull: 0 = x staged chunk by chunk, 1 = whole x row first, 2 = whole
+    // W_r and whole x row first (no ring, no per-chunk barriers).
     extern __shared__ float rsm[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const bool pool = (flags & ADAFUSE_POOL_MEAN) != 0;
@@ -106,6 +108,44 @@ __global__ void __launch_bounds__(kRouterThreads) pregate_kernel(const uint16_t*
         }
     };
 
+    float z = 0.f;
+    if (xfull == 2) {
+        // W_r rows padded to H + 4 floats (16-byte aligned, lanes 4 banks apart)
+        const int Hp = H + 4;
+        float* wall = rsm;
+        float* xall = rsm + (size_t)E * Hp;
+        for (int id = tid; id < E * (H / 4); id += kRouterThreads) {
+            const int e = id / (H / 4), jj = (id - e * (H / 4)) * 4;
+            cp_async_16(smem_u32(wall + (size_t)e * Hp + jj), Wr + (int64_t)e * H + jj);
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+#pragma unroll 8
+        for (int j = tid; j < H; j += kRouterThreads) xall[j] = bf16_at(x + t * ldx + j);
+        asm volatile("cp.async.wait_group 0;" ::: "memory");
+        __syncthreads();
+        if (warp != 0) return;
+        if (lane < E) {
+            const float* ws = wall + (size_t)lane * Hp;
+            const int n4 = H & ~15;
+            // Same order as the scalar loop: one product, one add, ascending j.
+            for (int jj = 0; jj < n4; jj += 16) {
+                float4 xv[4], wv[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    xv[u] = *reinterpret_cast<const float4*>(xall + jj + 4 * u);
+                    wv[u] = *reinterpret_cast<const float4*>(ws + jj + 4 * u);
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    z = __fadd_rn(z, __fmul_rn(xv[u].x, wv[u].x));
+                    z = __fadd_rn(z, __fmul_rn(xv[u].y, wv[u].y));
+                    z = __fadd_rn(z, __fmul_rn(xv[u].z, wv[u].z));
+                    z = __fadd_rn(z, __fmul_rn(xv[u].w, wv[u].w));
+                }
+            }
+            for (int jj = n4; jj < H; ++jj) z = __fadd_rn(z, __fmul_rn(xall[jj], ws[jj]));
+        }
+    } else {
     float* xall = rsm + kStages * SF;          // [H] when xfull
     for (int c = 0; c < kStages - 1; ++c) issue_w(c);
     if (xfull) {
@@ -114,7 +154,6 @@ __global__ void __launch_bounds__(kRouterThreads) pregate_kernel(const uint16_t*
     } else {
         load_x(0, tid, kRouterThreads);
     }
-    float z = 0.f;
     for (int c = 0; c < nchunks; ++c) {
         issue_w(c + kStages - 1);
         asm volatile("cp.async.wait_group %0;" ::"n"(kStages - 1) : "memory");
@@ -147,6 +186,7 @@ __global__ void __launch_bounds__(kRouterThreads) pregate_kernel(const uint16_t*
             load_x(c + 1, tid - 32, kRouterThreads - 32);
         }
         __syncthreads();                       // stage c % kStages may be refilled
+    }
     }
     if (warp != 0) return;
 
@@ -200,15 +240,17 @@ extern "C" int adafuse_pregate(const void* x, int64_t T, int32_t H, int64_t x_ro
     const bool pool = (flags & ADAFUSE_POOL_MEAN) != 0;
     if (!pool && T > 0x7fffffff) return ADAFUSE_ERR_UNSUPPORTED;
     const unsigned grid = pool ? 1u : (unsigned)T;
+    const int w16 = (H % 4 == 0 && (reinterpret_cast<uintptr_t>(W_r) & 15u) == 0) ? 1 : 0;
     size_t smem = sizeof(float) * af::kStages * af::stage_floats(E);
     const size_t smem_x = smem + sizeof(float) * (size_t)H;
-    const int xfull = (!pool && smem_x <= 200 * 1024) ? 1 : 0;
-    if (xfull) smem = smem_x;
+    const size_t smem_all = sizeof(float) * ((size_t)E * (H + 4) + (size_t)H);
+    int xfull = 0;
+    if (!pool && w16 && smem_all <= 200 * 1024) { xfull = 2; smem = smem_all; }      // whole W_r and x
+    else if (!pool && smem_x <= 200 * 1024) { xfull = 1; smem = smem_x; }            // whole x row
     if (smem > 48 * 1024 &&
         cudaFuncSetAttribute(af::pregate_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return ADAFUSE_ERR_CUDA;
     af::pregate_kernel<<<grid, af::kRouterThreads, smem, (cudaStream_t)stream>>>(
-        static_cast<const uint16_t*>(x), T, H, x_row_stride, W_r, b_r, E, k, flags, idx, gate, xfull,
-        (H % 4 == 0 && (reinterpret_cast<uintptr_t>(W_r) & 15u) == 0) ? 1 : 0);
+        static_cast<const uint16_t*>(x), T, H, x_row_stride, W_r, b_r, E, k, flags, idx, gate, xfull, w16);
     return af::cuda_err(cudaGetLastError());
 }
