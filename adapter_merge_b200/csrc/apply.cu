@@ -9,7 +9,8 @@
 //   1. segments  stable sort of the (token, slot) pairs by expert (segments.cu);
 //                gives the U experts the batch uses;
 //   2. shrink    the used experts' stacked A rows times x_l^T on the tensor
-//                cores, in 1024-column K-slices, fp32 partials to the workspace;
+//                cores, in 1024-column K-slices (256 for small plans), fp32
+//                partials to the workspace;
 //   3. finalize  slices summed in order, times each token's gate on that
 //                expert, stored as a bf16 hi/lo pair S_l[T, 2 * Kext]
 //                (hi and lo interleaved by groups of 32 columns);
@@ -19,7 +20,9 @@
 //                TMA, against both halves of S), all into one fp32 TMEM
 //                accumulator, then y = bf16(D^T).  A unit covers 128, 256 or
 //                512 output rows (taller for smaller T), whose MMAs share each
-//                staged x chunk.
+//                staged x chunk; below one unit per SM, units are split along
+//                K and the last split of each 32-row slice adds the fp32
+//                partials in split order.
 // Every operand moves by TMA: W and the experts' A and B rows through the
 // plan's tensor maps, x and S through per-call maps that the host builds (and
 // caches by pointer set, T and workspace) before the launches.  W is streamed
@@ -118,10 +121,12 @@ constexpr uint32_t kAChunkBytes = kTileM * kChunkK * 2;     // 16 KB: 128 rows x
 // ------------------------------------------------------------------ shrink
 //
 // S^T = Acat x^T for every linear, on the tensor cores: Acat stacks the A rows
-// of the U used experts (U*r rows, gathered by TMA in 8-row boxes), x^T is the
-// token tile.  Work units are (128-row tile of Acat, 1024-column K-slice of a
-// linear); each unit writes its fp32 partial [Npad x 128] to the workspace and
-// the finalize kernel adds the slices in order, applies the gates and rounds.
+// of the U used experts (U*r rows, gathered by TMA: boxes of 2-16 whole experts
+// for runs of consecutive expert ids where r is a power of two, else boxes of
+// up to 128 rows of one expert), x^T is the token tile.  Work units are
+// (128-row tile of Acat, K-slice of a linear); each unit writes its fp32
+// partial [Npad x 128] to the workspace and the finalize kernel adds the slices
+// in order, applies the gates and rounds.
 
 struct ShrinkArgs {
     const LinDesc* lins;
