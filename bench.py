@@ -53,13 +53,15 @@ def profiled_traffic(kernel_files, summary, key):
     if not os.path.exists(path):
         return None
     rec = {}
-    for line in open(path):
-        parts = line.strip().split(":")
-        if len(parts) == 2:
-            rec[parts[0].strip()] = parts[1].strip()
+    with open(path) as fh:
+        for line in fh:
+            parts = line.strip().split(":")
+            if len(parts) == 2:
+                rec[parts[0].strip()] = parts[1].strip()
     h = hashlib.sha256()
     for f in kernel_files:
-        h.update(open(os.path.join(ROOT, "adapter_merge_b200", "csrc", f), "rb").read())
+        with open(os.path.join(ROOT, "adapter_merge_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
     if rec.get("kernel_sources_sha256_16") != h.hexdigest()[:16] or key not in rec:
         return None
     return int(rec[key])
@@ -121,22 +123,25 @@ class ClockSampler:
 
     def stop(self):
         if self.proc is None:
+            self.f.close()
+            os.unlink(self.f.name)
             return None
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
         except subprocess.TimeoutExpired:
             self.proc.kill()
-        self.f.flush()
+        self.f.close()
         rows = []
-        for line in open(self.f.name):
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[5:9]))
-            except ValueError:
-                continue
+        with open(self.f.name) as fh:
+            for line in fh:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[5:9]))
+                except ValueError:
+                    continue
         os.unlink(self.f.name)
         if not rows:
             return None

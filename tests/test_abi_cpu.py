@@ -20,7 +20,8 @@ def L():
 
 
 def declared_functions():
-    src = open(HEADER).read()
+    with open(HEADER) as f:
+        src = f.read()
     return sorted(set(re.findall(r"ADAFUSE_API\s+[\w\s\*]+?\b(adafuse_\w+)\s*\(", src)))
 
 

@@ -40,7 +40,8 @@ MUTANTS = {
 @pytest.mark.parametrize("name", sorted(MUTANTS))
 def test_pins_catch_planted_mistake(name, tmp_path):
     pat, rep = MUTANTS[name]
-    src = open(SRC).read()
+    with open(SRC) as f:
+        src = f.read()
     mutated, n = re.subn(pat, lambda m: rep, src, count=1)
     assert n == 1, f"mutation {name} did not apply"
     csrc = tmp_path / "mutant.c"

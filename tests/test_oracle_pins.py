@@ -22,6 +22,11 @@ import oracle
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "handworked.json")
 
 
+def _golden():
+    with open(GOLDEN) as f:
+        return json.load(f)
+
+
 def bits(a) -> np.ndarray:
     """float values exactly representable in bf16 -> uint16 bit patterns."""
     t = torch.as_tensor(np.asarray(a, dtype=np.float32)).to(torch.bfloat16)
@@ -109,7 +114,7 @@ def test_bf16_rounding_single_step_from_double():
 # ----------------------------------------------------------------- router
 
 def test_router_handworked():
-    g = json.load(open(GOLDEN))
+    g = _golden()
     for key in ("router", "router_tie"):
         c = g[key]
         x = bits(np.array(c["x"], dtype=np.float32)[None, :])
@@ -250,7 +255,7 @@ def test_pregate_pool_routes_the_mean_row():
 # ------------------------------------------------------------------ merge
 
 def test_merge_handworked():
-    c = json.load(open(GOLDEN))["merge"]
+    c = _golden()["merge"]
     W = bits(np.array(c["W"])); A = bits(np.array(c["A"])); B = bits(np.array(c["B"]))
     out = oracle.merge_linear(W, A, B, c["idx"], c["gate"])
     assert np.array_equal(vals(out), np.array(c["W_out"]))
@@ -341,7 +346,7 @@ def test_switch_is_merge_with_negated_previous_gates():
 # ------------------------------------------------------------------ apply
 
 def test_apply_handworked():
-    g = json.load(open(GOLDEN))
+    g = _golden()
     m, c = g["merge"], g["apply"]
     y = oracle.apply_linear(bits(np.array(c["x"])), bits(np.array(m["W"])), bits(np.array(m["A"])),
                             bits(np.array(m["B"])), np.array(c["idx"]), np.array(c["gate"]))
@@ -402,7 +407,7 @@ def test_apply_zero_gates_is_base_gemm():
 # -------------------------------------------------------------- segments
 
 def test_segments_handworked_and_stable_sort():
-    c = json.load(open(GOLDEN))["segments"]
+    c = _golden()["segments"]
     off, perm, bad = oracle.segments(np.array(c["idx"]), c["E"])
     assert off.tolist() == c["offsets"] and perm.tolist() == c["perm"] and bad == 0
     rng = np.random.default_rng(20)
