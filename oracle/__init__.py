@@ -92,7 +92,9 @@ def max_threads() -> int:
 
 def bf16_to_f64(bits: np.ndarray) -> np.ndarray:
     bits = _u16(bits)
-    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    # signalling-NaN patterns widen to quiet NaNs; numpy flags that as "invalid"
+    with np.errstate(invalid="ignore"):
+        return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
 
 
 def bf16_from_f64(v: np.ndarray) -> np.ndarray:
