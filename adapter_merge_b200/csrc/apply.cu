@@ -185,11 +185,13 @@ __global__ void __launch_bounds__(kShrinkThreads, 1) shrink_tc_kernel(const __gr
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (threadIdx.x <= kMaxE) s_used[threadIdx.x] = a.used[threadIdx.x];
     for (int s = 0; s < a.ST; ++s)
         for (uint32_t o = threadIdx.x * 16; o < kAChunkBytes; o += kShrinkThreads * 16)
             st_shared_v4(smem_u32(base + (size_t)s * a.stage_bytes + o), make_uint4(0, 0, 0, 0));
     fence_proxy_async_smem();
+    griddep_wait();
+    griddep_launch_dependents();
+    if (threadIdx.x <= kMaxE) s_used[threadIdx.x] = a.used[threadIdx.x];
     __syncthreads();
     const int rows = s_used[0] * a.r;          // live rows of Acat
     if (warp == 1) {
@@ -358,6 +360,8 @@ __global__ void __launch_bounds__(128) shrink_finalize_kernel(const LinDesc* lin
                                                                int32_t total_ks, int32_t ksg, int32_t* cnt,
                                                                int32_t n_cnt)
 {
+    griddep_wait();
+    griddep_launch_dependents();
     // The apply kernel's split counters start from zero on every call.
     if (blockIdx.x == 0 && blockIdx.y == 0)
         for (int i = threadIdx.x; i < n_cnt; i += blockDim.x) cnt[i] = 0;
@@ -480,12 +484,14 @@ __global__ void __launch_bounds__(ApplyShape<H>::kThreads, 1) apply_fused_kernel
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (threadIdx.x <= kMaxE) s_used[threadIdx.x] = a.used[threadIdx.x];
     // Zero the A regions: expert chunks load only the 8-column groups they use.
     for (int s = 0; s < a.ST; ++s)
         for (uint32_t o = threadIdx.x * 16; o < kAChunkBytes * H; o += kApplyThreads * 16)
             st_shared_v4(smem_u32(base + (size_t)s * a.stage_bytes + o), make_uint4(0, 0, 0, 0));
     fence_proxy_async_smem();
+    griddep_wait();
+    griddep_launch_dependents();
+    if (threadIdx.x <= kMaxE) s_used[threadIdx.x] = a.used[threadIdx.x];
     __syncthreads();
     const int U = s_used[0];
     const int nKe = (U * a.r + 31) / 32;                    // expand chunks: 32 columns of Bcat each
@@ -786,8 +792,7 @@ int launch_apply_fused(const ApplyArgs& a, uint32_t smem, int grid, cudaStream_t
     if (cudaFuncSetAttribute(apply_fused_kernel<H>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
         cudaSuccess)
         return ADAFUSE_ERR_CUDA;
-    apply_fused_kernel<H><<<grid, ApplyShape<H>::kThreads, smem, s>>>(a);
-    return cuda_err(cudaGetLastError());
+    return launch_pdl(apply_fused_kernel<H>, dim3(grid), dim3(ApplyShape<H>::kThreads), smem, s, a);
 }
 
 int launch_apply_kernels(Plan* p, const WsLayout& w, uint8_t* wsb, const CUtensorMap* xmaps, void* const* yp,
@@ -839,12 +844,13 @@ int launch_apply_kernels(Plan* p, const WsLayout& w, uint8_t* wsb, const CUtenso
         if (cudaFuncSetAttribute(shrink_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
             cudaSuccess)
             return ADAFUSE_ERR_CUDA;
-        shrink_tc_kernel<<<(int)std::min<int64_t>(p->num_sms, w.n_su * w.n_tt), kShrinkThreads, smem, s>>>(sa);
-        if (cudaGetLastError() != cudaSuccess) return ADAFUSE_ERR_CUDA;
-        shrink_finalize_kernel<<<dim3((unsigned)p->n_lin, (unsigned)T), 128, 0, s>>>(
-            p->d_desc, P, used, idx, gate, S, T, k, p->r, w.Kext, Npad, w.tile, w.n_su, w.total_ks, w.ksg, cnt,
-            n_cnt);
-        if (cudaGetLastError() != cudaSuccess) return ADAFUSE_ERR_CUDA;
+        rc = launch_pdl(shrink_tc_kernel, dim3((unsigned)std::min<int64_t>(p->num_sms, w.n_su * w.n_tt)),
+                        dim3(kShrinkThreads), smem, s, sa);
+        if (rc != ADAFUSE_OK) return rc;
+        rc = launch_pdl(shrink_finalize_kernel, dim3((unsigned)p->n_lin, (unsigned)T), dim3(128), 0, s,
+                        (const LinDesc*)p->d_desc, (const float*)P, (const int32_t*)used, idx, gate, S, T, k, p->r,
+                        w.Kext, Npad, w.tile, w.n_su, w.total_ks, w.ksg, cnt, n_cnt);
+        if (rc != ADAFUSE_OK) return rc;
     }
 
     // Accumulators: two of H * Npad columns (Npad <= 256 / H).

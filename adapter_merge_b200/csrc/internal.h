@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
 #include <vector>
 
 #include "adafuse.h"
@@ -101,5 +102,26 @@ int launch_apply(Plan* p, const void* const* x_ptrs, void* const* y_ptrs, int64_
                  const float* gate, int32_t k, void* ws, size_t ws_bytes, cudaStream_t s);
 
 inline int cuda_err(cudaError_t e) { return e == cudaSuccess ? ADAFUSE_OK : ADAFUSE_ERR_CUDA; }
+
+// Launches a kernel with programmatic stream serialization, so that its
+// launch and shared-memory prologue overlap the tail of the previous kernel
+// in the stream.  Only for kernels that call griddep_wait() before any
+// access to global memory or TMEM.
+template <typename... Params, typename... Args>
+inline int launch_pdl(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                      Args&&... args)
+{
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cuda_err(cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...));
+}
 
 }  // namespace af

@@ -121,6 +121,33 @@ __device__ __forceinline__ uint32_t add_bf16x2(uint32_t w, uint32_t d0, uint32_t
     return pack_bf16x2(bf16lo(w) + __uint_as_float(d0), bf16hi(w) + __uint_as_float(d1));
 }
 
+// The selection into shared memory (one thread): s_e / s_g per slot, the old
+// selection negated in switch mode; out-of-range expert ids become zero-gate
+// empty slots and are flagged.  *s_skip = 1 for a switch between identical
+// selections.
+__device__ void read_selection(const MergeArgs& a, int* s_e, float* s_g, int* s_skip)
+{
+    int bad = 0;
+    int same = 1;
+    for (int s = 0; s < a.ns; ++s) {
+        int e;
+        float g;
+        if (s < a.k) { e = a.idx0[s]; g = a.gate0[s]; }
+        else { e = a.idx1[s - a.k]; g = -a.gate1[s - a.k]; }
+        if (e < 0 || e >= a.E) { bad = 1; e = -1; g = 0.f; }
+        s_e[s] = e;
+        s_g[s] = g;
+    }
+    if (a.mode == 1) {
+        for (int s = 0; s < a.k; ++s)
+            if (a.idx0[s] != a.idx1[s] || __float_as_uint(a.gate0[s]) != __float_as_uint(a.gate1[s])) same = 0;
+    } else {
+        same = 0;
+    }
+    *s_skip = same;
+    if (bad && blockIdx.x == 0) atomicOr(a.status, ADAFUSE_STATUS_BAD_INDEX);
+}
+
 __global__ void __launch_bounds__(kMergeThreads, 1) merge_fused_kernel(const __grid_constant__ MergeArgs a)
 {
     extern __shared__ uint8_t smem_raw[];
@@ -155,31 +182,15 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_fused_kernel(const __g
         for (int i = 0; i < 2; ++i) { mbar_init(&accfull[i], 1); mbar_init(&accempty[i], kEpiWarps); }
         mbar_init(donebar, 1);
         *abort_flag = 0;
-        int bad = 0;
-        int same = 1;
-        for (int s = 0; s < a.ns; ++s) {
-            int e;
-            float g;
-            if (s < a.k) { e = a.idx0[s]; g = a.gate0[s]; }
-            else { e = a.idx1[s - a.k]; g = -a.gate1[s - a.k]; }
-            if (e < 0 || e >= a.E) { bad = 1; e = -1; g = 0.f; }
-            s_e[s] = e;
-            s_g[s] = g;
-        }
-        if (a.mode == 1) {
-            for (int s = 0; s < a.k; ++s)
-                if (a.idx0[s] != a.idx1[s] || __float_as_uint(a.gate0[s]) != __float_as_uint(a.gate1[s])) same = 0;
-        } else {
-            same = 0;
-        }
-        *s_skip = same;
-        if (bad && blockIdx.x == 0) atomicOr(a.status, ADAFUSE_STATUS_BAD_INDEX);
         fence_mbar_init();
     }
     // Zero the B ring: stages of skipped slots and the K padding stay zero.
     for (uint32_t o = threadIdx.x * 16; o < (uint32_t)a.SB * BBytes; o += kMergeThreads * 16)
         st_shared_v4(smem_u32(sB + o), make_uint4(0, 0, 0, 0));
     fence_proxy_async_smem();
+    griddep_wait();
+    griddep_launch_dependents();
+    if (threadIdx.x == 0) read_selection(a, s_e, s_g, s_skip);
     __syncthreads();
     if (*s_skip) return;       // switch between identical selections: nothing to do
 
@@ -503,25 +514,6 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_rows_kernel(const __gr
         for (int i = 0; i < 2; ++i) { mbar_init(&accfull[i], 1); mbar_init(&accempty[i], kEpiWarps); }
         mbar_init(donebar, 1);
         *abort_flag = 0;
-        int bad = 0;
-        int same = 1;
-        for (int s = 0; s < a.ns; ++s) {
-            int e;
-            float g;
-            if (s < a.k) { e = a.idx0[s]; g = a.gate0[s]; }
-            else { e = a.idx1[s - a.k]; g = -a.gate1[s - a.k]; }
-            if (e < 0 || e >= a.E) { bad = 1; e = -1; g = 0.f; }
-            s_e[s] = e;
-            s_g[s] = g;
-        }
-        if (a.mode == 1) {
-            for (int s = 0; s < a.k; ++s)
-                if (a.idx0[s] != a.idx1[s] || __float_as_uint(a.gate0[s]) != __float_as_uint(a.gate1[s])) same = 0;
-        } else {
-            same = 0;
-        }
-        *s_skip = same;
-        if (bad && blockIdx.x == 0) atomicOr(a.status, ADAFUSE_STATUS_BAD_INDEX);
         fence_mbar_init();
     }
     // Zero every A slot: the K padding rows and the rows of skipped slots are
@@ -530,6 +522,9 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_rows_kernel(const __gr
         for (uint32_t o = threadIdx.x * 16; o < ATile; o += kMergeThreads * 16)
             st_shared_v4(smem_u32(sA + (size_t)st * ATile + o), make_uint4(0, 0, 0, 0));
     fence_proxy_async_smem();
+    griddep_wait();
+    griddep_launch_dependents();
+    if (threadIdx.x == 0) read_selection(a, s_e, s_g, s_skip);
     __syncthreads();
     if (*s_skip) return;       // switch between identical selections: nothing to do
 
@@ -859,9 +854,8 @@ int launch_merge_fused(Plan* p, const int32_t* idx0, const float* gate0, const i
             if (cudaFuncSetAttribute(merge_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
                 return ADAFUSE_ERR_CUDA;
             const int grid = (int)std::min<int64_t>(p->num_sms, p->merge_tiles);
-            merge_rows_kernel<<<grid, kMergeThreads, smem, s>>>(a);
             p->last_launches = 1;
-            return cuda_err(cudaGetLastError());
+            return launch_pdl(merge_rows_kernel, dim3(grid), dim3(kMergeThreads), smem, s, a);
         }
     }
     const uint32_t BBytes = (uint32_t)a.Kp * 256u;
@@ -886,9 +880,8 @@ int launch_merge_fused(Plan* p, const int32_t* idx0, const float* gate0, const i
     cudaError_t e = cudaFuncSetAttribute(merge_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return ADAFUSE_ERR_CUDA;
     const int grid = (int)std::min<int64_t>(p->num_sms, p->merge_tiles);
-    merge_fused_kernel<<<grid, kMergeThreads, smem, s>>>(a);
     p->last_launches = 1;
-    return cuda_err(cudaGetLastError());
+    return launch_pdl(merge_fused_kernel, dim3(grid), dim3(kMergeThreads), smem, s, a);
 }
 
 int launch_merge_per_linear(Plan* p, const int32_t* idx, const float* gate, int32_t k, cudaStream_t s)

@@ -26,6 +26,25 @@ __device__ __forceinline__ uint64_t globaltimer_ns()
     return t;
 }
 
+// ------------------------------------------- programmatic dependent launch
+// The library's kernels are launched with programmatic stream serialization:
+// a kernel may become resident while the previous kernel of the stream is
+// still running.  Each one sets up its shared memory and barriers first and
+// calls griddep_wait() before it touches global memory or TMEM; the wait
+// returns once the previous kernel has completed and its writes are visible
+// (at once when the launch had no programmatic dependency).
+__device__ __forceinline__ void griddep_wait()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// Lets the next kernel of the stream start launching.  It still waits, in
+// griddep_wait(), for this whole grid to finish.
+__device__ __forceinline__ void griddep_launch_dependents()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ mbarrier
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count)

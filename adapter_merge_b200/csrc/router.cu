@@ -61,6 +61,8 @@ __global__ void __launch_bounds__(kRouterThreads) pregate_kernel(const uint16_t*
     // xfull: 0 = x staged chunk by chunk, 1 = whole x row first, 2 = whole
     // W_r and whole x row first (no ring, no per-chunk barriers).
     extern __shared__ float rsm[];
+    griddep_wait();
+    griddep_launch_dependents();
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const bool pool = (flags & ADAFUSE_POOL_MEAN) != 0;
     const int64_t t = pool ? 0 : blockIdx.x;
@@ -250,7 +252,7 @@ extern "C" int adafuse_pregate(const void* x, int64_t T, int32_t H, int64_t x_ro
     if (smem > 48 * 1024 &&
         cudaFuncSetAttribute(af::pregate_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return ADAFUSE_ERR_CUDA;
-    af::pregate_kernel<<<grid, af::kRouterThreads, smem, (cudaStream_t)stream>>>(
-        static_cast<const uint16_t*>(x), T, H, x_row_stride, W_r, b_r, E, k, flags, idx, gate, xfull, w16);
-    return af::cuda_err(cudaGetLastError());
+    return af::launch_pdl(af::pregate_kernel, dim3(grid), dim3(af::kRouterThreads), smem, (cudaStream_t)stream,
+                          static_cast<const uint16_t*>(x), T, H, x_row_stride, W_r, b_r, E, k, flags, idx, gate,
+                          xfull, w16);
 }

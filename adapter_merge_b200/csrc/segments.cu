@@ -22,6 +22,8 @@ __global__ void __launch_bounds__(kSegThreads) segments_kernel(const int32_t* id
     __shared__ int cnt[kSegThreads][kMaxE + 1];
     __shared__ int s_off[kMaxE + 1];
     const int tid = threadIdx.x;
+    griddep_wait();
+    griddep_launch_dependents();
     const int64_t chunk = (P + kSegThreads - 1) / kSegThreads;
     const int64_t p0 = (int64_t)tid * chunk < P ? (int64_t)tid * chunk : P;
     const int64_t p1 = p0 + chunk < P ? p0 + chunk : P;
@@ -69,8 +71,8 @@ __global__ void __launch_bounds__(kSegThreads) segments_kernel(const int32_t* id
 int launch_segments(const int32_t* idx, int64_t T, int32_t k, int32_t E, int32_t* offsets, int32_t* perm,
                     int32_t* used, int32_t* status, cudaStream_t s)
 {
-    segments_kernel<<<1, kSegThreads, 0, s>>>(idx, T * k, E, offsets, perm, used, status);
-    return cuda_err(cudaGetLastError());
+    return launch_pdl(segments_kernel, dim3(1), dim3(kSegThreads), 0, s, idx, T * k, E, offsets, perm, used,
+                      status);
 }
 
 }  // namespace af

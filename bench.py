@@ -260,8 +260,10 @@ def run_sweep(args):
     128}.  A 33.5 MB layer fits in the 126 MB L2, so every point rotates
     through 8 independent copies (W, W', A, B and a plan each, 8 x 100+ MB
     touched per cycle) and each launch finds its operands in HBM.  Per point:
-    the device time of one launch (CUDA events around it, median), the time
-    per launch when launches run back to back (launch gaps included), and the
+    the device time of one call (CUDA events around it, median; a GPU sleep
+    queued before the first event keeps the device busy until the host has
+    queued the whole call, so host time does not count), the time per call
+    when calls run back to back (launch gaps and host time included), and the
     host time of the API call (launch overhead)."""
     import torch
     import adapter_merge_b200 as am
@@ -275,6 +277,7 @@ def run_sweep(args):
     peak, peak_kind = read_peaks()
     stream = torch.cuda.current_stream()
     NC, R = 8, 5                          # copies, rounds over the copies
+    SLEEP_CYCLES = 1_000_000              # ~0.5 ms of GPU sleep ahead of each timed call
     points = []
     t_begin = time.perf_counter()
     for E in (4, 8, 16, 32):
@@ -303,6 +306,7 @@ def run_sweep(args):
                     torch.cuda.synchronize()
                     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(NC * R)]
                     for i in range(NC * R):
+                        torch.cuda._sleep(SLEEP_CYCLES)
                         ev[i][0].record(stream)
                         fn(i % NC)
                         ev[i][1].record(stream)
