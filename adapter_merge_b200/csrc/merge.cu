@@ -10,7 +10,7 @@
 //
 // B200 design: one persistent CTA per SM, warp-specialised, two variants.
 //   merge_rows_kernel (k*r <= 128, every model configuration): 128 x 128
-//     tiles walked along the rows of W in groups of 2, 4 or 8 row blocks
+//     tiles walked along the rows of W in groups of 1, 2, 4 or 8 row blocks
 //     interleaved column by column.  Warp 0 loads W tiles by TMA (two
 //     64-column boxes, 128-byte swizzle) and, once per column block of a
 //     group, the raw A rows of the selected experts (MN-major, 128-byte
@@ -414,7 +414,7 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_fused_kernel(const __g
 // ------------------------------------------------------------------ row order
 
 // Row-order variant (k*r <= 128).  Tiles are walked along the rows of W in
-// groups of G (2, 4 or 8) 128-row blocks, the blocks of a group interleaved
+// groups of G (1, 2, 4 or 8) 128-row blocks, the blocks of a group interleaved
 // column block by column block: (block 0, cols 0-127), (block 1, cols 0-127),
 // ..., (block 0, cols 128-255), ...  Consecutive tiles of a CTA continue the
 // same rows of W (long contiguous DRAM runs), and the raw A rows of a
@@ -832,10 +832,13 @@ int launch_merge_fused(Plan* p, const int32_t* idx0, const float* gate0, const i
         // then the group size (less A traffic), then a second group slot (the
         // next group's Bcat built ahead), then A slots.  Groups of four or
         // eight only where a CTA walks enough tiles to amortise their builds.
+        // Single-block groups (a plain row walk, every tile its own A tile)
+        // only where they buy a W stage: at k*r = 128, G = 1 with four W
+        // stages ran the 13B switch 17 % faster than G = 2 with three.
         const uint32_t at = (uint32_t)a.Kp * 256u, bc = at;
         const bool long_walk = p->merge_tiles >= 128 * (int64_t)p->num_sms;
         int SW = 0, NA = 0, NAR = 0, G = 0;
-        for (int g : {8, 4, 2}) {
+        for (int g : {8, 4, 2, 1}) {
             if (g >= 4 && !long_walk) continue;
             for (int np : {2, 1})
                 for (int nar : {3, 2}) {

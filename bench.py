@@ -254,6 +254,21 @@ def run_reference(args):
     return 0
 
 
+def sweep_point_arg(text):
+    """The (E, r, k) of --point "E,r,k" (None for the whole grid); SystemExit
+    if it is not a point of the sweep grid."""
+    if not text:
+        return None
+    try:
+        pt = tuple(int(v) for v in text.split(","))
+    except ValueError:
+        pt = ()
+    if (len(pt) != 3 or pt[0] not in (4, 8, 16, 32) or pt[1] not in (8, 16, 32, 64) or pt[2] not in (1, 2, 4)
+            or pt[2] > pt[0] or pt[1] * pt[2] > 256):
+        raise SystemExit(f"--point {text}: not a point of the sweep grid")
+    return pt
+
+
 def run_sweep(args):
     """The single-linear 4096 x 4096 grid: E in {4, 8, 16, 32}, r in {8, 16,
     32, 64}, k in {1, 2, 4}; merge per (E, r, k) and apply per T in {1, 16,
@@ -276,6 +291,7 @@ def run_sweep(args):
     ambuild.build()
     peak, peak_kind = read_peaks()
     stream = torch.cuda.current_stream()
+    only = sweep_point_arg(args.point)
     NC, R = 8, 5                          # copies, rounds over the copies
     SLEEP_CYCLES = 1_000_000              # ~0.5 ms of GPU sleep ahead of each timed call
     points = []
@@ -283,7 +299,7 @@ def run_sweep(args):
     for E in (4, 8, 16, 32):
         for r in (8, 16, 32, 64):
             for k in (1, 2, 4):
-                if k > E or k * r > 256:
+                if k > E or k * r > 256 or (only and (E, r, k) != only):
                     continue
                 cfg = synth.sweep_point(E, r, k, 128)
                 lin = cfg.linears[0]
@@ -361,8 +377,9 @@ def run_sweep(args):
             "value": round(statistics.median(p["merge"]["gbs"] for p in points), 2), "unit": "GB/s",
             "n_gpus": 1, "higher_is_better": True, "dtype": "bf16",
             "data": "synthetic (seeded; gates = softmax of N(0,1) logits)",
-            "config": {"workload": "sweep 4096x4096, E in {4,8,16,32}, r in {8,16,32,64}, k in {1,2,4}, "
-                                   "T in {1,16,128}",
+            "config": {"workload": (f"sweep point 4096x4096, E={only[0]}, r={only[1]}, k={only[2]}, T in {{1,16,128}}"
+                                    if only else "sweep 4096x4096, E in {4,8,16,32}, r in {8,16,32,64}, "
+                                                 "k in {1,2,4}, T in {1,16,128}"),
                        "l2": f"{NC} rotated copies of every operand (no L2 reuse between launches)"},
             "peak": peak, "peak_source": f"{peak_kind} hbm_gbs",
             "merge_frac_of_peak": {"min": min(fr), "median": statistics.median(fr), "max": max(fr)},
@@ -381,6 +398,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--config", default="7b", choices=["7b", "13b", "sweep"],
                     help="sweep = the single-linear 4096^2 grid, measured per point (its own JSON line)")
+    ap.add_argument("--point", default="",
+                    help="with --config sweep: only this E,r,k point (e.g. 8,16,2)")
     ap.add_argument("--layers", type=int, default=0,
                     help="use only the first N layers (small profiling case); 0 = the full model")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -392,7 +411,10 @@ def main():
         args.warmup = 3
     if args.impl == "reference":
         return run_reference(args)
+    if args.point and args.config != "sweep":
+        raise SystemExit("--point needs --config sweep")
     if args.config == "sweep":
+        sweep_point_arg(args.point)          # reject a point outside the grid before any GPU work
         return run_sweep(args)
 
     import torch
