@@ -224,6 +224,57 @@ def test_merge_per_linear_baseline(am, cuda_device):
     check_merge(m, idx, gate.astype(np.float64), "per-linear")
 
 
+def test_calls_queued_back_to_back(am, cuda_device):
+    """merge -> apply -> switch -> apply -> pregate -> apply queued on one
+    stream behind a GPU sleep, no host synchronisation in between, the three
+    applies on one workspace with different T and inputs.  Each kernel may
+    start while its predecessor still runs (programmatic dependent launch);
+    every result must still be the one of the calls run one at a time."""
+    cfg = synth.custom([(1024, 2048), (2048, 1024), (520, 1032)], 6, 16, 2, 40, name="b2b")
+    m = Model(cfg, cuda_device)
+    d = lambda a_, t: torch.as_tensor(np.asarray(a_).astype(t)).to(cuda_device)
+    sel_a = (np.array([1, 4]), np.array([0.55, 0.3], dtype=np.float32))
+    sel_b = (np.array([2, 1]), np.array([0.4, 0.25], dtype=np.float32))
+    Ts = (16, 40, 7)
+    ins, outs, sels = [], [], []
+    for j, T in enumerate(Ts):
+        X, xs = synth.make_apply_inputs(cfg, T, 20 + j)
+        ins.append(xs)
+        outs.append([torch.full((T, l.d_out), float("nan"), dtype=torch.bfloat16, device=cuda_device)
+                     for l in cfg.linears])
+        sels.append(synth.random_selection(T, cfg.E, cfg.k, 30 + j, f"b2b{j}"))
+    xr = synth.make_router_input(cfg, 5, 3)
+    W_r = synth.normal((cfg.E, cfg.hidden), cfg.hidden ** -0.5, torch.float32, 3, "b2bwr")
+    xs_dev = [[x.to(cuda_device) for x in xs] for xs in ins]
+    ws = torch.empty(max(m.plan.workspace_bytes(T, cfg.k) for T in Ts), dtype=torch.uint8, device=cuda_device)
+    xr_d, W_r_d = xr.to(cuda_device), W_r.to(cuda_device)
+    sel_dev = [(d(i, np.int32), d(g, np.float32)) for i, g in sels]
+    sa = (d(sel_a[0], np.int32), d(sel_a[1], np.float32))
+    sb = (d(sel_b[0], np.int32), d(sel_b[1], np.float32))
+    torch.cuda.synchronize()
+
+    torch.cuda._sleep(20_000_000)                      # ~10 ms: everything below is queued before it ends
+    m.plan.merge(*sa)
+    m.plan.apply(xs_dev[0], outs[0], Ts[0], *sel_dev[0], ws)
+    m.plan.switch(*sb, *sa)
+    m.plan.apply(xs_dev[1], outs[1], Ts[1], *sel_dev[1], ws)
+    r_idx, r_gate = am.pregate(xr_d, W_r_d, cfg.k)
+    m.plan.apply(xs_dev[2], outs[2], Ts[2], *sel_dev[2], ws)
+    torch.cuda.synchronize()
+
+    for j in range(3):
+        check_apply(m, ins[j], outs[j], sels[j][0].numpy(), sels[j][1].numpy().astype(np.float64), f"queued apply {j}")
+    idx_ref, gate_ref, _ = oracle.pregate(u16(xr), W_r.numpy(), cfg.k)
+    assert np.array_equal(r_idx.cpu().numpy(), idx_ref)
+    for l in range(cfg.n_lin):
+        W, A, B = u16(m.w.W_views[l]), u16(m.w.A_views[l]), u16(m.w.B_views[l])
+        cur = oracle.merge_linear(W, A, B, sel_a[0], sel_a[1].astype(np.float64))
+        ref = oracle.merge_linear(cur, A, B, list(sel_b[0]) + list(sel_a[0]),
+                                  list(sel_b[1].astype(np.float64)) + list(-sel_a[1].astype(np.float64)))
+        assert_close_bf16(u16(m.W_out[l]), ref, f"queued merge + switch linear {l}")
+    assert m.plan.status() == (0, 0)
+
+
 def test_switch_in_place(am, cuda_device):
     """Switch old -> new on the merged weights: matches the oracle's switch of
     the oracle's own merged weights; identical selections leave W_out alone."""
