@@ -34,6 +34,16 @@
  *     skips the offending slot or gives up the wait, sets a bit in the plan's
  *     status word and finishes; read it with adafuse_plan_status.
  *   - A plan may be used from one stream at a time.
+ *   - The library's kernels are launched with programmatic stream
+ *     serialization (programmatic dependent launch): each one may start while
+ *     the previous kernel on the stream is still running. Before any
+ *     global-memory access it waits until that kernel has completed, so work
+ *     queued ahead of a call is ordered as usual. Each library kernel lets
+ *     the next kernel of the stream launch early. A caller's kernel launched
+ *     normally after a call waits for the call to finish, as always. A
+ *     caller's kernel launched with the programmatic-serialization
+ *     attribute must execute griddepcontrol.wait (cudaGridDependencySynchronize)
+ *     before it reads the call's outputs.
  */
 #ifndef ADAFUSE_H
 #define ADAFUSE_H
