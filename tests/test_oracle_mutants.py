@@ -34,16 +34,33 @@ MUTANTS = {
     "bf16_ties_away_from_zero": (r"double n = nearbyint\(a / q\);", "double n = round(a / q);"),
     "router_fused_multiply_add": (r"                float p = xj \* Wr\[\(int64_t\)e \* H \+ j\];\n                acc = acc \+ p;",
                                   "                acc = fmaf(xj, Wr[(int64_t)e * H + j], acc);"),
+    "router_bias_added_first": [(r"            float acc = 0\.0f;\n            for \(int32_t j = 0; j < H; \+\+j\) \{\n                float xj",
+                                 "            float acc = br ? br[e] : 0.0f;\n            for (int32_t j = 0; j < H; ++j) {\n                float xj"),
+                                (r"            if \(br\) acc = acc \+ br\[e\];\n            z\[t \* E \+ e\] = acc;",
+                                 "            z[t * E + e] = acc;")],
+    "softmax_without_max_shift": (r"double m = -INFINITY;\n        for \(int e = 0; e < E; \+\+e\) if \(!isnan\(zt\[e\]\) && \(double\)zt\[e\] > m\) m = \(double\)zt\[e\];",
+                                  "double m = 0.0;"),
+    "topk_nan_ranks_first": (r"    if \(na\) return 0;\n    if \(nb\) return 1;", "    if (na) return 1;\n    if (nb) return 0;"),
+    "pool_mean_divides_by_T_minus_1": (r"xbar\[j\] = acc / \(float\)T;", "xbar[j] = acc / (float)(T > 1 ? T - 1 : 1);"),
+    "merge_gate_squared": (r"acc \+= g\[s\] \* d;", "acc += g[s] * g[s] * d;"),
+    "apply_base_term_dropped": (r"            for \(int64_t i = 0; i < d_in; \+\+i\)\n                acc \+= orc_bf16_to_double\(x\[t \* d_in \+ i\]\) \* orc_bf16_to_double\(W\[o \* d_in \+ i\]\);",
+                                "            (void)W;"),
+    "apply_shrink_reads_token_0": (r"\* d_in \+ i\]\) \*\n                               orc_bf16_to_double\(x\[t \* d_in \+ i\]\);",
+                                   "* d_in + i]) *\n                               orc_bf16_to_double(x[i]);"),
+    "segments_count_shifted": (r"offsets\[e \+ 1\] \+= 1;", "offsets[e] += 1;"),
 }
 
 
 @pytest.mark.parametrize("name", sorted(MUTANTS))
 def test_pins_catch_planted_mistake(name, tmp_path):
-    pat, rep = MUTANTS[name]
+    sites = MUTANTS[name]
+    if isinstance(sites, tuple):
+        sites = [sites]
     with open(SRC) as f:
-        src = f.read()
-    mutated, n = re.subn(pat, lambda m: rep, src, count=1)
-    assert n == 1, f"mutation {name} did not apply"
+        mutated = f.read()
+    for pat, rep in sites:
+        mutated, n = re.subn(pat, lambda m: rep, mutated, count=1)
+        assert n == 1, f"mutation {name} did not apply"
     csrc = tmp_path / "mutant.c"
     csrc.write_text(mutated)
     lib = tmp_path / "libmutant.so"

@@ -185,6 +185,18 @@ def test_router_products_are_rounded_before_the_add():
     assert z[0, 0] == np.float32(0.0)
 
 
+def test_router_bias_added_after_the_sum():
+    """The bias is added once the products are summed (the reading the
+    kernel follows too, so that idx parity is exact): 0 + 2^-24 + 2^-24 =
+    2^-23 exactly, then + 1 gives 1 + 2^-23; starting the sum from the bias
+    would lose both tiny products (1 + 2^-24 rounds to 1) and give 1."""
+    x = bits(np.array([[1.0, 1.0]], dtype=np.float32))
+    W_r = np.array([[2.0 ** -24, 2.0 ** -24]], dtype=np.float32)
+    b_r = np.array([1.0], dtype=np.float32)
+    z = oracle.router_logits(x, W_r, b_r)
+    assert z[0, 0] == np.float32(1.0 + 2.0 ** -23)
+
+
 @pytest.mark.parametrize("E", [1, 2, 3, 4, 5])
 def test_topk_brute_force_all_tie_patterns(E):
     """Every logit pattern over {-1, 0, 1, nan}^E and every k: the selection is
@@ -227,6 +239,22 @@ def test_softmax_closed_forms_and_invariants():
     i0, _ = oracle.topk_softmax(z, 3)
     i1, _ = oracle.topk_softmax(z + np.float32(4.0), 3)
     assert np.array_equal(i0, i1)
+
+
+def test_softmax_large_logits_closed_form():
+    """Logits far outside exp's range: the probabilities still follow the
+    closed form p_i = 1 / sum_j exp(z_j - z_i) (a softmax computed without
+    subtracting the maximum overflows or underflows to 0/0 here)."""
+    cases = [[1000.0, 999.0, -1000.0, 0.0], [-1000.0, -1001.0, -1003.0, -2000.0], [88.5, 89.0, 90.0, -90.0]]
+    for zc in cases:
+        z = np.array([zc], dtype=np.float32)
+        idx, gate = oracle.topk_softmax(z, 2)
+        zz = z[0].astype(np.float64)
+        for s in range(2):
+            i = idx[0, s]
+            ref = 1.0 / math.fsum(math.exp(zz[j] - zz[i]) for j in range(4))
+            assert math.isclose(gate[0, s], ref, rel_tol=1e-14), (zc, s)
+        assert idx[0].tolist() == sorted(range(4), key=lambda e: (-zz[e], e))[:2]
 
 
 def test_pool_mean_exact_cases():
