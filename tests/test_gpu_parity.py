@@ -275,13 +275,15 @@ def test_calls_queued_back_to_back(am, cuda_device):
     assert m.plan.status() == (0, 0)
 
 
-def test_switch_in_place(am, cuda_device):
+@pytest.mark.parametrize("E,r,k", [(5, 16, 2), (6, 32, 2), (4, 8, 1)])
+def test_switch_in_place(am, cuda_device, E, r, k):
     """Switch old -> new on the merged weights: matches the oracle's switch of
-    the oracle's own merged weights; identical selections leave W_out alone."""
-    cfg = synth.custom([(384, 264), (136, 520)], 5, 16, 2, 1, name="mswitch")
+    the oracle's own merged weights; identical selections leave W_out alone.
+    2kr = 64, 128 (single-block groups) and 16."""
+    cfg = synth.custom([(384, 264), (136, 520)], E, r, k, 1, name=f"mswitch{E}{r}{k}")
     m = Model(cfg, cuda_device)
-    old_i, old_g = np.array([1, 4]), np.array([0.55, 0.3], dtype=np.float32)
-    new_i, new_g = np.array([2, 1]), np.array([0.4, 0.25], dtype=np.float32)
+    old_i, old_g = np.array([1, 4][:k]), np.array([0.55, 0.3][:k], dtype=np.float32)
+    new_i, new_g = np.array([2, 1][:k]), np.array([0.4, 0.25][:k], dtype=np.float32)
     run_merge(am, m, old_i, old_g, cuda_device)
     d = lambda a, t: torch.as_tensor(a.astype(t)).to(cuda_device)
     m.plan.switch(d(new_i, np.int32), d(new_g, np.float32), d(old_i, np.int32), d(old_g, np.float32))
