@@ -103,3 +103,43 @@ def test_binding_has_no_fallback(tmp_path, monkeypatch):
     monkeypatch.setattr(am, "_lib", None)
     with pytest.raises(RuntimeError):
         am.lib()
+
+
+C_CLIENT = r"""
+#include <stdio.h>
+#include <string.h>
+#include "adafuse.h"
+
+int main(void)
+{
+    adafuse_plan* plan = NULL;
+    adafuse_linear lin;
+    memset(&lin, 0, sizeof lin);
+    if (adafuse_version() != 100) return 1;
+    if (strcmp(adafuse_strerror(99), "unknown error") != 0) return 2;
+    if (adafuse_pregate(NULL, 1, 8, 8, NULL, NULL, 4, 2, 0, NULL, NULL, NULL) != ADAFUSE_ERR_INVALID_ARG) return 3;
+    if (adafuse_plan_create(&plan, NULL, 1, 4, 8, 0) != ADAFUSE_ERR_INVALID_ARG) return 4;
+    if (adafuse_merge(NULL, NULL, NULL, 2, NULL) != ADAFUSE_ERR_INVALID_ARG) return 5;
+    if (adafuse_apply_workspace_bytes(NULL, 4, 2) != 0) return 6;
+    adafuse_plan_destroy(NULL);
+    printf("ok %s\n", adafuse_strerror(ADAFUSE_ERR_UNSUPPORTED));
+    return 0;
+}
+"""
+
+
+def test_plain_c_client_builds_and_links(L, tmp_path):
+    """The header is a C ABI: a C11 program (no CUDA headers, -pedantic
+    -Werror) includes it, links the library and makes the calls that need no
+    device."""
+    import subprocess
+    src = tmp_path / "client.c"
+    src.write_text(C_CLIENT)
+    exe = tmp_path / "client"
+    libdir = os.path.dirname(L._name)
+    subprocess.check_call(["gcc", "-std=c11", "-Wall", "-Wextra", "-Werror", "-pedantic",
+                           "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe),
+                           "-L", libdir, "-l:" + os.path.basename(L._name), "-Wl,-rpath," + libdir])
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0, (r.returncode, r.stdout, r.stderr)
+    assert r.stdout.startswith("ok ")
