@@ -143,3 +143,26 @@ def test_plain_c_client_builds_and_links(L, tmp_path):
     r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
     assert r.returncode == 0, (r.returncode, r.stdout, r.stderr)
     assert r.stdout.startswith("ok ")
+
+
+def test_product_is_independent_of_the_oracle():
+    """The library, its binding and its build never name, import or link the
+    oracle, and the oracle never includes the library's sources: the two
+    share only the seeded input generators."""
+    pkg = os.path.join(ROOT, "adapter_merge_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h", ".c", ".cpp")):
+                with open(os.path.join(dirpath, f), errors="replace") as fh:
+                    text = fh.read()
+                assert "oracle" not in text.lower(), os.path.join(dirpath, f)
+    with open(os.path.join(ROOT, "include", "adafuse.h")) as fh:
+        assert "oracle" not in fh.read().lower()
+    odir = os.path.join(ROOT, "oracle")
+    for f in os.listdir(odir):
+        if f.endswith((".py", ".c", ".h")):
+            with open(os.path.join(odir, f)) as fh:
+                text = fh.read()
+            assert not re.search(r"^\s*(import|from)\s+adapter_merge_b200", text, re.M), f
+            assert not re.search(r"^\s*#\s*include\s*[<\"][^>\"]*(adafuse|csrc|ptx)", text, re.M), f
+            assert "libadafuse" not in text, f
