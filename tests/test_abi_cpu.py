@@ -166,3 +166,14 @@ def test_product_is_independent_of_the_oracle():
             assert not re.search(r"^\s*(import|from)\s+adapter_merge_b200", text, re.M), f
             assert not re.search(r"^\s*#\s*include\s*[<\"][^>\"]*(adafuse|csrc|ptx)", text, re.M), f
             assert "libadafuse" not in text, f
+
+
+def test_input_generators_import_neither_side():
+    """synth/ (seeded inputs for both sides) imports neither the library nor
+    the oracle."""
+    sdir = os.path.join(ROOT, "synth")
+    for f in os.listdir(sdir):
+        if f.endswith(".py"):
+            with open(os.path.join(sdir, f)) as fh:
+                text = fh.read()
+            assert not re.search(r"^\s*(import|from)\s+(oracle|adapter_merge_b200)\b", text, re.M), f
