@@ -1,5 +1,6 @@
-"""Host-side argument handling of the benchmark (no GPU): which measurement
-each command line reaches, and the sweep-point parser."""
+"""Host-side logic of the benchmark (no GPU): which measurement each command
+line reaches, the sweep-point parser, and the clock sampler's summary."""
+import os
 import sys
 
 import pytest
@@ -48,3 +49,34 @@ def test_main_dispatch(monkeypatch):
         _run_main(monkeypatch, ["--config", "sweep", "--point", "8,16,3"])
     with pytest.raises(SystemExit):
         _run_main(monkeypatch, ["--point", "8,16,2"])
+
+
+def test_clock_sampler_parses_nvidia_smi(tmp_path, monkeypatch):
+    """The sampler's summary of the nvidia-smi CSV it records: median SM
+    clock, max clock and power, and every throttle reason seen active (a
+    fake nvidia-smi on PATH stands in for the real one)."""
+    import time
+    import bench
+    fake = tmp_path / "nvidia-smi"
+    fake.write_text("#!/bin/sh\n"
+                    "echo '0, 1900, 1965, 700.5, 0x4, Not Active, Not Active, Not Active, Active'\n"
+                    "echo '0, 1800, 1965, 710.0, 0x4, Not Active, Not Active, Not Active, Active'\n"
+                    "echo '0, 1950, 1965, 650.0, 0x0, Active, Not Active, Not Active, Not Active'\n"
+                    "echo 'garbage line'\n"
+                    "exec sleep 30\n")
+    fake.chmod(0o755)
+    monkeypatch.setenv("PATH", str(tmp_path) + os.pathsep + os.environ.get("PATH", ""))
+    s = bench.ClockSampler(0)
+    s.start()
+    time.sleep(0.5)
+    c = s.stop()
+    assert c == {"sm_mhz": 1900.0, "sm_max_mhz": 1965.0, "power_w_max": 710.0, "samples": 3,
+                 "reasons": ["hw_slowdown", "sw_power_cap"]}
+
+
+def test_clock_sampler_without_nvidia_smi(tmp_path, monkeypatch):
+    import bench
+    monkeypatch.setenv("PATH", str(tmp_path))
+    s = bench.ClockSampler(0)
+    s.start()
+    assert s.stop() is None
