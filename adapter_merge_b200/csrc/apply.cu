@@ -26,7 +26,10 @@
 // Every operand moves by TMA: W and the experts' A and B rows through the
 // plan's tensor maps, x and S through per-call maps that the host builds (and
 // caches by pointer set, T and workspace) before the launches.  W is streamed
-// exactly once per token tile; the x and S tiles come from L2.
+// exactly once per token tile; the x and S tiles come from L2.  The four
+// launches use programmatic dependent launch: each kernel sets up its shared
+// memory while the previous one finishes, and waits for it before touching
+// global memory.
 #include <cudaTypedefs.h>
 
 #include <algorithm>

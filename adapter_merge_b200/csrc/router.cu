@@ -9,12 +9,13 @@
 //
 // One CTA per decision.  Warp 0 lane e owns expert e: its logit is the fp32 sum
 // of the products x_j * W_r[e, j] in ascending j (products rounded before the
-// add), so the decision is a fixed function of the inputs.  W_r streams
-// through a 4-stage cp.async ring (three 256-column chunks ahead).  The whole
-// x row is staged in shared memory before the chain starts when it fits (one
-// round of loads instead of one per chunk); otherwise, and for the pooled
-// mean, warps 1-3 stage the next chunk of x while warp 0 consumes the current
-// one.  Softmax and top-k are warp shuffles over the lanes (ties to the lower
+// add), so the decision is a fixed function of the inputs.  Where the whole
+// W_r (rows padded to H + 4 floats) and the x row fit in shared memory, both
+// are staged with 16-byte cp.async copies before the chain starts, which then
+// runs with no barrier.  Otherwise W_r streams through a 4-stage cp.async ring
+// (three 256-column chunks ahead), with the whole x row staged first when it
+// fits; for the pooled mean and larger rows, warps 1-3 stage the next chunk of
+// x while warp 0 consumes the current one.  Softmax and top-k are warp shuffles over the lanes (ties to the lower
 // index, NaN ranked last).
 #include "internal.h"
 #include "ptx.cuh"
