@@ -51,8 +51,7 @@ MUTANTS = {
 }
 
 
-@pytest.mark.parametrize("name", sorted(MUTANTS))
-def test_pins_catch_planted_mistake(name, tmp_path):
+def _apply(name):
     sites = MUTANTS[name]
     if isinstance(sites, tuple):
         sites = [sites]
@@ -60,14 +59,44 @@ def test_pins_catch_planted_mistake(name, tmp_path):
         mutated = f.read()
     for pat, rep in sites:
         mutated, n = re.subn(pat, lambda m: rep, mutated, count=1)
-        assert n == 1, f"mutation {name} did not apply"
-    csrc = tmp_path / "mutant.c"
+        if n != 1:
+            return None
+    return mutated
+
+
+def _run_pins_on(name, workdir):
+    """Build the mutant oracle and run the pin tests against it: (applied,
+    pytest return code, end of its output)."""
+    mutated = _apply(name)
+    if mutated is None:
+        return False, None, ""
+    d = workdir / name
+    d.mkdir()
+    csrc = d / "mutant.c"
     csrc.write_text(mutated)
-    lib = tmp_path / "libmutant.so"
+    lib = d / "libmutant.so"
     subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp",
                            "-ffp-contract=off", "-o", str(lib), str(csrc), "-lm"])
-    env = dict(os.environ, ADAFUSE_ORACLE_LIB=str(lib))
+    env = dict(os.environ, ADAFUSE_ORACLE_LIB=str(lib), OMP_NUM_THREADS="2")
     r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
                         os.path.join(ROOT, "tests", "test_oracle_pins.py")],
                        cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
-    assert r.returncode != 0, f"pins did not catch mutant {name}:\n{r.stdout[-2000:]}"
+    return True, r.returncode, r.stdout[-2000:]
+
+
+@pytest.fixture(scope="module")
+def mutant_runs(tmp_path_factory):
+    """Every mutant's pin run, several at a time (each is an independent
+    process on its own copy of the oracle)."""
+    from concurrent.futures import ThreadPoolExecutor
+    work = tmp_path_factory.mktemp("mutants")
+    names = sorted(MUTANTS)
+    with ThreadPoolExecutor(max_workers=max(1, min(8, (os.cpu_count() or 2) // 2))) as ex:
+        return dict(zip(names, ex.map(lambda n: _run_pins_on(n, work), names)))
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_planted_mistake(name, mutant_runs):
+    applied, rc, out = mutant_runs[name]
+    assert applied, f"mutation {name} did not apply"
+    assert rc != 0, f"pins did not catch mutant {name}:\n{out}"
