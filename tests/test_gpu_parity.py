@@ -46,6 +46,7 @@ def check_gates(g_gpu, g_ref):
     (300, 32, 17, 4, False, False),     # E = 32 lanes, ragged H
     (100, 5, 3, 5, True, True),         # k = E
     (8, 1, 2, 1, False, False),         # single expert
+    (4096, 8, 2000, 2, False, False),   # 2000 decisions: many waves of CTAs
 ])
 def test_pregate_matches_oracle(am, cuda_device, H, E, T, k, bias, renorm):
     x = synth.normal((T, H), 1.0, torch.bfloat16, 1, f"px{H}{E}{T}")
@@ -212,6 +213,21 @@ def test_merge_bad_index_skipped_and_flagged(am, cuda_device):
     rc, st = m.plan.status()
     assert rc == 0 and st == am.STATUS_BAD_INDEX
     check_merge(m, idx, gate.astype(np.float64), "bad index")
+    assert m.plan.status() == (0, 0)
+
+
+def test_merge_repeated_expert_gates_add(am, cuda_device):
+    """An expert picked in two slots contributes with the sum of its gates
+    (the oracle's sum over slots), in the merge and in the switch."""
+    cfg = synth.custom([(384, 264), (136, 520)], 5, 16, 3, 1, name="mrep")
+    m = Model(cfg, cuda_device)
+    idx, gate = np.array([2, 2, 0]), np.array([0.3, 0.2, 0.1], dtype=np.float32)
+    run_merge(am, m, idx, gate, cuda_device)
+    check_merge(m, idx, gate.astype(np.float64), "repeated expert")
+    one = Model(cfg, cuda_device, weights=m.w)
+    run_merge(am, one, np.array([2, 0, 4]), np.array([0.5, 0.1, 0.0], dtype=np.float32), cuda_device)
+    for a, b in zip(m.W_out, one.W_out):
+        assert_close_bf16(u16(a), u16(b), "repeated expert vs summed gate")
     assert m.plan.status() == (0, 0)
 
 
