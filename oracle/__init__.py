@@ -66,6 +66,8 @@ def _load():
                                          P, P, i32, i64, i64, i32]
         lib.orc_apply_linear.argtypes = [P, P, P, P, i32, i32, i32, i32, i64, i64,
                                          P, P, i32, i64, i64, P, i32]
+        lib.orc_apply_linear_f64.argtypes = [P, P, P, P, i32, i32, i32, i32, i64, i64,
+                                             P, P, i32, i64, i64, P, i32]
         lib.orc_segments.argtypes = [P, i64, i32, i32, P, P]
         lib.orc_segments.restype = i32
         lib.orc_max_threads.restype = i32
@@ -196,6 +198,25 @@ def apply_linear(x_bits, W_bits, A_bits, B_bits, idx, gate, tokens=None,
     _load().orc_apply_linear(_p(x), _p(W), _p(A), _p(B), d_out, d_in, E, r,
                              r * d_in, d_out * r, _p(idx), _p(gate), k, t0, t1,
                              _p(y), nthreads)
+    return y
+
+
+def apply_linear_f64(x_bits, W_bits, A_bits, B_bits, idx, gate, tokens=None,
+                     nthreads: int = 1) -> np.ndarray:
+    """As apply_linear, but the rows of y unrounded (float64): the partial
+    output of a row-parallel shard, whose sum over the shards is rounded once."""
+    x = _u16(x_bits); W = _u16(W_bits); A = _u16(A_bits); B = _u16(B_bits)
+    T, d_in = x.shape
+    d_out = W.shape[0]
+    E, r, _ = A.shape
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    gate = np.ascontiguousarray(gate, dtype=np.float64)
+    k = idx.shape[1]
+    t0, t1 = (0, T) if tokens is None else tokens
+    y = np.empty((t1 - t0, d_out), dtype=np.float64)
+    _load().orc_apply_linear_f64(_p(x), _p(W), _p(A), _p(B), d_out, d_in, E, r,
+                                 r * d_in, d_out * r, _p(idx), _p(gate), k, t0, t1,
+                                 _p(y), nthreads)
     return y
 
 

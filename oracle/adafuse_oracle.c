@@ -228,15 +228,18 @@ void orc_merge_linear(const uint16_t* W, uint16_t* Wout,
 
 /* Unmerged mixed-batch apply for one linear (segmented-gather form):
  *   u[t,s,j] = sum_i A_{e_ts}[j,i] * x[t,i]
- *   y[t,o]   = bf16( sum_i x[t,i] W[o,i] + sum_s g[t,s] sum_j B_{e_ts}[o,j] u[t,s,j] )
+ *   y[t,o]   = sum_i x[t,i] W[o,i] + sum_s g[t,s] sum_j B_{e_ts}[o,j] u[t,s,j]
  * for tokens t in [t0, t1).  Slots with an index outside [0, E) are skipped.
- * x is [T, d_in] row-major, y is [t1-t0, d_out] row-major. */
-void orc_apply_linear(const uint16_t* x, const uint16_t* W,
-                      const uint16_t* A, const uint16_t* B,
-                      int32_t d_out, int32_t d_in, int32_t E, int32_t r,
-                      int64_t a_es, int64_t b_es,
-                      const int32_t* idx, const double* gate, int32_t k,
-                      int64_t t0, int64_t t1, uint16_t* y, int32_t nthreads)
+ * x is [T, d_in] row-major; the result rows [t1-t0, d_out] go to y16 rounded
+ * once to bf16 (orc_apply_linear), or to y64 unrounded (orc_apply_linear_f64:
+ * the partial output of a row-parallel shard, whose sum over the shards is
+ * rounded once after the all-reduce). */
+static void apply_rows(const uint16_t* x, const uint16_t* W,
+                       const uint16_t* A, const uint16_t* B,
+                       int32_t d_out, int32_t d_in, int32_t E, int32_t r,
+                       int64_t a_es, int64_t b_es,
+                       const int32_t* idx, const double* gate, int32_t k,
+                       int64_t t0, int64_t t1, uint16_t* y16, double* y64, int32_t nthreads)
 {
 #ifdef _OPENMP
     if (nthreads < 1) nthreads = 1;
@@ -267,10 +270,31 @@ void orc_apply_linear(const uint16_t* x, const uint16_t* W,
                     d += orc_bf16_to_double(B[e * b_es + o * r + j]) * u[s * r + j];
                 acc += gate[t * k + s] * d;
             }
-            y[(t - t0) * d_out + o] = orc_bf16_from_double(acc);
+            if (y16) y16[(t - t0) * d_out + o] = orc_bf16_from_double(acc);
+            if (y64) y64[(t - t0) * d_out + o] = acc;
         }
         free(u);
     }
+}
+
+void orc_apply_linear(const uint16_t* x, const uint16_t* W,
+                      const uint16_t* A, const uint16_t* B,
+                      int32_t d_out, int32_t d_in, int32_t E, int32_t r,
+                      int64_t a_es, int64_t b_es,
+                      const int32_t* idx, const double* gate, int32_t k,
+                      int64_t t0, int64_t t1, uint16_t* y, int32_t nthreads)
+{
+    apply_rows(x, W, A, B, d_out, d_in, E, r, a_es, b_es, idx, gate, k, t0, t1, y, NULL, nthreads);
+}
+
+void orc_apply_linear_f64(const uint16_t* x, const uint16_t* W,
+                          const uint16_t* A, const uint16_t* B,
+                          int32_t d_out, int32_t d_in, int32_t E, int32_t r,
+                          int64_t a_es, int64_t b_es,
+                          const int32_t* idx, const double* gate, int32_t k,
+                          int64_t t0, int64_t t1, double* y, int32_t nthreads)
+{
+    apply_rows(x, W, A, B, d_out, d_in, E, r, a_es, b_es, idx, gate, k, t0, t1, NULL, y, nthreads);
 }
 
 /* -------------------------------------------------------------- segments */

@@ -423,6 +423,34 @@ def test_apply_merged_equals_unmerged_and_token_permutation():
     assert np.array_equal(yp, oracle.apply_linear(b(xt), b(Wt), b(At), b(Bt), idx, gate)[perm])
 
 
+def test_apply_f64_is_the_unrounded_apply_and_shards_sum():
+    """The unrounded apply (a row-parallel shard's partial output): on dyadic
+    inputs every product and sum is exact in fp64, so it equals numpy's
+    per-token result exactly, rounds to exactly apply_linear's bf16 output, and
+    the partials of a split of d_in into column blocks (W and A cut the same
+    way, B whole) add up exactly to the unsharded result."""
+    rng = np.random.default_rng(24)
+    T, d_out, d_in, E, r, k = 5, 16, 48, 4, 8, 2
+    W, A, B = _rand_adapters(rng, d_out, d_in, E, r)
+    x = dyadic(rng, (T, d_in), -4, 4, 1)
+    idx = np.stack([rng.permutation(E)[:k] for _ in range(T)]).astype(np.int32)
+    gate = dyadic(rng, (T, k), 1, 8, 3)
+    y64 = oracle.apply_linear_f64(bits(x), bits(W), bits(A), bits(B), idx, gate)
+    for t in range(T):
+        ref = x[t] @ W.T
+        for s in range(k):
+            e = idx[t, s]
+            ref = ref + gate[t, s] * ((x[t] @ A[e].T) @ B[e].T)
+        assert np.array_equal(y64[t], ref)
+    assert np.array_equal(oracle.bf16_from_f64(y64), oracle.apply_linear(bits(x), bits(W), bits(A), bits(B), idx, gate))
+    part = np.zeros_like(y64)
+    for c0, c1 in ((0, 16), (16, 40), (40, 48)):
+        part += oracle.apply_linear_f64(bits(np.ascontiguousarray(x[:, c0:c1])),
+                                        bits(np.ascontiguousarray(W[:, c0:c1])),
+                                        bits(np.ascontiguousarray(A[:, :, c0:c1])), bits(B), idx, gate)
+    assert np.array_equal(part, y64)
+
+
 def test_apply_zero_gates_is_base_gemm():
     rng = np.random.default_rng(19)
     W, A, B = _rand_adapters(rng, 12, 16, 3, 8)
