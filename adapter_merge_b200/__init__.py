@@ -12,7 +12,7 @@ from typing import Optional, Sequence
 
 __all__ = [
     "AdafuseError", "lib", "library_path", "pregate", "segments", "Plan", "PointerArrays",
-    "RENORM", "POOL_MEAN", "STATUS_BAD_INDEX", "STATUS_TIMEOUT",
+    "RENORM", "POOL_MEAN", "STATUS_BAD_INDEX", "STATUS_TIMEOUT", "PLAN_Y_F32", "round_bf16",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -29,6 +29,7 @@ RENORM = 1 << 0
 POOL_MEAN = 1 << 1
 STATUS_BAD_INDEX = 1 << 0
 STATUS_TIMEOUT = 1 << 1
+PLAN_Y_F32 = 1 << 0
 PLAN_TEST_STALL = 1 << 31
 
 # Every entry point the header declares.
@@ -37,7 +38,7 @@ EXPORTS = (
     "adafuse_switch", "adafuse_merge_per_linear", "adafuse_segments",
     "adafuse_apply_workspace_bytes", "adafuse_apply", "adafuse_plan_status",
     "adafuse_plan_last_launches", "adafuse_strerror", "adafuse_version",
-    "adafuse_apply_noalloc",
+    "adafuse_apply_noalloc", "adafuse_round_bf16",
 )
 
 
@@ -85,6 +86,7 @@ def lib():
     L.adafuse_apply_workspace_bytes.restype = ctypes.c_size_t
     L.adafuse_apply.argtypes = [P, P, P, i64, P, P, i32, P, ctypes.c_size_t, P]
     L.adafuse_apply_noalloc.argtypes = [P, P, P, i64, P, P, i32, P]
+    L.adafuse_round_bf16.argtypes = [P, P, i64, P]
     L.adafuse_plan_status.argtypes = [P, P, ctypes.POINTER(i32)]
     L.adafuse_plan_last_launches.argtypes = [P]
     L.adafuse_plan_last_launches.restype = i32
@@ -143,13 +145,28 @@ def segments(idx, E: int, status=None, stream=None):
     return offsets, perm, used
 
 
+def round_bf16(src, out=None, stream=None):
+    """bf16 round-to-nearest-even of an fp32 device tensor into `out` (a new
+    bf16 tensor of src's shape if None); returns out."""
+    import torch
+    if src.dtype != torch.float32 or not src.is_contiguous():
+        raise ValueError("round_bf16 takes a contiguous fp32 tensor")
+    if out is None:
+        out = torch.empty(src.shape, dtype=torch.bfloat16, device=src.device)
+    if out.dtype != torch.bfloat16 or not out.is_contiguous() or out.numel() != src.numel():
+        raise ValueError("round_bf16 writes a contiguous bf16 tensor of src's size")
+    _check(lib().adafuse_round_bf16(_ptr(src), _ptr(out), src.numel(), _stream(stream)), "adafuse_round_bf16")
+    return out
+
+
 class Plan:
     """A plan over a list of targeted linears sharing E rank-r adapters.
 
     `linears` is a sequence of (W, W_out, A, B) device tensors per linear:
     W, W_out bf16 [d_out, d_in]; A bf16 [E, r, d_in]; B bf16 [E, d_out, r]
     (any expert stride, row-major inside an expert).  The tensors must stay
-    alive while the plan exists.
+    alive while the plan exists.  `flags`: PLAN_Y_F32 makes apply write fp32
+    outputs (the row-parallel partials of tensor parallelism).
     """
 
     def __init__(self, linears: Sequence, E: int, r: int, flags: int = 0):

@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <algorithm>
 #include <utility>
 #include <vector>
 
@@ -76,10 +77,12 @@ struct Plan {
     int32_t last_launches = 0;
     // Per-call apply descriptors: TMA maps of every x_l and of the shrink
     // output, and the x / y pointer tables, rebuilt only when the caller's
-    // pointers, T or workspace change.
+    // pointers, T, k or workspace change (the shrink-output map's base and
+    // extent follow T * k).
     uint8_t* d_call = nullptr;
     bool call_valid = false;
     int64_t call_T = 0;
+    int32_t call_k = 0;
     const void* call_ws = nullptr;
     std::vector<const void*> call_x, call_y;
 };
@@ -95,7 +98,7 @@ int launch_merge_fused(Plan* p, const int32_t* idx0, const float* gate0, const i
                        const float* gate1, int32_t k, int mode, cudaStream_t s);
 int launch_merge_per_linear(Plan* p, const int32_t* idx, const float* gate, int32_t k, cudaStream_t s);
 int launch_segments(const int32_t* idx, int64_t T, int32_t k, int32_t E, int32_t* offsets, int32_t* perm,
-                    int32_t* used, int32_t* status, cudaStream_t s);
+                    int32_t* used, int32_t* status, cudaStream_t s, int32_t* zero = nullptr, int64_t n_zero = 0);
 size_t apply_workspace_bytes(const Plan* p, int64_t T, int32_t k);
 size_t apply_call_bytes(int n_lin);
 int launch_apply(Plan* p, const void* const* x_ptrs, void* const* y_ptrs, int64_t T, const int32_t* idx,

@@ -94,7 +94,7 @@ extern "C" int adafuse_plan_create(adafuse_plan** out, const adafuse_linear* lin
     if (!out || !lins || n_lin < 1) return ADAFUSE_ERR_INVALID_ARG;
     *out = nullptr;
     if (E < 1 || E > kMaxE || r < 8 || r % 8 != 0 || r > kMaxKr) return ADAFUSE_ERR_UNSUPPORTED;
-    if (flags & ~ADAFUSE_PLAN_TEST_STALL) return ADAFUSE_ERR_INVALID_ARG;
+    if (flags & ~(ADAFUSE_PLAN_TEST_STALL | ADAFUSE_PLAN_Y_F32)) return ADAFUSE_ERR_INVALID_ARG;
     for (int l = 0; l < n_lin; ++l) {
         const adafuse_linear& L = lins[l];
         if (!L.W || !L.W_out || !L.A || !L.B) return ADAFUSE_ERR_INVALID_ARG;

@@ -13,7 +13,12 @@ over its shards and calls the same entry points.
       x_s W_s^T + sum_s g_s (x_s A_s^T) B_s^T,
   and because the expand is linear in the shrink, the sum of the ranks'
   partials is the full y: one all-reduce (sum) of y completes it -- the
-  all-reduce a row-parallel layer of the backbone performs anyway.
+  all-reduce a row-parallel layer of the backbone performs anyway.  The
+  partials stay fp32 (a plan built with PLAN_Y_F32): rounding each to bf16
+  before the sum would cost up to half a bf16 ulp per rank, more than the
+  output tolerance where the partials cancel; the sum is rounded once, by the
+  library's round_bf16 kernel.  A rank therefore builds two plans, one over
+  its column-parallel linears and one (PLAN_Y_F32) over its row-parallel ones.
 
 This module only slices tensors and issues that all-reduce; every
 arithmetic step stays in the library's kernels.
@@ -72,12 +77,32 @@ def shard_input(kind: str, x, rank: int, world: int):
     raise ValueError(kind)
 
 
-def reduce_output(kind: str, y, group=None):
-    """Complete a rank's apply output: all-reduce (sum) the partial y of a
-    row-parallel linear; a column-parallel output is already final (its
-    columns).  Every rank must call this in the same order."""
+def plan_flags(kind: str) -> int:
+    """Plan flags for a rank's plan over linears of this kind: fp32 outputs
+    (PLAN_Y_F32) for row-parallel partials, bf16 for column-parallel ones."""
     if kind == ROW:
-        import torch.distributed as dist
-        if dist.is_initialized() and dist.get_world_size(group) > 1:
-            dist.all_reduce(y, op=dist.ReduceOp.SUM, group=group)
-    return y
+        from adapter_merge_b200 import PLAN_Y_F32
+        return PLAN_Y_F32
+    if kind == COLUMN:
+        return 0
+    raise ValueError(kind)
+
+
+def reduce_output(kind: str, y, out=None, group=None):
+    """Complete a rank's apply output.  Column-parallel: y (bf16) is already
+    final, the rank's block of output columns.  Row-parallel: y is the rank's
+    fp32 partial (PLAN_Y_F32); it is all-reduced (sum, in place), and if `out`
+    is given (a bf16 device tensor of y's shape) the sum is rounded once into
+    it by the library and `out` is returned, else the summed partial.  Every
+    rank must call this in the same order."""
+    if kind == COLUMN:
+        return y
+    if kind != ROW:
+        raise ValueError(kind)
+    import torch.distributed as dist
+    if dist.is_initialized() and dist.get_world_size(group) > 1:
+        dist.all_reduce(y, op=dist.ReduceOp.SUM, group=group)
+    if out is None:
+        return y
+    from adapter_merge_b200 import round_bf16
+    return round_bf16(y, out)

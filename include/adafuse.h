@@ -77,6 +77,15 @@ typedef struct CUstream_st* adafuse_stream_t;   /* same type as cudaStream_t */
 #define ADAFUSE_POOL_MEAN  (1u << 1)   /* pregate: one decision for the mean of the T rows */
 
 /* ---- plan flags ---- */
+/* The apply of this plan writes every y_l as fp32 [T, d_out] (4-byte aligned),
+ * the unrounded fp32 accumulator of x W^T + the LoRA term, instead of bf16.
+ * For the row-parallel shards of tensor parallelism (attention output and
+ * down projections split along d_in): each rank's y is a partial sum, and
+ * rounding it to bf16 before the ranks' partials are added loses up to half a
+ * bf16 ulp per partial, more than the output tolerance where the partials
+ * cancel.  With this flag the partials are added in fp32 (the all-reduce) and
+ * rounded once, by adafuse_round_bf16.  Merge and switch are unaffected. */
+#define ADAFUSE_PLAN_Y_F32       (1u << 0)
 /* Test hook for the failure path: every fused merge, switch or apply on a
  * plan created with this flag withholds the first shared-memory stage of CTA 0
  * of the merge or of the fused apply kernel, so that CTA's pipeline wait runs
@@ -113,7 +122,8 @@ typedef struct adafuse_plan adafuse_plan;     /* opaque, library-owned */
  * split of merge and apply, and the status word.  Everything is built once
  * here so that the hot calls do no host work beyond a launch.
  * The `lins` array (host) is copied; the tensors it points to must outlive the
- * plan.  Uses the current CUDA device.  `flags` is 0 or ADAFUSE_PLAN_TEST_STALL.
+ * plan.  Uses the current CUDA device.  `flags`: 0, or ADAFUSE_PLAN_Y_F32
+ * and / or ADAFUSE_PLAN_TEST_STALL.
  * Errors: INVALID_ARG (null pointers, n_lin < 1, other flags), UNSUPPORTED (E outside
  * [1, 32], r not a multiple of 8 or r > 256, d_out/d_in not multiples of 8,
  * misaligned pointers or strides), DEVICE (no sm_100 GPU), CUDA.
@@ -152,9 +162,10 @@ ADAFUSE_API int adafuse_pregate(const void* x, int64_t T, int32_t H, int64_t x_r
  * Fused all-layer merge (page pt section 2.B; page ja section 2.2): for every
  * linear of the plan, W_out = bf16_rne(W + sum_{s<k} gate[s] B_{idx[s]} A_{idx[s]}),
  * accumulated in fp32, in ONE kernel launch over all linears.  The gates are
- * folded into the concatenated A rows (rounded to bf16), the rank-(k*r)
- * contraction runs on the tensor cores, W streams through shared memory by
- * TMA.  idx int32 [k], gate fp32 [k] (device; e.g. row 0 of pregate's output).
+ * folded into one factor of the concatenated product, rounded to bf16: into
+ * the B rows (g_s B_{e_s}) when k*r <= 128, into the A rows (g_s A_{e_s})
+ * when k*r is above 128 (up to 256).  The rank-(k*r) contraction runs on the
+ * tensor cores, W streams through shared memory by TMA.  idx int32 [k], gate fp32 [k] (device; e.g. row 0 of pregate's output).
  * In place when W_out == W.
  * Errors: INVALID_ARG, UNSUPPORTED (k < 1, k > E, k*r > 256).
  */
@@ -205,24 +216,27 @@ ADAFUSE_API size_t adafuse_apply_workspace_bytes(const adafuse_plan* plan, int64
 /*
  * Segmented-gather apply, unmerged, for every linear of the plan:
  *   y_l[t, :] = bf16_rne( x_l[t, :] W_l^T + sum_s gate[t,s] (x_l[t, :] A_{idx[t,s]}^T) B_{idx[t,s]}^T )
- * with fp32 accumulation.  Four launches, whatever the number of linears:
+ * with fp32 accumulation.  Two launches, whatever the number of linears: the
  * segment build (stable sort of the pairs by expert; gives the U experts the
- * batch uses), shrink (the used experts' A rows times x^T on the tensor cores,
- * split over 1024-column K-slices, 256 for small plans), finalize (slices summed in order, gates
- * applied, kept as a pair of bf16 values whose sum is the fp32 result), then
- * one tensor-core kernel over all linears that streams W once and adds the
- * expand (the used experts' B rows against both halves of the shrink) into
- * the same fp32 accumulator.
+ * batch uses), then one persistent tensor-core kernel over all linears that
+ * runs the shrink first (the used experts' A rows times x^T, split over
+ * 1024-column K-slices, 256 for small plans; the last slice of each tile to
+ * finish adds the slices in order, applies the gates and keeps the result as
+ * a pair of bf16 values whose sum is the fp32 result), then streams W once
+ * and adds the expand (the used experts' B rows against both halves of the
+ * shrink) into the same fp32 accumulator, each linear's expand starting once
+ * its shrink is complete.
  *   x_ptrs   HOST array [n_lin] of device pointers, x_l bf16 [T, d_in_l] row-major,
  *            16-byte aligned
  *   y_ptrs   HOST array [n_lin] of device pointers, y_l bf16 [T, d_out_l] row-major
+ *            (fp32, 4-byte aligned, for a plan created with ADAFUSE_PLAN_Y_F32)
  *   idx/gate int32 / fp32 [T, k] (device), e.g. pregate's output
  *   workspace device, >= adafuse_apply_workspace_bytes(plan, T, k), 256-byte aligned
  * The call builds TMA descriptors for the x_l and the workspace and uploads
  * them (with the pointer tables) on `stream`; they are kept in the plan and
- * rebuilt only when the pointers, T or the workspace differ from the previous
- * call, so a serving loop that reuses its buffers does no host work beyond the
- * four launches.  The apply kernel's work units cover 512, 256 or 128 output
+ * rebuilt only when the pointers, T, k or the workspace differ from the
+ * previous call, so a serving loop that reuses its buffers does no host work
+ * beyond the two launches.  The apply kernel's work units cover 512, 256 or 128 output
  * rows with token tiles of 64, 128 or 256 (taller units for smaller T, as long
  * as the plan has two units per SM; with fewer than one per SM, units are
  * split along K and their fp32 partials added in a fixed order); T larger
@@ -249,7 +263,8 @@ ADAFUSE_API int adafuse_apply(adafuse_plan* plan, const void* const* x_ptrs, voi
  * workspace at all.  It calls no cudaMalloc, cudaFree or other allocating
  * routine, on the device or the host.
  *   - Limit: the call needs adafuse_apply_workspace_bytes(plan, T, k) plus
- *     about 128 bytes per linear for descriptors; if that exceeds 16 MiB it
+ *     (n_lin + 1) * 128 + n_lin * 8 bytes of descriptors, rounded up to a
+ *     multiple of 256; if that exceeds 16 MiB it
  *     returns ADAFUSE_ERR_WORKSPACE_TOO_SMALL and launches nothing (e.g. the
  *     224-linear Llama-2-7B plan with E = 8, r = 16, top-2 fits up to T = 16).
  *     At most 1024 linears (ADAFUSE_ERR_UNSUPPORTED beyond).
@@ -269,6 +284,21 @@ ADAFUSE_API int adafuse_apply(adafuse_plan* plan, const void* const* x_ptrs, voi
 ADAFUSE_API int adafuse_apply_noalloc(adafuse_plan* plan, const void* const* x_ptrs, void* const* y_ptrs,
                                       int64_t T, const int32_t* idx, const float* gate, int32_t k,
                                       adafuse_stream_t stream);
+
+/*
+ * Round fp32 values to bf16, round-to-nearest-even: out[i] = bf16_rne(in[i])
+ * for i < n (values above the bf16 range become +-inf, NaN stays NaN).  The
+ * last step of a tensor-parallel row-parallel apply: the ranks' fp32 partial
+ * outputs (ADAFUSE_PLAN_Y_F32) are summed by the caller's all-reduce, and this
+ * rounds the sum once, as the unsharded apply rounds its accumulator (page ja
+ * section 2.2 computes the fused product across layers; the sharding is this
+ * library's extension for multi-GPU serving).
+ *   in   device fp32 [n], 4-byte aligned
+ *   out  device bf16 [n], 2-byte aligned, not overlapping in
+ * One launch.  Errors: INVALID_ARG (null pointer with n > 0, n < 0, misaligned or
+ * overlapping buffers).  n == 0 launches nothing.
+ */
+ADAFUSE_API int adafuse_round_bf16(const float* in, void* out, int64_t n, adafuse_stream_t stream);
 
 /*
  * Synchronise `stream`, read the plan's device status word into

@@ -71,3 +71,58 @@ class Model:
                 self.W_out.append(self.W_out_flat[o:o + n].view(l.d_out, l.d_in))
                 o += n
         self.plan = am.Plan(list(zip(self.w.W_views, self.W_out, self.w.A_views, self.w.B_views)), cfg.E, cfg.r)
+
+
+def block_rows(d_out: int, salt: int, per_block: int = 2):
+    """Rows to check in every 128-row block of a linear: `per_block` rows per
+    block, their offsets inside the block rotating with the block index and
+    `salt` (e.g. the linear's index), so that over a model every tile of every
+    linear is checked and every TMEM lane quarter / epilogue warp of a tile is
+    reached."""
+    rows = []
+    for b in range((d_out + 127) // 128):
+        for q in range(per_block):
+            off = (7 * b + 3 * salt + q * (128 // per_block)) % 128
+            rows.append(min(b * 128 + off, d_out - 1))
+    return sorted(set(rows))
+
+
+def take_experts(A, B, slots, rows=None):
+    """The A and B stacks of the experts named in `slots` only (bit-for-bit
+    slices, on the device), with B cut to `rows`, and the slot indices
+    renumbered into the slices: the oracle then indexes exactly the operands
+    it would index in the whole stacks, at a fraction of the transfer.
+    Returns (A_sel [U, r, d_in], B_sel [U, len(rows), r], idx [len(slots)])
+    as host uint16 / int32 arrays."""
+    slots = [int(e) for e in slots]
+    uniq = sorted(set(slots))
+    pos = {e: i for i, e in enumerate(uniq)}
+    dev = A.device
+    sel = torch.tensor(uniq, dtype=torch.long, device=dev)
+    A_sel = A.index_select(0, sel)
+    B_sel = B.index_select(0, sel)
+    if rows is not None:
+        B_sel = B_sel.index_select(1, torch.as_tensor(rows, dtype=torch.long, device=dev))
+    return u16(A_sel), u16(B_sel), np.array([pos[e] for e in slots], dtype=np.int32)
+
+
+def merge_delta_bound_ok(W_out, W, A, B, slots, gates):
+    """A property of a merge that holds at any size, checked on the device over
+    every element of one linear: |W'_gpu - W| <= sum_s |g_s| * ||B_{e_s}[o, :]||_1
+    * max_j |A_{e_s}[j, i]| (a bound on |sum_s g_s B A|, with 1 % slack for the
+    bf16 rounding of the gated factor) + 2^-8 |W'_gpu| (the output rounding),
+    and every element finite.  It catches unwritten tiles (the output is filled
+    with NaN first) and tiles computed from another tile's W."""
+    Wf = W.float()
+    d = (W_out.float() - Wf).abs()
+    bound = torch.zeros_like(d)
+    for e, g in zip(slots, gates):
+        e = int(e)
+        if e < 0:
+            continue
+        brow = B[e].float().abs().sum(dim=1)               # [d_out]
+        acol = A[e].float().abs().amax(dim=0)              # [d_in]
+        bound.add_(torch.outer(brow, acol), alpha=abs(float(g)))
+    bound.mul_(1.01).add_(W_out.float().abs(), alpha=2.0 ** -8).add_(1e-30)
+    ok = bool(torch.isfinite(W_out.float()).all()) and bool((d <= bound).all())
+    return ok

@@ -77,7 +77,8 @@ def test_argument_errors_need_no_device(L):
     assert L.adafuse_plan_create(ctypes.byref(h), arr, 1, 0, 8, 0) == am.ERR_UNSUPPORTED
     assert L.adafuse_plan_create(ctypes.byref(h), arr, 1, 4, 12, 0) == am.ERR_UNSUPPORTED
     assert L.adafuse_plan_create(ctypes.byref(h), arr, 1, 4, 8, 3) == am.ERR_INVALID_ARG
-    assert L.adafuse_plan_create(ctypes.byref(h), arr, 1, 4, 8, (1 << 31) | 1) == am.ERR_INVALID_ARG
+    assert L.adafuse_plan_create(ctypes.byref(h), arr, 1, 4, 8, (1 << 31) | 2) == am.ERR_INVALID_ARG
+    assert L.adafuse_plan_create(ctypes.byref(h), arr, 1, 4, 8, am.PLAN_Y_F32 | 4) == am.ERR_INVALID_ARG
     bad = (am.Linear * 1)(am.Linear(4096 + 2, 8192, 16384, 32768, 16, 16, 128, 128))
     assert L.adafuse_plan_create(ctypes.byref(h), bad, 1, 4, 8, 0) == am.ERR_UNSUPPORTED
     bad = (am.Linear * 1)(am.Linear(4096, 8192, 16384, 32768, 12, 16, 128, 128))
@@ -92,6 +93,15 @@ def test_argument_errors_need_no_device(L):
     assert L.adafuse_apply_workspace_bytes(None, 4, 2) == 0
     v = ctypes.c_int32(0)
     assert L.adafuse_plan_status(None, None, ctypes.byref(v)) == am.ERR_INVALID_ARG
+    # rounding: null buffers, negative n, misaligned or overlapping buffers (no launch)
+    assert L.adafuse_round_bf16(None, fake, 4, None) == am.ERR_INVALID_ARG
+    assert L.adafuse_round_bf16(fake, None, 4, None) == am.ERR_INVALID_ARG
+    assert L.adafuse_round_bf16(fake, fake, -1, None) == am.ERR_INVALID_ARG
+    assert L.adafuse_round_bf16(P(258), P(4096), 4, None) == am.ERR_INVALID_ARG
+    assert L.adafuse_round_bf16(P(256), P(4097), 4, None) == am.ERR_INVALID_ARG
+    assert L.adafuse_round_bf16(P(256), P(256 + 14), 4, None) == am.ERR_INVALID_ARG
+    assert L.adafuse_round_bf16(P(256 + 6), P(256), 4, None) == am.ERR_INVALID_ARG
+    assert L.adafuse_round_bf16(None, None, 0, None) == am.OK
     assert L.adafuse_plan_last_launches(None) == 0
     L.adafuse_plan_destroy(None)
 

@@ -5,13 +5,17 @@ Acceptance: expert indices bit-exact; gates |d| <= 1e-6 + 1e-5 |g|; bf16
 outputs |d| <= 1e-2 |ref| + 1e-3 elementwise, and for the merge also the
 delta check in Frobenius norm (helpers.assert_delta_frobenius).
 """
+import concurrent.futures
+import os
+
 import numpy as np
 import pytest
 import torch
 
 import oracle
 import synth
-from helpers import ATOL, RTOL, Model, assert_close_bf16, assert_delta_frobenius, f64, u16
+from helpers import (ATOL, RTOL, Model, assert_close_bf16, assert_delta_frobenius, block_rows, f64,
+                     merge_delta_bound_ok, take_experts, u16)
 
 pytestmark = pytest.mark.gpu
 
@@ -363,7 +367,7 @@ def test_apply_tiny_chain_with_pregate(am, cuda_device):
     assert np.array_equal(idx.cpu().numpy(), idx_ref)
     check_apply(m, xs, ys, idx_ref, gate_ref, "tiny apply")
     assert m.plan.status() == (0, 0)
-    assert m.plan.last_launches == 4
+    assert m.plan.last_launches == 2
 
 
 # T <= 64, 65..128 and > 128 take apply units of 512, 256 and 128 output rows;
@@ -456,6 +460,28 @@ def test_apply_descriptor_cache_follows_pointers_and_T(am, cuda_device):
         check_apply(m, xs, ys, idx.numpy(), gate.numpy().astype(np.float64), f"cache T={T} seed={seed}")
 
 
+def test_apply_descriptor_cache_follows_k(am, cuda_device):
+    """Same plan, T, workspace and x / y buffers, but top-1, then top-2, then
+    top-1 again: the shrink output's place and width in the workspace follow
+    T * k, so the cached descriptors must be rebuilt when k changes."""
+    T = 64
+    cfg = synth.custom([(256, 392), (136, 264)], 6, 16, 2, T, name="acachek")
+    m = Model(cfg, cuda_device)
+    X, xs = synth.make_apply_inputs(cfg, T, 4)
+    xd = [x.to(cuda_device) for x in xs]
+    ys = [torch.empty((T, l.d_out), dtype=torch.bfloat16, device=cuda_device) for l in cfg.linears]
+    xp = am.PointerArrays(xd, ys)
+    ws = torch.empty(max(m.plan.workspace_bytes(T, k) for k in (1, 2)), dtype=torch.uint8, device=cuda_device)
+    for k in (1, 2, 1):
+        idx, gate = synth.random_selection(T, cfg.E, k, 10 + k, "acachek")
+        for y in ys:
+            y.fill_(float("nan"))
+        m.plan.apply(xp, None, T, idx.to(cuda_device), gate.to(cuda_device), ws)
+        torch.cuda.synchronize()
+        check_apply(m, xs, ys, idx.numpy(), gate.numpy().astype(np.float64), f"cache k={k}")
+    assert m.plan.status() == (0, 0)
+
+
 def test_apply_equals_merged_weights(am, cuda_device):
     """Merged form equals unmerged: with one shared selection, apply(x) agrees
     with x W'^T for the GPU's own merged W' to within the bf16 rounding of W'."""
@@ -475,122 +501,168 @@ def test_apply_equals_merged_weights(am, cuda_device):
 
 # ------------------------------------------------------------- full sizes
 
-def sampled_rows(lin, n=3):
-    return [(0, 1), (lin.d_out // 2, lin.d_out // 2 + 1), (lin.d_out - 1, lin.d_out)][:n]
+ORACLE_THREADS = max(1, min(16, os.cpu_count() or 1))
+
+
+def merge_rows_check(W_out, W, A, B, rows, slots, gates, what, base=None, base_slots=None, base_gates=None):
+    """The oracle on `rows` of one linear, against the GPU's rows.  Merge: rows of
+    bf16(W + sum_s g_s B A).  With `base` set (a switch), the expected rows are
+    the oracle's switch of the oracle's own merge of `base_slots`: rows are
+    independent, so each one is exact whatever rows are left out."""
+    rt = torch.as_tensor(rows, dtype=torch.long, device=W.device)
+    W_rows = u16(W.index_select(0, rt))
+    got = u16(W_out.index_select(0, rt))
+    all_slots = list(slots) + (list(base_slots) if base is not None else [])
+    A_sel, B_sel, ii = take_experts(A, B, all_slots, rows)
+    ns = len(slots)
+    if base is None:
+        ref = oracle.merge_linear(W_rows, A_sel, B_sel, ii, gates, nthreads=ORACLE_THREADS)
+        assert_close_bf16(got, ref, what)
+        dz = oracle.merge_linear(np.zeros_like(W_rows), A_sel, B_sel, ii, gates, nthreads=ORACLE_THREADS)
+        assert_delta_frobenius(got, W_rows, ref, dz, what)
+    else:
+        cur = oracle.merge_linear(W_rows, A_sel, B_sel, ii[ns:], base_gates, nthreads=ORACLE_THREADS)
+        ref = oracle.merge_linear(cur, A_sel, B_sel, list(ii[:ns]) + list(ii[ns:]),
+                                  list(gates) + [-g for g in base_gates], nthreads=ORACLE_THREADS)
+        assert_close_bf16(got, ref, what)
 
 
 @pytest.mark.parametrize("cfg_fn", [synth.llama7b, synth.llama13b])
-def test_full_size_merge_sampled(am, cuda_device, cfg_fn):
-    """Full model, in the benchmark's launch configuration: pregate on one
-    token, one merge launch over every linear; sampled rows of a spread of
-    linears against the oracle (rows are independent, so a row is exact)."""
+def test_full_size_merge_every_tile(am, cuda_device, cfg_fn):
+    """Full model in the benchmark's launch configuration: pregate on one
+    token, then ONE merge launch over every linear.  Against the oracle: two
+    rows in every 128-row block of every linear (their offsets inside the
+    block rotating with the block and the linear, so every tile of every
+    linear, every row-block group and its tail, and every CTA's range is
+    checked), with the delta check per linear.  On every element: written
+    (the output starts as NaN) and within a bound on |dW|.  Then the in-place
+    switch to another selection, checked the same way against the oracle's
+    switch of the oracle's merged rows."""
     cfg = cfg_fn()
     m = Model(cfg, cuda_device)
+    m.W_out_flat.fill_(float("nan"))
     xr = synth.make_router_input(cfg, 1, 0, device=cuda_device)
     idx, gate = am.pregate(xr, m.w.W_r, cfg.k)
     m.plan.merge(idx[0], gate[0])
     torch.cuda.synchronize()
+    assert m.plan.status() == (0, 0)
     idx_ref, gate_ref, _ = oracle.pregate(u16(xr), m.w.W_r.cpu().numpy(), cfg.k)
     assert np.array_equal(idx.cpu().numpy(), idx_ref)
+    sel = [int(e) for e in idx_ref[0]]
     g = gate.cpu().numpy()[0].astype(np.float64)
-    picks = sorted(set([0, 1, 4, 6, cfg.n_lin // 2, cfg.n_lin // 2 + 5, cfg.n_lin - 1]))
-    for l in picks:
-        lin = cfg.linears[l]
-        W, A, B = u16(m.w.W_views[l]), u16(m.w.A_views[l]), u16(m.w.B_views[l])
-        for rr in sampled_rows(lin):
-            ref = oracle.merge_linear(W, A, B, idx_ref[0], g, rows=rr)
-            got = u16(m.W_out[l][rr[0]:rr[1]])
-            assert_close_bf16(got, ref, f"{cfg.name} linear {l} rows {rr}")
-            dz = oracle.merge_linear(np.zeros_like(W), A, B, idx_ref[0], g, rows=rr)
-            assert_delta_frobenius(got, W[rr[0]:rr[1]], ref, dz, f"{cfg.name} linear {l} rows {rr}")
-    assert m.plan.status() == (0, 0)
+    checked = 0
+    for l, lin in enumerate(cfg.linears):
+        Wl, Ol, Al, Bl = m.w.W_views[l], m.W_out[l], m.w.A_views[l], m.w.B_views[l]
+        assert merge_delta_bound_ok(Ol, Wl, Al, Bl, sel, g), f"{cfg.name} merge linear {l}: bound or NaN"
+        rows = block_rows(lin.d_out, l)
+        merge_rows_check(Ol, Wl, Al, Bl, rows, sel, g, f"{cfg.name} merge linear {l}")
+        checked += len(rows)
+    assert checked >= 2 * sum((l.d_out + 127) // 128 for l in cfg.linears)
 
-    # In-place switch to another selection at full size (rank 2kr, the same
-    # launch configuration as the benchmark's switch): sampled rows against
-    # the oracle's switch of the oracle's own merged rows.
-    new_i = np.array([(int(idx_ref[0][s]) + 1 + s) % cfg.E for s in range(cfg.k)], dtype=np.int32)
-    if len(set(new_i.tolist())) < cfg.k:
-        new_i = np.arange(cfg.k, dtype=np.int32)
+    new_i = [(sel[s] + 1 + s) % cfg.E for s in range(cfg.k)]
+    if len(set(new_i)) < cfg.k:
+        new_i = list(range(cfg.k))
     new_g = np.linspace(0.5, 0.2, cfg.k).astype(np.float32)
-    d = lambda a_, t: torch.as_tensor(a_.astype(t)).to(cuda_device)
+    d = lambda a_, t: torch.as_tensor(np.asarray(a_).astype(t)).to(cuda_device)
     m.plan.switch(d(new_i, np.int32), d(new_g, np.float32), idx[0], gate[0])
     torch.cuda.synchronize()
-    for l in picks[:4]:
-        lin = cfg.linears[l]
-        W, A, B = u16(m.w.W_views[l]), u16(m.w.A_views[l]), u16(m.w.B_views[l])
-        for rr in sampled_rows(lin)[:2]:
-            cur = oracle.merge_linear(W, A, B, idx_ref[0], g, rows=rr)
-            Bs = np.ascontiguousarray(B[:, rr[0]:rr[1], :])           # the same rows of the B stack
-            ref = oracle.merge_linear(cur, A, Bs, list(new_i) + list(idx_ref[0]),
-                                      list(new_g.astype(np.float64)) + list(-g))
-            assert_close_bf16(u16(m.W_out[l][rr[0]:rr[1]]), ref, f"{cfg.name} switch linear {l} rows {rr}")
     assert m.plan.status() == (0, 0)
+    for l, lin in enumerate(cfg.linears):
+        Wl, Ol, Al, Bl = m.w.W_views[l], m.W_out[l], m.w.A_views[l], m.w.B_views[l]
+        assert bool(torch.isfinite(Ol.float()).all()), f"{cfg.name} switch linear {l}: non-finite"
+        rows = block_rows(lin.d_out, l + 61, per_block=1)
+        merge_rows_check(Ol, Wl, Al, Bl, rows, new_i, list(new_g.astype(np.float64)),
+                         f"{cfg.name} switch linear {l}", base=True, base_slots=sel, base_gates=list(g))
 
 
 @pytest.mark.parametrize("cfg_fn", [synth.llama7b, synth.llama13b])
-def test_full_size_apply_sampled(am, cuda_device, cfg_fn):
-    """Batched decode at full size: per-sequence routing on each sequence's
-    first token, one apply over every linear; sampled (linear, token) rows
-    against the oracle."""
+def test_full_size_apply_every_unit(am, cuda_device, cfg_fn):
+    """Batched decode at full size in the benchmark's launch configuration:
+    per-sequence routing on each sequence's first token, then ONE apply over
+    every linear.  Against the oracle: two whole tokens of every linear (a
+    token's row of y spans every apply unit of the linear), the tokens
+    rotating with the linear index.  On every element: written (y starts as
+    NaN)."""
     cfg = cfg_fn()
     T = cfg.T_apply
     m = Model(cfg, cuda_device)
     X, xs_dev = synth.make_apply_inputs(cfg, T, 0, device=cuda_device)
-    ys = [torch.empty((T, l.d_out), dtype=torch.bfloat16, device=cuda_device) for l in cfg.linears]
+    Y = torch.full((sum(T * l.d_out for l in cfg.linears),), float("nan"), dtype=torch.bfloat16,
+                   device=cuda_device)
+    ys, o = [], 0
+    for l in cfg.linears:
+        ys.append(Y[o:o + T * l.d_out].view(T, l.d_out))
+        o += T * l.d_out
     xp = am.PointerArrays(xs_dev, ys)
-    yp = None
     xr = synth.make_router_input(cfg, T, 0, device=cuda_device, tag="xfirst")
     idx, gate = am.pregate(xr, m.w.W_r, cfg.k)
     ws = torch.empty(m.plan.workspace_bytes(T, cfg.k), dtype=torch.uint8, device=cuda_device)
-    m.plan.apply(xp, yp, T, idx, gate, ws)
+    m.plan.apply(xp, None, T, idx, gate, ws)
     torch.cuda.synchronize()
+    assert m.plan.status() == (0, 0)
+    assert bool(torch.isfinite(Y.float()).all()), "apply left outputs unwritten"
     idx_ref, gate_ref, _ = oracle.pregate(u16(xr), m.w.W_r.cpu().numpy(), cfg.k)
     assert np.array_equal(idx.cpu().numpy(), idx_ref)
     g = gate.cpu().numpy().astype(np.float64)
-    picks = sorted(set([0, 3, 4, 6, cfg.n_lin // 2, cfg.n_lin - 1]))
-    for l in picks:
-        W, A, B = u16(m.w.W_views[l]), u16(m.w.A_views[l]), u16(m.w.B_views[l])
-        x = u16(xs_dev[l])
-        for t in (0, T // 2, T - 1):
-            ref = oracle.apply_linear(x, W, A, B, idx_ref, g, tokens=(t, t + 1), nthreads=8)
-            assert_close_bf16(u16(ys[l][t:t + 1]), ref, f"{cfg.name} apply linear {l} token {t}")
-    assert m.plan.status() == (0, 0)
+
+    def job(l, W, A, B, x, toks, got):
+        for t, row in zip(toks, got):
+            ref = oracle.apply_linear(x, W, A, B, idx_ref, g, tokens=(t, t + 1), nthreads=1)
+            assert_close_bf16(row[None, :], ref, f"{cfg.name} apply linear {l} token {t}")
+        return len(toks)
+
+    checked = 0
+    with concurrent.futures.ThreadPoolExecutor(ORACLE_THREADS) as pool:
+        futs = []
+        for l in range(cfg.n_lin):
+            toks = sorted({(3 * l) % T, (3 * l + T // 2 + 1) % T})
+            got = u16(ys[l])[toks]
+            futs.append(pool.submit(job, l, u16(m.w.W_views[l]), u16(m.w.A_views[l]), u16(m.w.B_views[l]),
+                                    u16(xs_dev[l]), toks, got))
+            if len(futs) >= 2 * ORACLE_THREADS:          # bound the host copies in flight
+                checked += futs.pop(0).result()
+        for f in futs:
+            checked += f.result()
+    assert checked >= cfg.n_lin
 
 
 # ------------------------------------------------------------------- sweep
 
-SWEEP = [  # (E, r, k, T): single 4096 x 4096 linear, every value of each axis covered
-    (4, 8, 1, 1), (8, 16, 2, 16), (16, 32, 4, 128), (32, 64, 2, 1), (4, 64, 4, 16),
-    (32, 8, 4, 128), (8, 32, 1, 128), (16, 16, 2, 1), (32, 64, 4, 16), (4, 16, 4, 1),
-]
+SWEEP_GRID = [(E, r, k) for E in (4, 8, 16, 32) for r in (8, 16, 32, 64) for k in (1, 2, 4)
+              if k <= E and k * r <= 256]
 
 
-@pytest.mark.parametrize("E,r,k,T", SWEEP)
-def test_sweep_point_merge_and_apply(am, cuda_device, E, r, k, T):
-    """The single-layer sweep: gates from the softmax of N(0,1) logits; merge
-    (sampled rows, with the delta check) and apply at batch T (all tokens for
-    T <= 16, sampled tokens above)."""
-    cfg = synth.sweep_point(E, r, k, T)
+@pytest.mark.parametrize("E,r,k", SWEEP_GRID)
+def test_sweep_point_merge_and_apply(am, cuda_device, E, r, k):
+    """Every (E, r, k) of the single-layer sweep (4096 x 4096 W, gates from the
+    softmax of N(0, 1) logits): the merge on two rows of every 128-row block
+    (delta check included) and the apply at batch 1, 16 and 128 on every
+    token up to 16 and on eight rotating tokens at 128."""
+    cfg = synth.sweep_point(E, r, k, 128)
     m = Model(cfg, cuda_device)
-    z = synth.normal((T, E), 1.0, torch.float32, 9, f"sweep-logits-{E}-{T}").numpy()
+    m.W_out_flat.fill_(float("nan"))
+    z = synth.normal((128, E), 1.0, torch.float32, 9, f"sweep-logits-{E}-{r}-{k}").numpy()
     idx, gate = oracle.topk_softmax(z, k)
     gate32 = gate.astype(np.float32)
     run_merge(am, m, idx[0], gate32[0], cuda_device)
-    W, A, B = u16(m.w.W_views[0]), u16(m.w.A_views[0]), u16(m.w.B_views[0])
-    for rr in ((0, 2), (2047, 2049), (4090, 4096)):
-        ref = oracle.merge_linear(W, A, B, idx[0], gate32[0].astype(np.float64), rows=rr)
-        got = u16(m.W_out[0][rr[0]:rr[1]])
-        assert_close_bf16(got, ref, f"sweep merge rows {rr}")
-        dz = oracle.merge_linear(np.zeros_like(W), A, B, idx[0], gate32[0].astype(np.float64), rows=rr)
-        assert_delta_frobenius(got, W[rr[0]:rr[1]], ref, dz, f"sweep merge rows {rr}")
-    X, xs = synth.make_apply_inputs(cfg, T, 9)
-    xd = [x.to(cuda_device) for x in xs]
-    ys = [torch.empty((T, 4096), dtype=torch.bfloat16, device=cuda_device)]
-    ws = torch.empty(m.plan.workspace_bytes(T, k), dtype=torch.uint8, device=cuda_device)
-    m.plan.apply(xd, ys, T, torch.as_tensor(idx).to(cuda_device), torch.as_tensor(gate32).to(cuda_device), ws)
-    torch.cuda.synchronize()
-    toks = [(0, T)] if T <= 16 else [(0, 1), (T // 2, T // 2 + 1), (T - 1, T)]
-    for tt in toks:
-        ref = oracle.apply_linear(u16(xs[0]), W, A, B, idx, gate32.astype(np.float64), tokens=tt, nthreads=8)
-        assert_close_bf16(u16(ys[0][tt[0]:tt[1]]), ref, f"sweep apply tokens {tt}")
+    Wl, Ol, Al, Bl = m.w.W_views[0], m.W_out[0], m.w.A_views[0], m.w.B_views[0]
+    g0 = gate32[0].astype(np.float64)
+    assert merge_delta_bound_ok(Ol, Wl, Al, Bl, idx[0], g0), "sweep merge: bound or NaN"
+    merge_rows_check(Ol, Wl, Al, Bl, block_rows(4096, E + r + k), idx[0], g0, f"sweep E{E} r{r} k{k} merge")
+    W, A, B = u16(Wl), u16(Al), u16(Bl)
+    for T in (1, 16, 128):
+        X, xs = synth.make_apply_inputs(cfg, T, 9)
+        xd = [x.to(cuda_device) for x in xs]
+        ys = [torch.full((T, 4096), float("nan"), dtype=torch.bfloat16, device=cuda_device)]
+        ws = torch.empty(m.plan.workspace_bytes(T, k), dtype=torch.uint8, device=cuda_device)
+        ii, gg = idx[:T], gate32[:T]
+        m.plan.apply(xd, ys, T, torch.as_tensor(ii).to(cuda_device), torch.as_tensor(gg).to(cuda_device), ws)
+        torch.cuda.synchronize()
+        assert bool(torch.isfinite(ys[0].float()).all()), f"sweep apply T={T}: unwritten outputs"
+        toks = range(T) if T <= 16 else sorted({(E + r + k + 17 * j) % T for j in range(8)} | {0, T - 1})
+        x = u16(xs[0])
+        got = u16(ys[0])
+        for t in toks:
+            ref = oracle.apply_linear(x, W, A, B, ii, gg.astype(np.float64), tokens=(t, t + 1))
+            assert_close_bf16(got[t:t + 1], ref, f"sweep E{E} r{r} k{k} apply T={T} token {t}")
     assert m.plan.status() == (0, 0)

@@ -5,8 +5,9 @@ synchronise the device).  Instead of a caller-provided workspace it uses a
 fixed 16 MiB array in the library's own device memory.
 
 These tests call it through the C ABI and check it against the regular
-adafuse_apply on the same inputs, on two calls in a row (the array keeps the
-previous call's contents, which must not leak into the next result), and check
+adafuse_apply on the same inputs, and against the oracle, on two calls in a
+row (the array keeps the previous call's contents, which must not leak into
+the next result), and check
 that a call too big for the array is refused before anything is launched.
 This file is collected last so that a run stopping at its first failure has
 already run every other test.
@@ -15,6 +16,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 import synth
 from helpers import Model, assert_close_bf16, u16
 
@@ -48,6 +50,11 @@ def test_noalloc_apply_matches_apply_on_two_calls_in_a_row(am, cuda_device):
         torch.cuda.synchronize()
         for l in range(cfg.n_lin):
             assert_close_bf16(u16(y[l]), u16(y_ref[l]), f"no-alloc apply, call T={T}, linear {l}")
+            # and directly against the oracle, so this test stands on its own
+            ref = oracle.apply_linear(u16(xs[l]), u16(m.w.W_views[l]), u16(m.w.A_views[l]),
+                                      u16(m.w.B_views[l]), idx.cpu().numpy(),
+                                      gate.cpu().numpy().astype(np.float64))
+            assert_close_bf16(u16(y[l]), ref, f"no-alloc apply vs oracle, call T={T}, linear {l}")
         assert m.plan.status() == (0, 0)
 
 
