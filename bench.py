@@ -45,26 +45,30 @@ def read_peaks():
     return FALLBACK_HBM_GBS, "fallback"
 
 
-def profiled_traffic(kernel_files, summary, key):
-    """DRAM bytes per launch recorded in a profiles/ summary, if the kernel's
-    sources still hash to the fingerprint recorded with them; else None."""
+RECORDS = os.path.join(ROOT, "profiles", "records.json")
+
+
+def kernel_fingerprint(files):
+    """First 16 hex digits of the sha256 of the kernel's source files (csrc/)."""
     import hashlib
-    path = os.path.join(ROOT, "profiles", summary)
-    if not os.path.exists(path):
-        return None
-    rec = {}
-    with open(path) as fh:
-        for line in fh:
-            parts = line.strip().split(":")
-            if len(parts) == 2:
-                rec[parts[0].strip()] = parts[1].strip()
     h = hashlib.sha256()
-    for f in kernel_files:
+    for f in files:
         with open(os.path.join(ROOT, "adapter_merge_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
-    if rec.get("kernel_sources_sha256_16") != h.hexdigest()[:16] or key not in rec:
+    return h.hexdigest()[:16]
+
+
+def profile_record(kernel):
+    """The ncu figures recorded for `kernel` in profiles/records.json, if its
+    sources still hash to the fingerprint recorded with them; else None (the
+    counters describe another build)."""
+    if not os.path.exists(RECORDS):
         return None
-    return int(rec[key])
+    with open(RECORDS) as fh:
+        rec = json.load(fh).get(kernel)
+    if not rec or rec.get("kernel_sources_sha256_16") != kernel_fingerprint(rec["sources"]):
+        return None
+    return rec
 
 
 def merge_bytes(cfg, k):
@@ -269,33 +273,23 @@ def sweep_point_arg(text):
     return pt
 
 
-def run_sweep(args):
+def measure_sweep(dev, peak, only=None, NC=8, R=5, Ts=(1, 16, 128)):
     """The single-linear 4096 x 4096 grid: E in {4, 8, 16, 32}, r in {8, 16,
-    32, 64}, k in {1, 2, 4}; merge per (E, r, k) and apply per T in {1, 16,
-    128}.  A 33.5 MB layer fits in the 126 MB L2, so every point rotates
-    through 8 independent copies (W, W', A, B and a plan each, 8 x 100+ MB
-    touched per cycle) and each launch finds its operands in HBM.  Per point:
-    the device time of one call (CUDA events around it, median; a GPU sleep
+    32, 64}, k in {1, 2, 4}; merge per (E, r, k) and apply per T in Ts.  A
+    33.5 MB layer fits in the 126 MB L2, so every point rotates through NC
+    independent copies (W, W', A, B and a plan each, NC x 100+ MB touched per
+    cycle) and each launch finds its operands in HBM.  Per point: the device
+    time of one call (CUDA events around it, median of NC * R; a GPU sleep
     queued before the first event keeps the device busy until the host has
     queued the whole call, so host time does not count), the time per call
     when calls run back to back (launch gaps and host time included), and the
     host time of the API call (launch overhead)."""
     import torch
     import adapter_merge_b200 as am
-    from adapter_merge_b200 import build as ambuild
     import synth
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    ambuild.build()
-    peak, peak_kind = read_peaks()
     stream = torch.cuda.current_stream()
-    only = sweep_point_arg(args.point)
-    NC, R = 8, 5                          # copies, rounds over the copies
     SLEEP_CYCLES = 1_000_000              # ~0.5 ms of GPU sleep ahead of each timed call
     points = []
-    t_begin = time.perf_counter()
     for E in (4, 8, 16, 32):
         for r in (8, 16, 32, 64):
             for k in (1, 2, 4):
@@ -346,7 +340,7 @@ def run_sweep(args):
                                 "back_to_back_us": round(m_b2b * 1e3, 2), "host_us_per_call": round(m_host, 2),
                                 "bytes": mb},
                       "apply": []}
-                for T in (1, 16, 128):
+                for T in Ts:
                     X, xs = synth.make_apply_inputs(cfg, T, 5, device=dev)
                     ys = [torch.empty((T, lin.d_out), dtype=torch.bfloat16, device=dev)]
                     xp = am.PointerArrays(xs, ys)
@@ -361,7 +355,8 @@ def run_sweep(args):
                                         "frac_of_peak": round(ab / (a_dev * 1e-3) / 1e9 / peak, 3),
                                         "tokens_per_s": round(T / (a_dev * 1e-3), 1),
                                         "back_to_back_us": round(a_b2b * 1e3, 2),
-                                        "host_us_per_call": round(a_host, 2), "launches": 4, "bytes": ab})
+                                        "host_us_per_call": round(a_host, 2),
+                                        "launches": copies[0][2].last_launches, "bytes": ab})
                 for (_, _, plan) in copies:
                     rc, st = plan.status()
                     if rc != 0 or st != 0:
@@ -370,6 +365,44 @@ def run_sweep(args):
                 points.append(pt)
                 del copies
                 torch.cuda.empty_cache()
+    return points
+
+
+def sweep_summary(points, seconds):
+    """Medians over the sweep grid: the merge per contraction depth k*r, the
+    apply per batch T (device time of one call and its fraction of the peak)."""
+    by_kr, by_T = {}, {}
+    for p in points:
+        by_kr.setdefault(p["k"] * p["r"], []).append(p["merge"])
+        for a in p["apply"]:
+            by_T.setdefault(a["T"], []).append(a)
+
+    def med(rows):
+        return {"us": round(statistics.median(x["us"] for x in rows), 2),
+                "frac_of_peak": round(statistics.median(x["frac_of_peak"] for x in rows), 3),
+                "frac_min": round(min(x["frac_of_peak"] for x in rows), 3),
+                "frac_max": round(max(x["frac_of_peak"] for x in rows), 3), "points": len(rows)}
+    return {"merge_by_kr": {str(kr): med(v) for kr, v in sorted(by_kr.items())},
+            "apply_by_T": {str(T): med(v) for T, v in sorted(by_T.items())},
+            "points": len(points), "seconds": round(seconds, 1),
+            "workload": "one 4096x4096 linear, E in {4,8,16,32}, r in {8,16,32,64}, k in {1,2,4}; "
+                        "apply at T in {1,16,128}",
+            "l2": "8 rotated copies of every operand (no L2 reuse between launches)"}
+
+
+def run_sweep(args):
+    """`--config sweep`: the whole grid (or one --point), one JSON line."""
+    import torch
+    from adapter_merge_b200 import build as ambuild
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    ambuild.build()
+    peak, peak_kind = read_peaks()
+    only = sweep_point_arg(args.point)
+    t_begin = time.perf_counter()
+    points = measure_sweep(dev, peak, only)
     if rank == 0:
         fr = [p["merge"]["frac_of_peak"] for p in points]
         line = {
@@ -380,14 +413,93 @@ def run_sweep(args):
             "config": {"workload": (f"sweep point 4096x4096, E={only[0]}, r={only[1]}, k={only[2]}, T in {{1,16,128}}"
                                     if only else "sweep 4096x4096, E in {4,8,16,32}, r in {8,16,32,64}, "
                                                  "k in {1,2,4}, T in {1,16,128}"),
-                       "l2": f"{NC} rotated copies of every operand (no L2 reuse between launches)"},
+                       "l2": "8 rotated copies of every operand (no L2 reuse between launches)"},
             "peak": peak, "peak_source": f"{peak_kind} hbm_gbs",
             "merge_frac_of_peak": {"min": min(fr), "median": statistics.median(fr), "max": max(fr)},
+            "summary": sweep_summary(points, time.perf_counter() - t_begin),
             "seconds": round(time.perf_counter() - t_begin, 1),
             "points": points,
         }
         print(json.dumps(line), flush=True)
     return 0
+
+
+def measure_13b(dev, peak, steps=10):
+    """The Llama-2-13B-shaped stack (280 linears, E=16, r=32, top-2): the
+    full-model merge for one request and the batch-32 segmented apply, each
+    preceded by its pregate, device time by CUDA events (mean of `steps`
+    after three warm-ups), weights resident."""
+    import torch
+    import adapter_merge_b200 as am
+    import synth
+    cfg = synth.llama13b()
+    stream = torch.cuda.current_stream()
+    w = synth.make_weights(cfg, 1300, device=dev)
+    W_out = torch.empty_like(w.W)
+    views, o = [], 0
+    for l in cfg.linears:
+        n = l.d_out * l.d_in
+        views.append(W_out[o:o + n].view(l.d_out, l.d_in))
+        o += n
+    plan = am.Plan(list(zip(w.W_views, views, w.A_views, w.B_views)), cfg.E, cfg.r)
+    T = cfg.T_apply
+    x_req = synth.make_router_input(cfg, 1, 1300, device=dev, tag="xreq")
+    x_first = synth.make_router_input(cfg, T, 1300, device=dev, tag="xfirst")
+    X, xs = synth.make_apply_inputs(cfg, T, 1300, device=dev)
+    ys = [torch.empty((T, l.d_out), dtype=torch.bfloat16, device=dev) for l in cfg.linears]
+    xp = am.PointerArrays(xs, ys)
+    ws = torch.empty(plan.workspace_bytes(T, cfg.k), dtype=torch.uint8, device=dev)
+
+    def ev_mean(fn):
+        for _ in range(3):
+            fn(None)
+        torch.cuda.synchronize()
+        e = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
+        for i in range(steps):
+            fn(e[i])
+        torch.cuda.synchronize()
+        return sum(a.elapsed_time(b) for a, b in e) / steps
+
+    def merge(ev):
+        i1, g1 = am.pregate(x_req, w.W_r, cfg.k)
+        if ev is not None:
+            ev[0].record(stream)
+        plan.merge(i1[0], g1[0])
+        if ev is not None:
+            ev[1].record(stream)
+
+    state = {}
+
+    def apply(ev):
+        iT, gT = am.pregate(x_first, w.W_r, cfg.k)
+        if ev is not None:
+            ev[0].record(stream)
+        plan.apply(xp, None, T, iT, gT, ws)
+        if ev is not None:
+            ev[1].record(stream)
+        state["idx"] = iT
+
+    m_ms = ev_mean(merge)
+    a_ms = ev_mean(apply)
+    rc, st = plan.status()
+    if rc != 0 or st != 0:
+        raise RuntimeError(f"device status {st} in the 13B measurement")
+    U = int(torch.unique(state["idx"]).numel())
+    mb, ab = merge_bytes(cfg, cfg.k), apply_bytes(cfg, T, U)
+    plan.destroy()
+    out = {"workload": f"{cfg.name}: {cfg.n_lin} linears, E={cfg.E}, r={cfg.r}, top-{cfg.k}; merge for one "
+                       f"request, apply for T={T} sequences",
+           "merge": {"ms": round(m_ms, 4), "gbs": round(mb / (m_ms * 1e-3) / 1e9, 1),
+                     "frac_of_peak": round(mb / (m_ms * 1e-3) / 1e9 / peak, 4), "bytes": mb,
+                     "note": "merge kernel alone (the router launch before it is outside the events)"},
+           "apply": {"T": T, "ms": round(a_ms, 4), "tokens_per_s": round(T / (a_ms * 1e-3), 1),
+                     "gbs": round(ab / (a_ms * 1e-3) / 1e9, 1),
+                     "frac_of_peak": round(ab / (a_ms * 1e-3) / 1e9 / peak, 4), "bytes": ab,
+                     "distinct_experts": U, "note": "one apply call (all its launches)"},
+           "steps": steps}
+    del w, W_out, X, ys, ws
+    torch.cuda.empty_cache()
+    return out
 
 
 def main():
@@ -405,7 +517,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-extras", action="store_true",
-                    help="skip the switch / per-linear merge / pooled-router measurements")
+                    help="skip the switch / per-linear merge / pooled-router / 13B / sweep measurements")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -523,10 +635,11 @@ def main():
         [total_ms, mean(merge_part), mean(merge_kernel), mean(apply_part), mean(apply_call)], dist, dev)
 
     mb = merge_bytes(cfg, cfg.k)
+    rec_merge = profile_record("merge_rows_kernel")
+    rec_apply = profile_record("apply_fused_kernel")
     traffic = None
-    if cfg.name == "llama2-7b":
-        traffic = profiled_traffic(["merge.cu", "ptx.cuh", "internal.h"], "merge_rows_kernel_llama2-7b-2layer.md",
-                                   "traffic_bytes_per_full_llama2_7b_launch")
+    if rec_merge and cfg.name == rec_merge.get("full_workload"):
+        traffic = rec_merge.get("dram_bytes_per_full_launch")
     ab = apply_bytes(cfg, T, U)
     peak, peak_kind = read_peaks()
     merge_gbs = job_throughput(world, mb, m_part)
@@ -678,6 +791,17 @@ def main():
             "pregate_pooled": {"ms": round(pool_ms, 4), "tokens": T,
                                "note": "one decision from the mean of the T router inputs"},
         }
+        if world == 1 and cfg.name == "llama2-7b":
+            # The other two model-scale workloads, measured on the same GPU
+            # after the 7B model is freed: the 13B stack and the single-layer
+            # sweep (per-GPU numbers; replicas would repeat them).
+            del w, W_out, W_out_views, X, xs, Y, ys, xp, ws
+            plan.destroy()
+            plan = None
+            torch.cuda.empty_cache()
+            extras["llama2_13b"] = measure_13b(dev, peak)
+            t_sw = time.perf_counter()
+            extras["sweep"] = sweep_summary(measure_sweep(dev, peak, R=3), time.perf_counter() - t_sw)
 
     cpu = None
     if rank == 0 and not args.no_cpu_baseline:
@@ -705,22 +829,29 @@ def main():
             "apply": {"tokens_per_s": round(apply_tps, 1), "ms": round(a_part, 4), "call_ms": round(a_call, 4),
                       "gbs": round(apply_gbs, 2), "bytes": ab, "distinct_experts": U,
                       "frac_of_peak": round(apply_gbs / peak, 4),
-                      "note": "call = segments + shrink + finalize + fused apply (4 launches)"},
+                      "note": "call = segment build + fused shrink/apply kernel (2 launches)"},
             "roofline": {"bound": "hbm", "kernel": "merge_rows_kernel", "achieved": round(kern_gbs, 2),
                          "peak": peak, "unit": "GB/s", "frac": round(kern_gbs / peak, 4),
                          "peak_source": f"{peak_kind} hbm_gbs (burst copy)",
                          "algorithmic_bytes": mb,
                          "traffic": traffic,
-                         "traffic_source": ("ncu dram bytes, 2-layer capture scaled by elements "
-                                            "(profiles/merge_rows_kernel_llama2-7b-2layer.md)") if traffic else None},
-            "gpu_launches": 7 * args.steps,
+                         "traffic_source": ("ncu dram__bytes_read.sum + dram__bytes_write.sum of a 2-layer "
+                                            "capture of this kernel build, scaled to the full model by "
+                                            "elements") if traffic else None},
+            "tensor_pipe_pct": {
+                "merge_rows_kernel": rec_merge.get("tensor_pipe_pct") if rec_merge else None,
+                "apply_fused_kernel": rec_apply.get("tensor_pipe_pct") if rec_apply else None,
+                "source": "ncu sm__pipe_tensor_cycles_active (% of peak) of a small capture of this kernel "
+                          "build (2-layer merge, 4-layer apply); null when the sources changed since"},
+            "gpu_launches": 5 * args.steps,
             "clocks": clocks,
             "e2e": e2e,
             "cpu_baseline": cpu,
             "extras": extras,
         }
         print(json.dumps(line), flush=True)
-    plan.destroy()
+    if plan is not None:
+        plan.destroy()
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()

@@ -80,3 +80,37 @@ def test_clock_sampler_without_nvidia_smi(tmp_path, monkeypatch):
     s = bench.ClockSampler(0)
     s.start()
     assert s.stop() is None
+
+
+def test_profile_record_needs_the_recorded_fingerprint(tmp_path, monkeypatch):
+    """A profile record is reported only while the kernel's sources hash to
+    the fingerprint recorded with it."""
+    import json
+    import bench
+    fp = bench.kernel_fingerprint(["merge.cu", "ptx.cuh"])
+    recs = {"merge_rows_kernel": {"sources": ["merge.cu", "ptx.cuh"], "kernel_sources_sha256_16": fp,
+                                  "tensor_pipe_pct": 4.0},
+            "apply_fused_kernel": {"sources": ["apply.cu"], "kernel_sources_sha256_16": "0" * 16,
+                                   "tensor_pipe_pct": 18.0}}
+    path = tmp_path / "records.json"
+    path.write_text(json.dumps(recs))
+    monkeypatch.setattr(bench, "RECORDS", str(path))
+    assert bench.profile_record("merge_rows_kernel")["tensor_pipe_pct"] == 4.0
+    assert bench.profile_record("apply_fused_kernel") is None
+    assert bench.profile_record("no_such_kernel") is None
+    monkeypatch.setattr(bench, "RECORDS", str(tmp_path / "absent.json"))
+    assert bench.profile_record("merge_rows_kernel") is None
+
+
+def test_sweep_summary_groups_by_depth_and_batch():
+    import bench
+    pts = []
+    for (E, r, k, us) in ((8, 16, 1, 20.0), (4, 8, 2, 22.0), (8, 16, 2, 30.0)):
+        pts.append({"E": E, "r": r, "k": k, "merge": {"us": us, "frac_of_peak": 10.0 / us},
+                    "apply": [{"T": T, "us": us + T, "frac_of_peak": 5.0 / (us + T)} for T in (1, 16)]})
+    s = bench.sweep_summary(pts, 12.3)
+    assert set(s["merge_by_kr"]) == {"16", "32"}
+    assert s["merge_by_kr"]["16"]["points"] == 2 and s["merge_by_kr"]["16"]["us"] == 21.0
+    assert s["merge_by_kr"]["32"]["us"] == 30.0
+    assert s["apply_by_T"]["16"]["points"] == 3 and s["apply_by_T"]["1"]["us"] == 23.0
+    assert s["points"] == 3 and s["seconds"] == 12.3
