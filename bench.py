@@ -5,7 +5,8 @@ One step = one pass of the whole path on the Llama-2-7B-shaped workload:
   request start : pregate (router on the request's token) -> fused merge of
                   all 224 linears (W' = W + sum_s g_s B_s A_s, one launch);
   batched decode: pregate (first token of each of 64 sequences) -> segment
-                  build -> shrink -> fused segmented apply over all 224 linears.
+                  build -> one kernel: shrink, then the fused segmented apply
+                  over all 224 linears.
 `value` is the merge throughput in GB/s of algorithmic bytes (W read + W'
 write + the selected adapters); the apply throughput (tokens/s and GB/s) is
 reported beside it.  Inputs are seeded synthetic tensors resident in HBM,

@@ -76,7 +76,7 @@ uint16_t orc_bf16_from_double(double v)
     } else {
         f = (float)rv;                     /* exact: rv has <= 8 significant bits */
     }
-    if (v < 0) f = -f;
+    if (signbit(v)) f = -f;              /* the sign of a zero result is the operand's */
     uint32_t u;
     memcpy(&u, &f, 4);
     return (uint16_t)(u >> 16);

@@ -48,6 +48,7 @@ MUTANTS = {
     "apply_shrink_reads_token_0": (r"\* d_in \+ i\]\) \*\n                               orc_bf16_to_double\(x\[t \* d_in \+ i\]\);",
                                    "* d_in + i]) *\n                               orc_bf16_to_double(x[i]);"),
     "segments_count_shifted": (r"offsets\[e \+ 1\] \+= 1;", "offsets[e] += 1;"),
+    "bf16_negative_zero_to_positive": (r"if \(signbit\(v\)\) f = -f;", "if (v < 0) f = -f;"),
     "apply_f64_partial_rounded": (r"if \(y64\) y64\[\(t - t0\) \* d_out \+ o\] = acc;",
                                   "if (y64) y64[(t - t0) * d_out + o] = orc_bf16_to_double(orc_bf16_from_double(acc));"),
 }

@@ -71,7 +71,10 @@ def test_bf16_rounding_matches_torch_on_fp32_values():
     f = f[np.isfinite(f)]
     mids = ((np.arange(1 << 16, dtype=np.uint32) << 16) | 0x8000).view(np.float32)
     mids = mids[np.isfinite(mids)]
-    for v in (f, mids):
+    # signed zeros, and values of either sign that round to a zero
+    zeros = np.array([0.0, -0.0, 2.0 ** -134, -(2.0 ** -134), -(2.0 ** -140), 2.0 ** -149, -(2.0 ** -149)],
+                     dtype=np.float32)
+    for v in (f, mids, zeros):
         ours = oracle.bf16_from_f64(v.astype(np.float64))
         ref = torch.from_numpy(v.copy()).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
         assert np.array_equal(ours, ref)
@@ -105,6 +108,8 @@ def test_bf16_rounding_single_step_from_double():
     # signs, zero, overflow and subnormals
     assert int(oracle.bf16_from_f64(np.array([-1.0]))[0]) == 0xBF80
     assert int(oracle.bf16_from_f64(np.array([0.0]))[0]) == 0x0000
+    assert int(oracle.bf16_from_f64(np.array([-0.0]))[0]) == 0x8000
+    assert int(oracle.bf16_from_f64(np.array([-(2.0 ** -140)]))[0]) == 0x8000
     assert int(oracle.bf16_from_f64(np.array([1e39]))[0]) == 0x7F80
     assert int(oracle.bf16_from_f64(np.array([2.0 ** -133]))[0]) == 0x0001
     assert int(oracle.bf16_from_f64(np.array([2.0 ** -134]))[0]) == 0x0000   # tie -> even (0)
