@@ -57,9 +57,12 @@ struct WsLayout {
     int32_t shape, tile;    // apply units of 128 << shape rows; tokens per tile
     int32_t ksg, total_ks;  // shrink K-slice width shrink_ks(ksg); slices over all linears
     int32_t nsplit;         // K-splits per apply unit
+    bool fused;             // shrink units inside the apply kernel (small plans, T <= 32)
     int64_t n_grp;          // apply units (before splitting) over all token tiles
     int64_t n_su;           // shrink units per token tile: Mt x total K-slices
 };
+
+constexpr int kMaxSplit = 16;                     // K-splits per apply unit, at most
 
 // Unit height for a batch of T tokens.  A taller unit issues more MMAs per x
 // chunk it stages; its token tile (256 >> shape) must still cover T, or W is
@@ -91,13 +94,19 @@ WsLayout ws_layout(const Plan* p, int64_t T, int32_t k)
     w.nsplit = 1;
     if (w.n_grp < p->num_sms) {
         double best = 1e30;
-        for (int sp = 1; sp <= std::min(16, std::max(1, max_kb / 4)); ++sp) {
+        for (int sp = 1; sp <= std::min(kMaxSplit, std::max(1, max_kb / 4)); ++sp) {
             const int64_t waves = (w.n_grp * sp + p->num_sms - 1) / p->num_sms;
             const double cost = (double)waves * (1.0 / sp + 0.15);
             if (cost < best - 1e-9) { best = cost; w.nsplit = sp; }
         }
     }
-    // Narrow shrink slices only when the wide ones leave SMs without a unit.
+    // With fewer apply units than SMs and a few tokens, the shrink runs as
+    // work units of the apply kernel, on the SMs the apply units leave free
+    // and off the critical path; otherwise as a kernel of its own followed by
+    // the finalize kernel (whose CTA per (linear, token) is the faster
+    // finalize once a tile holds more than a few tokens).  Narrow shrink
+    // slices only when the wide ones leave SMs without a unit.
+    w.fused = w.n_grp < p->num_sms && T <= 8;
     w.ksg = (int64_t)w.Mt * p->total_ks[0] * token_tiles(T, w.shape) < p->num_sms ? 1 : 0;
     w.total_ks = p->total_ks[w.ksg];
     w.n_su = (int64_t)w.Mt * w.total_ks;
@@ -134,6 +143,10 @@ __device__ __forceinline__ bool mbar_wait_drain2(uint64_t* bar, uint32_t parity)
 }
 
 constexpr uint32_t kAChunkBytes = kTileM * kChunkK * 2;     // 16 KB: 128 rows x 64 cols bf16
+// Pipeline stages of the shrink and apply kernels: as many as shared memory
+// holds, up to 16 (small stages, e.g. one 16 KB W chunk and a few tokens of
+// x, need many in flight per SM to cover the loaded memory latency).
+constexpr int kMaxStages = 16;
 
 // A shrink unit: Acat tile mq (rows mq*128 ..) against K-slice ks of linear
 // l, columns [k0, k0 + nK * 64) of d_in.
@@ -156,6 +169,265 @@ struct ShrinkUnit {
         nK = (k1 - k0 + kChunkK - 1) / kChunkK;
     }
 };
+
+// ------------------------------------------------------------------ shrink
+//
+// S^T = Acat x^T for every linear, on the tensor cores: Acat stacks the A rows
+// of the U used experts (U*r rows, gathered by TMA: boxes of 2-16 whole experts
+// for runs of consecutive expert ids where r is a power of two, else boxes of
+// up to 128 rows of one expert), x^T is the token tile.  Work units are
+// (128-row tile of Acat, K-slice of a linear); each unit writes its fp32
+// partial [Npad x 128] to the workspace.  Plans with at least one apply unit
+// per SM run the shrink as this kernel of its own, followed by the finalize
+// kernel (slices added in order, gates applied, rounded); smaller plans run
+// the same units inside the apply kernel (below), finalized by the warp that
+// completes a slice last.
+
+struct ShrinkArgs {
+    const LinDesc* lins;
+    const CUtensorMap* maps;
+    const CUtensorMap* xmaps;
+    const int32_t* used;
+    float* P;
+    int32_t* status;
+    int64_t n_su;
+    int32_t n_lin, r, Npad, n_tt, total_ks, tile, ksg;
+    int32_t ST, box_rows, run_max;
+    uint32_t stage_bytes, off_bar, acc_stride, tmem_cols;
+};
+
+constexpr int kShrinkThreads = 192;
+
+__global__ void __launch_bounds__(kShrinkThreads, 1) shrink_tc_kernel(const __grid_constant__ ShrinkArgs a)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(base + a.off_bar);
+    uint64_t* empty = full + a.ST;
+    uint64_t* accfull = empty + a.ST;
+    uint64_t* accempty = accfull + 2;
+    uint64_t* donebar = accempty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(donebar + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    int* s_used = reinterpret_cast<int*>(tmem_slot + 4);     // [1 + kMaxE]
+    int* s_loads = s_used + 1 + kMaxE;                        // [kTileM / 8]: A loads of the current unit
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < a.ST; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
+        for (int i = 0; i < 2; ++i) { mbar_init(&accfull[i], 1); mbar_init(&accempty[i], 4); }
+        mbar_init(donebar, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    for (int s = 0; s < a.ST; ++s)
+        for (uint32_t o = threadIdx.x * 16; o < kAChunkBytes; o += kShrinkThreads * 16)
+            st_shared_v4(smem_u32(base + (size_t)s * a.stage_bytes + o), make_uint4(0, 0, 0, 0));
+    fence_proxy_async_smem();
+    griddep_wait();
+    griddep_launch_dependents();
+    if (threadIdx.x <= kMaxE) s_used[threadIdx.x] = a.used[threadIdx.x];
+    __syncthreads();
+    const int rows = s_used[0] * a.r;          // live rows of Acat
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, a.tmem_cols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    const int64_t total = a.n_su * a.n_tt;
+    const int64_t u_begin = (int64_t)blockIdx.x * total / gridDim.x;
+    const int64_t u_end = ((int64_t)blockIdx.x + 1) * total / gridDim.x;
+    const uint32_t xbytes = (uint32_t)a.Npad * 128u;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int64_t gc = 0, issued = 0;
+            bool stop = false;
+            for (int64_t ua = u_begin; ua < u_end && !stop; ++ua) {
+                const int tt = (int)(ua / a.n_su);
+                ShrinkUnit su;
+                su.at(a.lins, a.n_lin, a.total_ks, a.ksg, ua - (int64_t)tt * a.n_su);
+                if (su.mq * kTileM >= rows) continue;
+                const CUtensorMap* mA = a.maps + (size_t)su.l * kMapsPerLinear + kMapA;
+                const CUtensorMap* mX = a.xmaps + su.l;
+                const int R = a.box_rows;               // A rows per box (divides r and 128)
+                int ng = 0;
+                for (int g = 0; g < kTileM / R; ++g) if (su.mq * kTileM + g * R < rows) ++ng;
+                // One box per expert (R == r): a run of consecutive expert ids
+                // is loaded in pieces of 2^i whole experts.  Entry: expert |
+                // map << 8 | tile position << 16.
+                int nload = 0;
+                if (a.run_max > 1) {
+                    const int q0 = su.mq * (kTileM / R), q1 = q0 + ng;
+                    for (int q = q0; q < q1;) {
+                        int e = s_used[1 + q], L = 1;
+                        while (q + L < q1 && s_used[1 + q + L] == e + L) ++L;
+                        while (L > 0) {
+                            int D = 1, mi = -1;
+                            while (2 * D <= L && 2 * D <= a.run_max) { D *= 2; ++mi; }
+                            s_loads[nload++] = e | ((mi < 0 ? kMapA : kMapARun + mi) << 8) | ((q - q0) << 16);
+                            q += D; e += D; L -= D;
+                        }
+                    }
+                }
+                for (int kc = 0; kc < su.nK; ++kc, ++gc) {
+                    const int s = (int)(gc % a.ST);
+                    if (!mbar_wait(&empty[s], (uint32_t)((gc / a.ST) & 1) ^ 1u, abort_flag)) { stop = true; break; }
+                    uint8_t* dst = base + (size_t)s * a.stage_bytes;
+                    const int col = su.k0 + kc * kChunkK;
+                    mbar_arrive_expect_tx(&full[s], (uint32_t)(ng * R) * 128u + xbytes);
+                    if (a.run_max > 1) {
+                        for (int i = 0; i < nload; ++i) {
+                            const int v = s_loads[i];
+                            tma_load_3d(dst + (size_t)(v >> 16) * R * 128u,
+                                        a.maps + (size_t)su.l * kMapsPerLinear + ((v >> 8) & 0xff), &full[s], col, 0,
+                                        v & 0xff);
+                        }
+                    } else {
+                        for (int g = 0; g < ng; ++g) {
+                            const int c = su.mq * kTileM + g * R;
+                            const int qq = c / a.r, j0 = c - qq * a.r;
+                            tma_load_3d(dst + (size_t)g * R * 128u, mA, &full[s], col, j0, s_used[1 + qq]);
+                        }
+                    }
+                    tma_load_2d(dst + kAChunkBytes, mX, &full[s], col, tt * a.tile);
+                    issued = gc + 1;
+                }
+            }
+            for (int64_t g = std::max<int64_t>(0, issued - a.ST); g < issued; ++g)
+                mbar_wait_drain2(&full[g % a.ST], (uint32_t)((g / a.ST) & 1));
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t idesc = make_idesc_bf16(kTileM, (uint32_t)a.Npad, 0u, 0u);
+            int64_t gc = 0, uc = 0;
+            bool stop = false;
+            for (int64_t ua = u_begin; ua < u_end && !stop; ++ua) {
+                const int tt = (int)(ua / a.n_su);
+                ShrinkUnit su;
+                su.at(a.lins, a.n_lin, a.total_ks, a.ksg, ua - (int64_t)tt * a.n_su);
+                if (su.mq * kTileM >= rows) continue;
+                const int acc = (int)(uc & 1);
+                if (!mbar_wait(&accempty[acc], (uint32_t)((uc >> 1) & 1) ^ 1u, abort_flag)) break;
+                tc_fence_after();
+                const uint32_t d = tmem_base + (uint32_t)acc * a.acc_stride;
+                for (int kc = 0; kc < su.nK; ++kc, ++gc) {
+                    const int s = (int)(gc % a.ST);
+                    if (!mbar_wait(&full[s], (uint32_t)((gc / a.ST) & 1), abort_flag)) { stop = true; break; }
+                    tc_fence_after();
+                    const uint32_t aaddr = smem_u32(base + (size_t)s * a.stage_bytes);
+#pragma unroll
+                    for (int kk = 0; kk < kChunkK / 16; ++kk)
+                        tc_mma_bf16(d, make_sdesc(aaddr + (uint32_t)kk * 32u, 16u, 1024u, kLayoutSw128),
+                                    make_sdesc(aaddr + kAChunkBytes + (uint32_t)kk * 32u, 16u, 1024u, kLayoutSw128),
+                                    idesc, (kc | kk) ? 1u : 0u);
+                    tc_commit(&empty[s]);
+                }
+                if (stop) break;
+                tc_commit(&accfull[acc]);
+                ++uc;
+            }
+            tc_commit(donebar);
+            mbar_wait_drain2(donebar, 0);
+        }
+        __syncwarp();
+    } else {
+        const int q = warp & 3;
+        int64_t uc = 0;
+        for (int64_t ua = u_begin; ua < u_end; ++ua) {
+            const int tt = (int)(ua / a.n_su);
+            const int64_t u = ua - (int64_t)tt * a.n_su;
+            ShrinkUnit su;
+            su.at(a.lins, a.n_lin, a.total_ks, a.ksg, u);
+            if (su.mq * kTileM >= rows) continue;
+            const int acc = (int)(uc & 1);
+            bool ok = mbar_wait(&accfull[acc], (uint32_t)((uc >> 1) & 1), abort_flag);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            tc_fence_after();
+            float* Pu = a.P + ((int64_t)tt * a.n_su + u) * a.Npad * kTileM + q * 32 + lane;
+            const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)acc * a.acc_stride;
+            for (int c0 = 0; c0 < a.Npad; c0 += 32) {
+                uint32_t v[32];
+                if (a.Npad - c0 >= 32) {
+                    tc_ld_x32(tbase + (uint32_t)c0, v);
+                } else {
+                    uint32_t h[16];
+                    tc_ld_x16(tbase + (uint32_t)c0, h);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) { v[i] = h[i]; v[16 + i] = 0; }
+                }
+                tc_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    if (c0 + i < a.Npad) Pu[(int64_t)(c0 + i) * kTileM] = __uint_as_float(v[i]);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&accempty[acc]);
+            ++uc;
+        }
+    }
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, a.tmem_cols);
+    }
+    if (threadIdx.x == 0 && *abort_flag) atomicOr(a.status, ADAFUSE_STATUS_TIMEOUT);
+}
+
+// s = coef(t, c) * (sum over the K-slices of linear l of the partials), for
+// c < U*r (zero for the padding columns up to Kext); coef(t, c) is the sum of
+// token t's gates on expert used[1 + c/r] (zero if t did not pick it).  s is
+// stored as two bf16 values, hi = bf16(s) and lo = bf16(s - hi), whose sum
+// carries s to about 2^-17 relative: the expand multiplies both halves by the
+// same B rows, so the LoRA term keeps close to fp32 precision even where it
+// cancels most of the base product.  Row layout of S_l[t]: for each group of
+// 32 columns, its 32 hi values then its 32 lo values, so that one 64-column
+// box of S feeds both halves of an expand chunk.
+__global__ void __launch_bounds__(128) shrink_finalize_kernel(const LinDesc* lins, const float* P, const int32_t* used,
+                                                               const int32_t* idx, const float* gate, uint16_t* S,
+                                                               int64_t T, int32_t k, int32_t r, int32_t Kext,
+                                                               int32_t Npad, int32_t tile, int64_t n_su,
+                                                               int32_t total_ks, int32_t ksg)
+{
+    griddep_wait();
+    griddep_launch_dependents();
+    __shared__ int s_used[kMaxE + 1];
+    __shared__ int s_idx[kMaxSlots];
+    __shared__ float s_gate[kMaxSlots];
+    const int l = blockIdx.x;
+    const int64_t t = blockIdx.y;
+    if (threadIdx.x <= kMaxE) s_used[threadIdx.x] = used[threadIdx.x];
+    if (threadIdx.x < k) { s_idx[threadIdx.x] = idx[t * k + threadIdx.x]; s_gate[threadIdx.x] = gate[t * k + threadIdx.x]; }
+    __syncthreads();
+    const int rows = s_used[0] * r;
+    const int ks_base = __ldg(&lins[l].ks_base[ksg]), n_ks = __ldg(&lins[l].n_ks[ksg]);
+    const int tt = (int)(t / tile), tl = (int)(t - (int64_t)tt * tile);
+    uint16_t* Srow = S + ((int64_t)l * T + t) * (2 * Kext);
+    for (int c = threadIdx.x; c < Kext; c += blockDim.x) {
+        float v = 0.f;
+        if (c < rows) {
+            const int e = s_used[1 + c / r];
+            float coef = 0.f;
+            for (int s = 0; s < k; ++s) if (s_idx[s] == e) coef += s_gate[s];
+            if (coef != 0.f) {
+                const int mq = c / kTileM, cl = c - mq * kTileM;
+                const float* p = P + (((int64_t)tt * n_su + (int64_t)mq * total_ks + ks_base) * Npad + tl) * kTileM + cl;
+                float sum = 0.f;
+                for (int ks = 0; ks < n_ks; ++ks) sum += p[(int64_t)ks * Npad * kTileM];
+                v = coef * sum;
+            }
+        }
+        const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+        const int o = 64 * (c >> 5) + (c & 31);              // [hi 32 | lo 32] per 32-column group
+        Srow[o] = __bfloat16_as_ushort(hi);
+        Srow[o + 32] = __bfloat16_as_ushort(__float2bfloat16_rn(v - __bfloat162float(hi)));
+    }
+}
 
 // ------------------------------------------------------------------ apply
 
@@ -183,6 +455,7 @@ struct ApplyArgs {
     int32_t bcols;                  // columns per B-row box of the expand: 8, 16 or 32
     int32_t stall;                  // test hook: CTA 0 withholds its first stage
     int32_t y_f32;                  // outputs are the fp32 accumulators (ADAFUSE_PLAN_Y_F32), not bf16
+    int32_t s_done;                 // S was finished by earlier launches: expand chunks need no wait
     float* Yp;                      // split partials [groups][nsplit][Npad][128 H] fp32
     int32_t* cnt;                   // [groups] splits finished (cleared by the segment build)
     int32_t ST;
@@ -263,6 +536,7 @@ __device__ __forceinline__ void release_counters(int32_t* sched)
 __device__ __forceinline__ void finalize_slice(const ApplyArgs& a, const int* s_used, int l, int tt, int mq, int q,
                                                int lane)
 {
+    constexpr int kTok = 4;                                  // tokens per step: independent loads in flight
     const int rows = s_used[0] * a.r;
     const int c = mq * kTileM + q * 32 + lane;
     if (c >= a.Kext) return;
@@ -271,25 +545,38 @@ __device__ __forceinline__ void finalize_slice(const ApplyArgs& a, const int* s_
     const float* p = a.P + (((int64_t)tt * a.n_su + (int64_t)mq * a.total_ks + ks_base) * a.Npad) * kTileM +
                      q * 32 + lane;
     const int64_t slice = (int64_t)a.Npad * kTileM;
-    for (int tl = 0; tl < a.Npad; ++tl) {
-        const int64_t t = (int64_t)tt * a.tile + tl;
-        if (t >= a.T) break;
-        float v = 0.f;
-        if (e >= 0) {
-            float coef = 0.f;
-            for (int s = 0; s < a.k; ++s)
-                if (__ldg(&a.idx[t * a.k + s]) == e) coef += __ldg(&a.gate[t * a.k + s]);
-            if (coef != 0.f) {
-                float sum = 0.f;
-                for (int ks = 0; ks < n_ks; ++ks) sum += __ldcg(p + (int64_t)ks * slice + (int64_t)tl * kTileM);
-                v = coef * sum;
-            }
+    const int64_t t_left = a.T - (int64_t)tt * a.tile;
+    const int n_tok = t_left < a.Npad ? (int)t_left : a.Npad;
+    for (int tl0 = 0; tl0 < n_tok; tl0 += kTok) {
+        float coef[kTok], sum[kTok];
+#pragma unroll
+        for (int j = 0; j < kTok; ++j) {
+            coef[j] = 0.f;
+            sum[j] = 0.f;
+            const int64_t t = (int64_t)tt * a.tile + tl0 + j;
+            if (e >= 0 && tl0 + j < n_tok)
+                for (int s = 0; s < a.k; ++s)
+                    if (__ldg(&a.idx[t * a.k + s]) == e) coef[j] += __ldg(&a.gate[t * a.k + s]);
         }
-        const __nv_bfloat16 hi = __float2bfloat16_rn(v);
-        uint16_t* Srow = a.S + ((int64_t)l * a.T + t) * (2 * a.Kext);
-        const int o = 64 * (c >> 5) + (c & 31);              // [hi 32 | lo 32] per 32-column group
-        Srow[o] = __bfloat16_as_ushort(hi);
-        Srow[o + 32] = __bfloat16_as_ushort(__float2bfloat16_rn(v - __bfloat162float(hi)));
+        for (int ks = 0; ks < n_ks; ++ks) {
+            float v[kTok];
+#pragma unroll
+            for (int j = 0; j < kTok; ++j)
+                v[j] = (coef[j] != 0.f) ? __ldcg(p + (int64_t)ks * slice + (int64_t)(tl0 + j) * kTileM) : 0.f;
+#pragma unroll
+            for (int j = 0; j < kTok; ++j) sum[j] += v[j];
+        }
+#pragma unroll
+        for (int j = 0; j < kTok; ++j) {
+            if (tl0 + j >= n_tok) break;
+            const int64_t t = (int64_t)tt * a.tile + tl0 + j;
+            const float v = coef[j] * sum[j];
+            const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+            uint16_t* Srow = a.S + ((int64_t)l * a.T + t) * (2 * a.Kext);
+            const int o = 64 * (c >> 5) + (c & 31);          // [hi 32 | lo 32] per 32-column group
+            Srow[o] = __bfloat16_as_ushort(hi);
+            Srow[o + 32] = __bfloat16_as_ushort(__float2bfloat16_rn(v - __bfloat162float(hi)));
+        }
     }
 }
 
@@ -449,7 +736,7 @@ __global__ void __launch_bounds__(ApplyShape<H>::kThreads, 1) apply_fused_kernel
                 bool s_ready = false;
                 for (int kc = c0; kc < c1; ++kc, ++gc) {
                     const int s = (int)(gc % a.ST);
-                    if (kc >= nKb && !s_ready) {
+                    if (kc >= nKb && !s_ready && !a.s_done) {
                         // S of this linear and token tile: every 32-row slice
                         // finalized (released by the finalizing warps)
                         const int* rp = a.ready + (int64_t)tt * a.n_lin + l;
@@ -687,7 +974,8 @@ __global__ void __launch_bounds__(ApplyShape<H>::kThreads, 1) apply_fused_kernel
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&accempty[acc]);
-            if (a.nsplit > 1) {
+            // Units split along K only at H = 1 (fewer units than SMs).
+            if (H == 1 && a.nsplit > 1) {
                 __threadfence();
                 __syncwarp();
                 int last = 0;
@@ -697,27 +985,34 @@ __global__ void __launch_bounds__(ApplyShape<H>::kThreads, 1) apply_fused_kernel
                 if (last) {
                     __threadfence();
                     const float* p0 = a.Yp + ((int64_t)g * a.nsplit * a.Npad) * kApplyRows + rin;
-                    for (int c0 = 0; c0 < a.Npad; c0 += 32) {
-                        // 32 independent loads per split in flight; each sum
-                        // still runs over the splits in order
-                        float v[32];
+                    // Four tokens at a time, every split's partial loaded
+                    // before any is added (one round of L2 latency instead of
+                    // one per split); each sum still runs over the splits in
+                    // order, so the result does not depend on which split
+                    // finished last.
+                    constexpr int kTk = 4;
+                    const int n_tok = T - tb < a.Npad ? (int)(T - tb) : a.Npad;
+                    for (int c0 = 0; c0 < n_tok; c0 += kTk) {
+                        float t[kMaxSplit][kTk];
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) v[i] = 0.f;
-                        for (int s2 = 0; s2 < a.nsplit; ++s2) {
-                            const float* ps = p0 + ((int64_t)s2 * a.Npad + c0) * kApplyRows;
-                            float t[32];
+                        for (int s2 = 0; s2 < kMaxSplit; ++s2)
 #pragma unroll
-                            for (int i = 0; i < 32; ++i)
-                                t[i] = (c0 + i < a.Npad) ? __ldcg(ps + (int64_t)i * kApplyRows) : 0.f;
+                            for (int i = 0; i < kTk; ++i)
+                                t[s2][i] = (s2 < a.nsplit && c0 + i < n_tok)
+                                               ? __ldcg(p0 + ((int64_t)s2 * a.Npad + c0 + i) * kApplyRows) : 0.f;
+                        float v[kTk];
 #pragma unroll
-                            for (int i = 0; i < 32; ++i) v[i] += t[i];
+                        for (int i = 0; i < kTk; ++i) {
+                            v[i] = 0.f;
+#pragma unroll
+                            for (int s2 = 0; s2 < kMaxSplit; ++s2) v[i] += t[s2][i];
                         }
                         if (row < d_out) {
-                            uint32_t vb[32];
-#pragma unroll
-                            for (int i = 0; i < 32; ++i) vb[i] = __float_as_uint(v[i]);
-                            store_y_rows(y, a.y_f32, (tb + c0) * d_out + row, d_out, min(32, a.Npad - c0),
-                                         T - tb - c0, vb);
+                            for (int i = 0; i < kTk && c0 + i < n_tok; ++i) {
+                                const int64_t off = (tb + c0 + i) * d_out + row;
+                                if (a.y_f32) static_cast<float*>(y)[off] = v[i];
+                                else static_cast<uint16_t*>(y)[off] = __bfloat16_as_ushort(__float2bfloat16_rn(v[i]));
+                            }
                         }
                     }
                 }
@@ -782,16 +1077,60 @@ int launch_apply_kernels(Plan* p, const WsLayout& w, uint8_t* wsb, const CUtenso
                              reinterpret_cast<int32_t*>(wsb + w.off_cnt), w.n_zero);
     if (rc != ADAFUSE_OK) return rc;
 
+    if (!w.fused) {
+        // The shrink as a kernel of its own, then the finalize.
+        uint32_t accs = 32;
+        while (accs < (uint32_t)Npad) accs <<= 1;
+        const uint32_t stage_bytes = kAChunkBytes + (uint32_t)Npad * 128u;
+        const int ST = std::min(kMaxStages, (int)((kSmemMax - 2048u) / stage_bytes));
+        if (ST < 2 || 2 * accs > 512) return ADAFUSE_ERR_UNSUPPORTED;
+        const uint32_t smem = (uint32_t)ST * stage_bytes + 1024u + 1024u;
+        ShrinkArgs sa{};
+        sa.lins = p->d_desc;
+        sa.maps = p->d_maps;
+        sa.xmaps = xmaps;
+        sa.used = used;
+        sa.P = reinterpret_cast<float*>(wsb + w.off_P);
+        sa.status = p->d_status;
+        sa.n_su = w.n_su;
+        sa.n_lin = p->n_lin;
+        sa.r = p->r;
+        sa.Npad = Npad;
+        sa.n_tt = w.n_tt;
+        sa.total_ks = w.total_ks;
+        sa.ksg = w.ksg;
+        sa.tile = w.tile;
+        sa.ST = ST;
+        sa.box_rows = p->a_box_rows;
+        sa.run_max = p->a_run_max;
+        sa.stage_bytes = stage_bytes;
+        sa.off_bar = (uint32_t)ST * stage_bytes;
+        sa.acc_stride = accs;
+        sa.tmem_cols = 2 * accs;
+        if (cudaFuncSetAttribute(shrink_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+            cudaSuccess)
+            return ADAFUSE_ERR_CUDA;
+        rc = launch_pdl(shrink_tc_kernel, dim3((unsigned)std::min<int64_t>(p->num_sms, w.n_su * w.n_tt)),
+                        dim3(kShrinkThreads), smem, s, sa);
+        if (rc != ADAFUSE_OK) return rc;
+        rc = launch_pdl(shrink_finalize_kernel, dim3((unsigned)p->n_lin, (unsigned)T), dim3(128), 0, s,
+                        (const LinDesc*)p->d_desc, (const float*)sa.P, (const int32_t*)used, idx, gate,
+                        reinterpret_cast<uint16_t*>(wsb + w.off_S), T, k, p->r, w.Kext, Npad, w.tile, w.n_su,
+                        w.total_ks, w.ksg);
+        if (rc != ADAFUSE_OK) return rc;
+    }
+
     // Accumulators: two of H * Npad columns (Npad <= 256 / H).
     uint32_t accs = 32;
     while (accs < (uint32_t)(Npad * H)) accs <<= 1;
     const uint32_t stage_bytes = kAChunkBytes * H + (uint32_t)Npad * 128u;
-    const int ST = std::min(8, (int)((kSmemMax - 2048u) / stage_bytes));
+    const int ST = std::min(kMaxStages, (int)((kSmemMax - 2048u) / stage_bytes));
     if (ST < 2 || 2 * accs > 512) return ADAFUSE_ERR_UNSUPPORTED;
     const uint32_t smem = (uint32_t)ST * stage_bytes + 1024u + 1024u;
-    const int64_t n_sh = w.n_su * w.n_tt;
+    const int64_t n_sh = w.fused ? w.n_su * w.n_tt : 0;
     const int64_t n_apply = w.n_grp * w.nsplit;
     if (n_sh + n_apply > 0x7fffffff) return ADAFUSE_ERR_UNSUPPORTED;
+    if (w.nsplit > 1 && H != 1) return ADAFUSE_ERR_UNSUPPORTED;     // never: splits imply the shortest units
     ApplyArgs a{};
     a.lins = p->d_desc;
     a.maps = p->d_maps;
@@ -820,6 +1159,7 @@ int launch_apply_kernels(Plan* p, const WsLayout& w, uint8_t* wsb, const CUtenso
     a.bcols = p->b_box_cols;
     a.stall = (p->flags & ADAFUSE_PLAN_TEST_STALL) ? 1 : 0;
     a.y_f32 = (p->flags & ADAFUSE_PLAN_Y_F32) ? 1 : 0;
+    a.s_done = w.fused ? 0 : 1;
     a.Yp = w.nsplit > 1 ? reinterpret_cast<float*>(wsb + w.off_Yp) : nullptr;
     a.cnt = w.nsplit > 1 ? reinterpret_cast<int32_t*>(wsb + w.off_cnt) : nullptr;
     a.status = p->d_status;
@@ -835,7 +1175,7 @@ int launch_apply_kernels(Plan* p, const WsLayout& w, uint8_t* wsb, const CUtenso
     a.ST = ST;
     a.off_bar = (uint32_t)ST * stage_bytes;
     const int grid = (int)std::min<int64_t>(p->num_sms, n_sh + n_apply);
-    p->last_launches = 2;
+    p->last_launches = w.fused ? 2 : 4;
     switch (H) {
     case 1: return launch_apply_fused<1>(a, smem, grid, s);
     case 2: return launch_apply_fused<2>(a, smem, grid, s);

@@ -20,7 +20,8 @@
 //     (dW = Bcat[128 x Kp] * Acat[Kp x 128], K = k*r) into one of two TMEM
 //     accumulators of 128 columns.
 //   merge_fused_kernel (k*r up to 256): tiles walked down 128-column strips;
-//     warps 2-3 build the gate-scaled A strip once per strip, the B rows of
+//     the raw A rows of each strip come by TMA and warps 2-3 scale them by
+//     the gates in place (Acat, MN-major, 128-byte swizzle), the B rows of
 //     each tile come by TMA.
 //   In both, warps 4-11 are the epilogue: each warp takes a 32-row x 64-column
 //   slice: dW from TMEM (tcgen05.ld), W from the swizzled smem tile, W + dW
@@ -164,7 +165,8 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_fused_kernel(const __g
     uint64_t* accfull = aempty + a.NA;
     uint64_t* accempty = accfull + 2;
     uint64_t* donebar = accempty + 2;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(donebar + 1);
+    uint64_t* aload = donebar + 1;                // raw A rows of a strip slot landed (TMA)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(aload + a.NA);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     int* s_skip = reinterpret_cast<int*>(tmem_slot + 2);
     int* s_e = reinterpret_cast<int*>(tmem_slot + 4);
@@ -178,15 +180,18 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_fused_kernel(const __g
     if (threadIdx.x == 0) {
         for (int i = 0; i < a.SW; ++i) { mbar_init(&wfull[i], 1); mbar_init(&wempty[i], kEpiWarps); }
         for (int i = 0; i < a.SB; ++i) { mbar_init(&bfull[i], 1); mbar_init(&bempty[i], 1); }
-        for (int i = 0; i < a.NA; ++i) { mbar_init(&afull[i], 2); mbar_init(&aempty[i], 1); }
+        for (int i = 0; i < a.NA; ++i) { mbar_init(&afull[i], 2); mbar_init(&aempty[i], 1); mbar_init(&aload[i], 1); }
         for (int i = 0; i < 2; ++i) { mbar_init(&accfull[i], 1); mbar_init(&accempty[i], kEpiWarps); }
         mbar_init(donebar, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
-    // Zero the B ring: stages of skipped slots and the K padding stay zero.
+    // Zero the B ring and the A strip slots: stages of skipped slots and the
+    // K padding are never loaded and stay zero.
     for (uint32_t o = threadIdx.x * 16; o < (uint32_t)a.SB * BBytes; o += kMergeThreads * 16)
         st_shared_v4(smem_u32(sB + o), make_uint4(0, 0, 0, 0));
+    for (uint32_t o = threadIdx.x * 16; o < (uint32_t)a.NA * ABytes; o += kMergeThreads * 16)
+        st_shared_v4(smem_u32(sA + o), make_uint4(0, 0, 0, 0));
     fence_proxy_async_smem();
     griddep_wait();
     griddep_launch_dependents();
@@ -257,7 +262,7 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_fused_kernel(const __g
             TileIt it;
             it.init(a.lins, a.n_lin, t_begin);
             const uint32_t idesc = make_idesc_bf16(kTileM, kTileN, 0u, 1u);
-            const uint32_t sbo_a = (uint32_t)a.Kp * 16u;     // n-group stride of Acat
+            const uint32_t lbo_a = (uint32_t)a.Kp * 128u;    // 64-column halves of the A strip
             int64_t strip_seq = -1;
             for (int64_t i = 0; i < count; ++i) {
                 const bool first = (i == 0) || (it.rt == 0);
@@ -275,7 +280,7 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_fused_kernel(const __g
                 const uint32_t aaddr = smem_u32(sA + (size_t)ab * ABytes);
                 for (int kk = 0; kk < a.Kp / 16; ++kk) {
                     const uint64_t adesc = make_sdesc(baddr + (uint32_t)kk * 4096u, 2048u, 128u, kLayoutNone);
-                    const uint64_t bdesc = make_sdesc(aaddr + (uint32_t)kk * 256u, 128u, sbo_a, kLayoutNone);
+                    const uint64_t bdesc = make_sdesc(aaddr + (uint32_t)kk * 2048u, lbo_a, 1024u, kLayoutSw128);
                     tc_mma_bf16(d, adesc, bdesc, idesc, kk > 0 ? 1u : 0u);
                 }
                 tc_commit(&accfull[acc]);
@@ -289,12 +294,21 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_fused_kernel(const __g
         __syncwarp();
     } else if (warp == 2 || warp == 3) {
         // ------------------------------------------------------------ Acat builder
+        // The raw A rows of the selected experts for the strip's 128 columns
+        // come by TMA (3-D map over the expert stack, MN-major, 128-byte
+        // swizzle: K row c of column half h at bytes h*Kp*128 + c*128), then
+        // both warps scale each loaded row by its slot's gate in place.
+        // Rows of skipped slots and the K padding are never loaded and stay
+        // zero; columns past d_in arrive as zeros.
         if (count > 0) {
             const int tb = (warp - 2) * 32 + lane;
-            const uint32_t sbo_a = (uint32_t)a.Kp * 16u;
             TileIt it;
             it.init(a.lins, a.n_lin, t_begin);
-            int64_t strip_seq = -1;
+            int nvalid = 0;
+            for (int s2 = 0; s2 < a.ns; ++s2) if (s_e[s2] >= 0) ++nvalid;
+            const uint32_t abytes = (uint32_t)nvalid * (uint32_t)a.r * 256u;     // 2 halves x r rows x 128 B
+            const int R = a.box_rows;
+            int64_t strip_seq = -1, loaded = -1;
             for (int64_t i = 0; i < count; ++i) {
                 if (i == 0 || it.rt == 0) {
                     ++strip_seq;
@@ -302,37 +316,42 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_fused_kernel(const __g
                     bool ok = mbar_wait(&aempty[ab], (uint32_t)((strip_seq / a.NA) & 1) ^ 1u, abort_flag);
                     ok = __all_sync(0xffffffffu, ok);
                     if (!ok) break;
-                    const LinDesc L = a.lins[it.l];
                     const int n0 = it.strip * kTileN;
-                    const uint32_t abase = smem_u32(sA + (size_t)ab * ABytes);
-                    const int total = a.Kp * 16;         // (row c, 8-column group) pairs
-                    for (int id0 = 0; id0 < total; id0 += 64 * 8) {
-                        uint4 v[8];
-                        float gs[8];
+                    uint8_t* adst = sA + (size_t)ab * ABytes;
+                    if (warp == 2 && lane == 0) {
+                        const CUtensorMap* mA = a.maps + (size_t)it.l * kMapsPerLinear + kMapA;
+                        mbar_arrive_expect_tx(&aload[ab], abytes);
+                        for (int s2 = 0; s2 < a.ns; ++s2) {
+                            const int e = s_e[s2];
+                            if (e < 0) continue;
+                            for (int h = 0; h < 2; ++h)
+                                for (int j0 = 0; j0 < a.r; j0 += R)
+                                    tma_load_3d(adst + (size_t)h * a.Kp * 128u + (size_t)((s2 * a.r + j0) / 8) * 1024u,
+                                                mA, &aload[ab], n0 + 64 * h, j0, e);
+                        }
+                        loaded = strip_seq;
+                    }
+                    ok = mbar_wait(&aload[ab], (uint32_t)((strip_seq / a.NA) & 1), abort_flag);
+                    ok = __all_sync(0xffffffffu, ok);
+                    if (!ok) break;
+                    const int rowchunks = a.Kp * 8;               // 16-byte chunks per column half
+                    const int chunks = 2 * rowchunks;
+                    for (int id0 = tb; id0 < chunks; id0 += 4 * 64) {
+                        uint4 v[4];
+                        float gs[4];
+                        bool slot[4];
 #pragma unroll
-                        for (int u = 0; u < 8; ++u) {
-                            const int id = id0 + u * 64 + tb;
-                            v[u] = make_uint4(0, 0, 0, 0);
-                            gs[u] = 0.f;
-                            if (id < total) {
-                                const int c = id >> 4, ng = id & 15;
-                                const int s = c / a.r, j = c - s * a.r;
-                                const int col = n0 + ng * 8;
-                                if (s < a.ns && s_e[s] >= 0 && col < L.d_in) {
-                                    v[u] = ld_global_nc_v4(L.A + (int64_t)s_e[s] * L.a_es + (int64_t)j * L.d_in + col);
-                                    gs[u] = s_g[s];
-                                }
-                            }
+                        for (int u = 0; u < 4; ++u) {
+                            const int id = id0 + u * 64;
+                            const int c = (id % rowchunks) >> 3;       // K row of the chunk
+                            const int s2 = c / a.r;
+                            slot[u] = id < chunks && s2 < a.ns && s_e[s2] >= 0;
+                            gs[u] = slot[u] ? s_g[s2] : 0.f;
+                            v[u] = slot[u] ? ld_shared_v4(smem_u32(adst) + (uint32_t)id * 16u) : make_uint4(0, 0, 0, 0);
                         }
 #pragma unroll
-                        for (int u = 0; u < 8; ++u) {
-                            const int id = id0 + u * 64 + tb;
-                            if (id < total) {
-                                const int c = id >> 4, ng = id & 15;
-                                st_shared_v4(abase + (uint32_t)ng * sbo_a + (uint32_t)(c >> 3) * 128u + (uint32_t)(c & 7) * 16u,
-                                             scale_bf16x8(v[u], gs[u]));
-                            }
-                        }
+                        for (int u = 0; u < 4; ++u)
+                            if (slot[u]) st_shared_v4(smem_u32(adst) + (uint32_t)(id0 + u * 64) * 16u, scale_bf16x8(v[u], gs[u]));
                     }
                     fence_proxy_async_smem();
                     __syncwarp();
@@ -340,6 +359,9 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_fused_kernel(const __g
                 }
                 if (i + 1 < count) it.next(a.lins, a.n_lin);
             }
+            // After an abort the last A loads may still be in flight.
+            if (warp == 2 && lane == 0 && loaded >= 0)
+                mbar_wait_drain(&aload[loaded % a.NA], (uint32_t)((loaded / a.NA) & 1));
         }
     } else {
         // ------------------------------------------------------------ epilogue
@@ -499,6 +521,7 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_rows_kernel(const __gr
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(donebar + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     int* s_skip = reinterpret_cast<int*>(tmem_slot + 2);
+    volatile int* s_bfirst = reinterpret_cast<volatile int*>(tmem_slot + 3);   // first B-row loads issued
     int* s_e = reinterpret_cast<int*>(tmem_slot + 4);
     float* s_g = reinterpret_cast<float*>(s_e + kMaxSlots);
 
@@ -514,6 +537,7 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_rows_kernel(const __gr
         for (int i = 0; i < 2; ++i) { mbar_init(&accfull[i], 1); mbar_init(&accempty[i], kEpiWarps); }
         mbar_init(donebar, 1);
         *abort_flag = 0;
+        *s_bfirst = 0;
         fence_mbar_init();
     }
     // Zero every A slot: the K padding rows and the rows of skipped slots are
@@ -553,18 +577,22 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_rows_kernel(const __gr
             const uint32_t abytes = (uint32_t)nvalid * (uint32_t)a.r * 256u;    // 2 halves x r rows x 128 B
             const int R = a.box_rows;
             int64_t issued = 0, aseq = -1, a_issued = 0;
+            // The SM's TMA engine serves requests in issue order: the first
+            // group's B rows (issued by the Bcat builder) and the first A
+            // tile go ahead of the W stream, so the first MMA does not wait
+            // behind every W stage of the ring.
+            {
+                const uint64_t t0 = globaltimer_ns();
+                while (!*s_bfirst && !*abort_flag) {
+                    if (globaltimer_ns() - t0 > kWaitLimitNs) { *abort_flag = 1; break; }
+                }
+            }
             for (int64_t i = 0; i < count; ++i) {
                 const int sw = (int)(i % a.SW);
                 if (!mbar_wait(&empty[sw], (uint32_t)((i / a.SW) & 1) ^ 1u, abort_flag)) break;
                 const CUtensorMap* mW = a.maps + (size_t)it.l * kMapsPerLinear + kmap_in;
                 const int n0 = it.strip * kTileN, m0 = it.rt() * kTileM;
                 uint8_t* dst = sStage + (size_t)sw * a.stage_bytes;
-                if (!(a.stall && blockIdx.x == 0 && i == 0)) {
-                    mbar_arrive_expect_tx(&full[sw], kWTileBytes);
-                    tma_load_2d(dst, mW, &full[sw], n0, m0);
-                    tma_load_2d(dst + kWBoxBytes, mW, &full[sw], n0 + 64, m0);
-                    issued = i + 1;
-                }
                 if (i == 0 || it.col_first()) {
                     // the A rows of this column block, for every tile of the group
                     const int as = (int)(++aseq % a.NAR);
@@ -581,6 +609,12 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_rows_kernel(const __gr
                                             mA, &afull[as], n0 + 64 * h, j0, e);
                     }
                     a_issued = aseq + 1;
+                }
+                if (!(a.stall && blockIdx.x == 0 && i == 0)) {
+                    mbar_arrive_expect_tx(&full[sw], kWTileBytes);
+                    tma_load_2d(dst, mW, &full[sw], n0, m0);
+                    tma_load_2d(dst + kWBoxBytes, mW, &full[sw], n0 + 64, m0);
+                    issued = i + 1;
                 }
                 if (i + 1 < count) it.next(a.lins, a.n_lin);
             }
@@ -665,19 +699,33 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_rows_kernel(const __gr
                                                 &bcload[ps], j0, (a.G * it.gi + bq) * kTileM, e);
                             }
                         loaded = pseq;
+                        if (pseq == 0) *s_bfirst = 1;
                     }
                     ok = mbar_wait(&bcload[ps], (uint32_t)((pseq / NP) & 1), abort_flag);
                     ok = __all_sync(0xffffffffu, ok);
                     if (!ok) break;
                     const int groups = a.Kp / 8;
                     const int chunks = it.nb * groups * kTileM;      // 16-byte chunks: (block, column group, row)
-                    for (int id = tb; id < chunks; id += 64) {
-                        const int cg = (id / kTileM) % groups;
-                        const int s2 = (cg * 8) / a.r;
-                        const uint32_t addr = smem_u32(gbase) + (uint32_t)id * 16u;   // = block*BcBytes + cg*2048 + row*16
-                        uint4 v = make_uint4(0, 0, 0, 0);
-                        if (s2 < a.ns && s_e[s2] >= 0) v = scale_bf16x8(ld_shared_v4(addr), s_g[s2]);
-                        st_shared_v4(addr, v);
+                    // four chunks per step, their loads issued together
+                    for (int id0 = tb; id0 < chunks; id0 += 4 * 64) {
+                        uint4 v[4];
+                        float gs[4];
+                        bool live[4], slot[4];
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const int id = id0 + u * 64;
+                            const int cg = (id / kTileM) % groups;
+                            const int s2 = (cg * 8) / a.r;
+                            live[u] = id < chunks;
+                            slot[u] = live[u] && s2 < a.ns && s_e[s2] >= 0;
+                            gs[u] = slot[u] ? s_g[s2] : 0.f;
+                            v[u] = slot[u] ? ld_shared_v4(smem_u32(gbase) + (uint32_t)id * 16u) : make_uint4(0, 0, 0, 0);
+                        }
+#pragma unroll
+                        for (int u = 0; u < 4; ++u)
+                            if (live[u])    // address = block*BcBytes + cg*2048 + row*16
+                                st_shared_v4(smem_u32(gbase) + (uint32_t)(id0 + u * 64) * 16u,
+                                             slot[u] ? scale_bf16x8(v[u], gs[u]) : make_uint4(0, 0, 0, 0));
                     }
                     fence_proxy_async_smem();
                     __syncwarp();
