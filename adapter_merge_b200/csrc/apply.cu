@@ -985,34 +985,27 @@ __global__ void __launch_bounds__(ApplyShape<H>::kThreads, 1) apply_fused_kernel
                 if (last) {
                     __threadfence();
                     const float* p0 = a.Yp + ((int64_t)g * a.nsplit * a.Npad) * kApplyRows + rin;
-                    // Four tokens at a time, every split's partial loaded
-                    // before any is added (one round of L2 latency instead of
-                    // one per split); each sum still runs over the splits in
-                    // order, so the result does not depend on which split
-                    // finished last.
-                    constexpr int kTk = 4;
-                    const int n_tok = T - tb < a.Npad ? (int)(T - tb) : a.Npad;
-                    for (int c0 = 0; c0 < n_tok; c0 += kTk) {
-                        float t[kMaxSplit][kTk];
+                    for (int c0 = 0; c0 < a.Npad; c0 += 32) {
+                        // 32 independent loads per split in flight; each sum
+                        // still runs over the splits in order
+                        float v[32];
 #pragma unroll
-                        for (int s2 = 0; s2 < kMaxSplit; ++s2)
+                        for (int i = 0; i < 32; ++i) v[i] = 0.f;
+                        for (int s2 = 0; s2 < a.nsplit; ++s2) {
+                            const float* ps = p0 + ((int64_t)s2 * a.Npad + c0) * kApplyRows;
+                            float t[32];
 #pragma unroll
-                            for (int i = 0; i < kTk; ++i)
-                                t[s2][i] = (s2 < a.nsplit && c0 + i < n_tok)
-                                               ? __ldcg(p0 + ((int64_t)s2 * a.Npad + c0 + i) * kApplyRows) : 0.f;
-                        float v[kTk];
+                            for (int i = 0; i < 32; ++i)
+                                t[i] = (c0 + i < a.Npad) ? __ldcg(ps + (int64_t)i * kApplyRows) : 0.f;
 #pragma unroll
-                        for (int i = 0; i < kTk; ++i) {
-                            v[i] = 0.f;
-#pragma unroll
-                            for (int s2 = 0; s2 < kMaxSplit; ++s2) v[i] += t[s2][i];
+                            for (int i = 0; i < 32; ++i) v[i] += t[i];
                         }
                         if (row < d_out) {
-                            for (int i = 0; i < kTk && c0 + i < n_tok; ++i) {
-                                const int64_t off = (tb + c0 + i) * d_out + row;
-                                if (a.y_f32) static_cast<float*>(y)[off] = v[i];
-                                else static_cast<uint16_t*>(y)[off] = __bfloat16_as_ushort(__float2bfloat16_rn(v[i]));
-                            }
+                            uint32_t vb[32];
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) vb[i] = __float_as_uint(v[i]);
+                            store_y_rows(y, a.y_f32, (tb + c0) * d_out + row, d_out, min(32, a.Npad - c0),
+                                         T - tb - c0, vb);
                         }
                     }
                 }

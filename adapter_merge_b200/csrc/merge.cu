@@ -62,6 +62,7 @@ struct MergeArgs {
 };
 
 constexpr int kMergeThreads = 384;
+constexpr int kMergeThreadsTB = 448;     // row kernel with Bcat in TMEM: two more builder warps
 constexpr uint32_t kWTileBytes = kTileM * kTileN * 2;       // 32 KB
 constexpr uint32_t kWBoxBytes = kWTileBytes / 2;            // 16 KB: 64 cols x 128 rows
 constexpr int kEpiWarps = 8;
@@ -500,13 +501,15 @@ struct GroupTileIt {
     __device__ bool group_last() const { return b == nb - 1 && strip == n_strips - 1; }
 };
 
-__global__ void __launch_bounds__(kMergeThreads, 1) merge_rows_kernel(const __grid_constant__ MergeArgs a)
+template <bool kTB>
+__global__ void __launch_bounds__(kTB ? kMergeThreadsTB : kMergeThreads, 1)
+    merge_rows_kernel(const __grid_constant__ MergeArgs a)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sStage = base;                       // SW x W tile (32 KB)
     uint8_t* sA = base + a.off_A;                 // NAR x A tile [Kp x 128], MN-major, 128-byte swizzle
-    uint8_t* sBcat = base + a.off_B;              // NA x [128 x Kp] gate-scaled B rows, G per group slot
+    uint8_t* sBcat = base + a.off_B;              // NA x [128 x Kp] gate-scaled B rows, G per group slot (smem Bcat)
     const int NP = a.NA / a.G;                    // Bcat group slots
     uint64_t* full = reinterpret_cast<uint64_t*>(base + a.off_bar);
     uint64_t* empty = full + a.SW;
@@ -533,7 +536,7 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_rows_kernel(const __gr
     if (threadIdx.x == 0) {
         for (int i = 0; i < a.SW; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], kEpiWarps + 1); }
         for (int i = 0; i < a.NAR; ++i) { mbar_init(&afull[i], 1); mbar_init(&aempty[i], 1); }
-        for (int i = 0; i < NP; ++i) { mbar_init(&bcfull[i], 2); mbar_init(&bcempty[i], 1); mbar_init(&bcload[i], 1); }
+        for (int i = 0; i < NP; ++i) { mbar_init(&bcfull[i], kTB ? 4 : 2); mbar_init(&bcempty[i], 1); mbar_init(&bcload[i], 1); }
         for (int i = 0; i < 2; ++i) { mbar_init(&accfull[i], 1); mbar_init(&accempty[i], kEpiWarps); }
         mbar_init(donebar, 1);
         *abort_flag = 0;
@@ -543,7 +546,7 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_rows_kernel(const __gr
     // Zero every A slot: the K padding rows and the rows of skipped slots are
     // never loaded and must read as finite zeros.
     for (int st = 0; st < a.NAR; ++st)
-        for (uint32_t o = threadIdx.x * 16; o < ATile; o += kMergeThreads * 16)
+        for (uint32_t o = threadIdx.x * 16; o < ATile; o += blockDim.x * 16)
             st_shared_v4(smem_u32(sA + (size_t)st * ATile + o), make_uint4(0, 0, 0, 0));
     fence_proxy_async_smem();
     griddep_wait();
@@ -552,8 +555,11 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_rows_kernel(const __gr
     __syncthreads();
     if (*s_skip) return;       // switch between identical selections: nothing to do
 
+    // TMEM: two 128-column accumulators, then (kTB) the Bcat group slots,
+    // Kp / 2 columns per row block.
+    constexpr uint32_t kTmemCols = kTB ? 512u : 256u;
     if (warp == 1) {
-        tmem_alloc(tmem_slot, 256);
+        tmem_alloc(tmem_slot, kTmemCols);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -581,7 +587,7 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_rows_kernel(const __gr
             // group's B rows (issued by the Bcat builder) and the first A
             // tile go ahead of the W stream, so the first MMA does not wait
             // behind every W stage of the ring.
-            {
+            if (!kTB) {                 // (B rows in TMEM come by plain loads)
                 const uint64_t t0 = globaltimer_ns();
                 while (!*s_bfirst && !*abort_flag) {
                     if (globaltimer_ns() - t0 > kWaitLimitNs) { *abort_flag = 1; break; }
@@ -593,10 +599,14 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_rows_kernel(const __gr
                 const CUtensorMap* mW = a.maps + (size_t)it.l * kMapsPerLinear + kmap_in;
                 const int n0 = it.strip * kTileN, m0 = it.rt() * kTileM;
                 uint8_t* dst = sStage + (size_t)sw * a.stage_bytes;
-                if (i == 0 || it.col_first()) {
-                    // the A rows of this column block, for every tile of the group
+                // The A rows of this column block, for every tile of the
+                // group.  The first tile's go ahead of its W tile (the TMA
+                // engine serves an SM's requests in issue order); later ones
+                // follow their W tile, so a full A ring never holds up the W
+                // stream.
+                auto issue_a = [&]() -> bool {
                     const int as = (int)(++aseq % a.NAR);
-                    if (!mbar_wait(&aempty[as], (uint32_t)((aseq / a.NAR) & 1) ^ 1u, abort_flag)) break;
+                    if (!mbar_wait(&aempty[as], (uint32_t)((aseq / a.NAR) & 1) ^ 1u, abort_flag)) return false;
                     const CUtensorMap* mA = a.maps + (size_t)it.l * kMapsPerLinear + kMapA;
                     uint8_t* adst = sA + (size_t)as * ATile;
                     mbar_arrive_expect_tx(&afull[as], abytes);
@@ -609,13 +619,16 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_rows_kernel(const __gr
                                             mA, &afull[as], n0 + 64 * h, j0, e);
                     }
                     a_issued = aseq + 1;
-                }
+                    return true;
+                };
+                if (i == 0 && !issue_a()) break;
                 if (!(a.stall && blockIdx.x == 0 && i == 0)) {
                     mbar_arrive_expect_tx(&full[sw], kWTileBytes);
                     tma_load_2d(dst, mW, &full[sw], n0, m0);
                     tma_load_2d(dst + kWBoxBytes, mW, &full[sw], n0 + 64, m0);
                     issued = i + 1;
                 }
+                if (i > 0 && it.col_first() && !issue_a()) break;
                 if (i + 1 < count) it.next(a.lins, a.n_lin);
             }
             // Drain the TMA loads still in flight before the CTA may exit.
@@ -650,10 +663,15 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_rows_kernel(const __gr
                 const uint32_t d = tmem_base + (uint32_t)acc * kTileN;
                 const uint32_t bcaddr = smem_u32(sBcat + (size_t)(ps * a.G + it.b) * BcBytes);
                 const uint32_t aaddr = smem_u32(sA + (size_t)as * ATile);
+                const uint32_t bc_tmem = tmem_base + 256u + (uint32_t)((ps * a.G + it.b) * (a.Kp / 2));
                 for (int kk = 0; kk < a.Kp / 16; ++kk) {
-                    const uint64_t adesc = make_sdesc(bcaddr + (uint32_t)kk * 4096u, 2048u, 128u, kLayoutNone);
                     const uint64_t bdesc = make_sdesc(aaddr + (uint32_t)kk * 2048u, lbo_a, 1024u, kLayoutSw128);
-                    tc_mma_bf16(d, adesc, bdesc, idesc, kk > 0 ? 1u : 0u);
+                    if (kTB) {
+                        tc_mma_bf16_ta(d, bc_tmem + (uint32_t)kk * 8u, bdesc, idesc, kk > 0 ? 1u : 0u);
+                    } else {
+                        const uint64_t adesc = make_sdesc(bcaddr + (uint32_t)kk * 4096u, 2048u, 128u, kLayoutNone);
+                        tc_mma_bf16(d, adesc, bdesc, idesc, kk > 0 ? 1u : 0u);
+                    }
                 }
                 tc_commit(&accfull[acc]);
                 tc_commit(&empty[sw]);
@@ -665,7 +683,59 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_rows_kernel(const __gr
             mbar_wait_drain(donebar, 0);
         }
         __syncwarp();
-    } else if (warp == 2 || warp == 3) {
+    } else if (kTB && (warp == 2 || warp == 3 || warp >= 4 + kEpiWarps)) {
+        // ------------------------------------------------------------ Bcat builder (TMEM)
+        // Warps 2, 3, 12 and 13 cover TMEM lane quarters 2, 3, 0 and 1: each
+        // lane loads its row's B values of every selected expert (16-byte
+        // global loads), scales them by the slot's gate, packs them two bf16
+        // per 32-bit column (lower K index in the low half) and stores them
+        // into the group slot's TMEM columns; slots without an expert, the K
+        // padding and rows past d_out are zeros.
+        if (count > 0) {
+            const int q = warp & 3;
+            GroupTileIt it;
+            it.init(a.lins, a.n_lin, t_begin, a.G);
+            int64_t pseq = -1;
+            for (int64_t i = 0; i < count; ++i) {
+                if (i == 0 || it.group_first()) {
+                    ++pseq;
+                    const int ps = (int)(pseq % NP);
+                    bool ok = mbar_wait(&bcempty[ps], (uint32_t)((pseq / NP) & 1) ^ 1u, abort_flag);
+                    ok = __all_sync(0xffffffffu, ok);
+                    if (!ok) break;
+                    tc_fence_after();
+                    const LinDesc& L = a.lins[it.l];
+                    const uint16_t* Bp = L.B;
+                    const int64_t b_es = L.b_es;
+                    const int d_out = L.d_out;
+                    for (int bq = 0; bq < it.nb; ++bq) {
+                        const int row = (a.G * it.gi + bq) * kTileM + q * 32 + lane;
+                        const uint32_t col0 = 256u + (uint32_t)((ps * a.G + bq) * (a.Kp / 2));
+                        for (int k32 = 0; k32 < a.Kp / 32; ++k32) {
+                            uint4 v[4];
+#pragma unroll
+                            for (int pc = 0; pc < 4; ++pc) {
+                                const int c = k32 * 32 + pc * 8;          // 8 consecutive K of one slot
+                                const int s2 = c / a.r, jj = c - s2 * a.r;
+                                v[pc] = make_uint4(0, 0, 0, 0);
+                                if (s2 < a.ns && s_e[s2] >= 0 && row < d_out)
+                                    v[pc] = scale_bf16x8(ld_global_nc_v4(Bp + (int64_t)s_e[s2] * b_es + (int64_t)row * a.r + jj),
+                                                         s_g[s2]);
+                            }
+                            const uint32_t w[16] = {v[0].x, v[0].y, v[0].z, v[0].w, v[1].x, v[1].y, v[1].z, v[1].w,
+                                                    v[2].x, v[2].y, v[2].z, v[2].w, v[3].x, v[3].y, v[3].z, v[3].w};
+                            tc_st_x16(tmem_base + ((uint32_t)(q * 32) << 16) + col0 + (uint32_t)k32 * 16u, w);
+                        }
+                    }
+                    tc_wait_st();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&bcfull[ps]);
+                }
+                if (i + 1 < count) it.next(a.lins, a.n_lin);
+            }
+        }
+    } else if (!kTB && (warp == 2 || warp == 3)) {
         // ------------------------------------------------------------ Bcat builder
         if (count > 0) {
             const int tb = (warp - 2) * 32 + lane;
@@ -737,7 +807,7 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_rows_kernel(const __gr
             if (warp == 2 && lane == 0 && loaded >= 0)
                 mbar_wait_drain(&bcload[loaded % NP], (uint32_t)((loaded / NP) & 1));
         }
-    } else {
+    } else if (warp >= 4 && warp < 4 + kEpiWarps) {
         // ------------------------------------------------------------ epilogue
         const int ew = warp - 4;
         const int q = warp & 3;
@@ -797,7 +867,7 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_rows_kernel(const __gr
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, 256);
+        tmem_dealloc(tmem_base, kTmemCols);
     }
     if (threadIdx.x == 0 && *abort_flag) atomicOr(a.status, ADAFUSE_STATUS_TIMEOUT);
 }
@@ -883,17 +953,27 @@ int launch_merge_fused(Plan* p, const int32_t* idx0, const float* gate0, const i
         // Single-block groups (a plain row walk, every tile its own A tile)
         // only where they buy a W stage: at k*r = 128, G = 1 with four W
         // stages ran the 13B switch 17 % faster than G = 2 with three.
-        const uint32_t at = (uint32_t)a.Kp * 256u, bc = at;
+        //
+        // Above k*r = 64 (and K a multiple of 32) the Bcat of each group lives
+        // in TMEM instead (Kp / 2 columns per row block beside the two
+        // accumulators, at most 256 columns), so shared memory holds only W
+        // stages and A tiles and a group can share each A tile among up to
+        // four row blocks without giving up a W stage.
+        const uint32_t at = (uint32_t)a.Kp * 256u;
+        const bool tb = a.Kp > 64 && a.Kp % 32 == 0;
+        const uint32_t bc = tb ? 0u : at;                    // smem per Bcat block
         const bool long_walk = p->merge_tiles >= 128 * (int64_t)p->num_sms;
         int SW = 0, NA = 0, NAR = 0, G = 0;
         for (int g : {8, 4, 2, 1}) {
             if (g >= 4 && !long_walk) continue;
-            for (int np : {2, 1})
+            for (int np : {2, 1}) {
+                if (tb && np * g * (a.Kp / 2) > 256) continue;
                 for (int nar : {3, 2}) {
                     const int64_t room = (int64_t)kSmemMax - 2048 - (int64_t)np * g * bc - (int64_t)nar * at;
                     const int sw = room > 0 ? (int)std::min<int64_t>(4, room / kWTileBytes) : 0;
                     if (sw > SW) { SW = sw; NA = np * g; NAR = nar; G = g; }
                 }
+            }
         }
         if (SW >= 2) {
             a.SW = SW; a.SB = 0; a.NA = NA; a.NAR = NAR; a.G = G;
@@ -902,11 +982,18 @@ int launch_merge_fused(Plan* p, const int32_t* idx0, const float* gate0, const i
             a.off_B = a.off_A + (uint32_t)NAR * at;
             a.off_bar = a.off_B + (uint32_t)NA * bc;
             const uint32_t smem = a.off_bar + 1024u + 1024u;
-            if (cudaFuncSetAttribute(merge_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-                return ADAFUSE_ERR_CUDA;
             const int grid = (int)std::min<int64_t>(p->num_sms, p->merge_tiles);
             p->last_launches = 1;
-            return launch_pdl(merge_rows_kernel, dim3(grid), dim3(kMergeThreads), smem, s, a);
+            if (tb) {
+                if (cudaFuncSetAttribute(merge_rows_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem) != cudaSuccess)
+                    return ADAFUSE_ERR_CUDA;
+                return launch_pdl(merge_rows_kernel<true>, dim3(grid), dim3(kMergeThreadsTB), smem, s, a);
+            }
+            if (cudaFuncSetAttribute(merge_rows_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+                cudaSuccess)
+                return ADAFUSE_ERR_CUDA;
+            return launch_pdl(merge_rows_kernel<false>, dim3(grid), dim3(kMergeThreads), smem, s, a);
         }
     }
     const uint32_t BBytes = (uint32_t)a.Kp * 256u;

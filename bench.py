@@ -482,11 +482,27 @@ def measure_13b(dev, peak, steps=10):
 
     m_ms = ev_mean(merge)
     a_ms = ev_mean(apply)
+    # in-place switch between two selections (rank 2kr = 128 here)
+    sel = [(torch.tensor(i_, dtype=torch.int32, device=dev), torch.tensor(g_, dtype=torch.float32, device=dev))
+           for i_, g_ in (((1, 5), (0.4, 0.3)), ((6, 2), (0.5, 0.2)))]
+    plan.merge(*sel[0])
+    cur = {"i": 0}
+
+    def switch(ev):
+        new, old = sel[(cur["i"] + 1) % 2], sel[cur["i"] % 2]
+        if ev is not None:
+            ev[0].record(stream)
+        plan.switch(new[0], new[1], old[0], old[1])
+        if ev is not None:
+            ev[1].record(stream)
+        cur["i"] += 1
+
+    s_ms = ev_mean(switch)
     rc, st = plan.status()
     if rc != 0 or st != 0:
         raise RuntimeError(f"device status {st} in the 13B measurement")
     U = int(torch.unique(state["idx"]).numel())
-    mb, ab = merge_bytes(cfg, cfg.k), apply_bytes(cfg, T, U)
+    mb, ab, sb = merge_bytes(cfg, cfg.k), apply_bytes(cfg, T, U), merge_bytes(cfg, 2 * cfg.k)
     plan.destroy()
     out = {"workload": f"{cfg.name}: {cfg.n_lin} linears, E={cfg.E}, r={cfg.r}, top-{cfg.k}; merge for one "
                        f"request, apply for T={T} sequences",
@@ -497,6 +513,9 @@ def measure_13b(dev, peak, steps=10):
                      "gbs": round(ab / (a_ms * 1e-3) / 1e9, 1),
                      "frac_of_peak": round(ab / (a_ms * 1e-3) / 1e9 / peak, 4), "bytes": ab,
                      "distinct_experts": U, "note": "one apply call (all its launches)"},
+           "switch": {"ms": round(s_ms, 4), "gbs": round(sb / (s_ms * 1e-3) / 1e9, 1),
+                      "frac_of_peak": round(sb / (s_ms * 1e-3) / 1e9 / peak, 4), "bytes": sb,
+                      "note": "W' <- W' - dW(old) + dW(new) in place, one launch, rank 2kr = 128"},
            "steps": steps}
     del w, W_out, X, ys, ws
     torch.cuda.empty_cache()
@@ -685,17 +704,51 @@ def main():
         h_sel = torch.empty((4, cfg.k), dtype=torch.float32, pin_memory=True)
         ne = 3
 
+        # With the weights on the host, the merge is pipelined over chunks of
+        # layers through the same public calls (one plan and one merge call
+        # per chunk): the copy in of chunk c+1, the merge of chunk c and the
+        # copy out of chunk c-1 overlap on three streams, so the two PCIe
+        # directions run at once.
+        chunks = []
+        if full:
+            per = max(1, len(cfg.linears) // 8)
+            for c0 in range(0, len(cfg.linears), per):
+                c1 = min(len(cfg.linears), c0 + per)
+                ow = sum(l.d_out * l.d_in for l in cfg.linears[:c0])
+                nw = sum(l.d_out * l.d_in for l in cfg.linears[c0:c1])
+                oa = sum(cfg.E * cfg.r * l.d_in for l in cfg.linears[:c0])
+                na = sum(cfg.E * cfg.r * l.d_in for l in cfg.linears[c0:c1])
+                ob = sum(cfg.E * l.d_out * cfg.r for l in cfg.linears[:c0])
+                nb = sum(cfg.E * l.d_out * cfg.r for l in cfg.linears[c0:c1])
+                cplan = am.Plan(list(zip(w.W_views[c0:c1], W_out_views[c0:c1], w.A_views[c0:c1],
+                                         w.B_views[c0:c1])), cfg.E, cfg.r)
+                chunks.append((cplan, slice(ow, ow + nw), slice(oa, oa + na), slice(ob, ob + nb)))
+            s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+
         def e2e_merge(ev, resident):
             ev[0].record(stream)
-            if not resident:
-                w.W.copy_(h_W, non_blocking=True)
-                w.A.copy_(h_A, non_blocking=True)
-                w.B.copy_(h_B, non_blocking=True)
             x_req.copy_(h_xreq, non_blocking=True)
             idx1, gate1 = am.pregate(x_req, w.W_r, cfg.k)
-            plan.merge(idx1[0], gate1[0])
-            if not resident:
-                h_Wout.copy_(W_out, non_blocking=True)
+            if resident:
+                plan.merge(idx1[0], gate1[0])
+            else:
+                s_in.wait_stream(stream)
+                done_in, done_m = [], []
+                for (cplan, sw_, sa_, sb_) in chunks:
+                    with torch.cuda.stream(s_in):
+                        w.W[sw_].copy_(h_W[sw_], non_blocking=True)
+                        w.A[sa_].copy_(h_A[sa_], non_blocking=True)
+                        w.B[sb_].copy_(h_B[sb_], non_blocking=True)
+                        e_in = torch.cuda.Event()
+                        e_in.record(s_in)
+                    stream.wait_event(e_in)
+                    cplan.merge(idx1[0], gate1[0], stream=stream)
+                    e_m = torch.cuda.Event()
+                    e_m.record(stream)
+                    with torch.cuda.stream(s_out):
+                        s_out.wait_event(e_m)
+                        h_Wout[sw_].copy_(W_out[sw_], non_blocking=True)
+                stream.wait_stream(s_out)
             h_sel[0].copy_(idx1[0].view(torch.float32), non_blocking=True)
             h_sel[1].copy_(gate1[0], non_blocking=True)
             ev[1].record(stream)
@@ -739,12 +792,16 @@ def main():
                "resident": {"value": round(job_throughput(world, mb, em_r), 2), "unit": "GB/s",
                             "h2d_bytes_per_step": x_req.numel() * 2, "d2h_bytes_per_step": 2 * cfg.k * 4,
                             "note": "weights and adapters resident; only the router input and the selection cross"},
-               "note": ("merge with W, A, B in and W' out through pinned host buffers each step; apply with "
-                        "x in and y out (weights resident)") if full else
+               "note": ("merge with W, A, B in and W' out through pinned host buffers each step, pipelined "
+                        "over 8 chunks of layers (a plan and a merge call per chunk; copies in, merges and "
+                        "copies out overlap on three streams); apply with x in and y out (weights "
+                        "resident)") if full else
                        ("host memory holds no pinned model copy per rank: merge with the router input in and "
                         "the selection out (weights resident); apply with x in and y out")}
         if full:
-            del h_W, h_A, h_B, h_Wout
+            for (cplan, *_rest) in chunks:
+                cplan.destroy()
+            del h_W, h_A, h_B, h_Wout, chunks
 
     # The NEXT rows on the same plan, outside the timed region: in-place switch
     # between two selections (rank 2kr), the one-launch-per-linear merge, and
