@@ -455,7 +455,6 @@ struct ApplyArgs {
     int32_t bcols;                  // columns per B-row box of the expand: 8, 16 or 32
     int32_t stall;                  // test hook: CTA 0 withholds its first stage
     int32_t y_f32;                  // outputs are the fp32 accumulators (ADAFUSE_PLAN_Y_F32), not bf16
-    int32_t s_done;                 // S was finished by earlier launches: expand chunks need no wait
     float* Yp;                      // split partials [groups][nsplit][Npad][128 H] fp32
     int32_t* cnt;                   // [groups] splits finished (cleared by the segment build)
     int32_t ST;
@@ -591,7 +590,7 @@ __device__ __forceinline__ void finalize_slice(const ApplyArgs& a, const int* s_
 // share, all K-major; W, A and x use the 128-byte swizzle, B rows the layouts
 // of their boxes.  Block h of an apply unit accumulates in TMEM columns
 // [h*Npad, (h+1)*Npad) of the unit's accumulator; a shrink unit uses block 0.
-template <int H>
+template <int H, bool kFused>
 __global__ void __launch_bounds__(ApplyShape<H>::kThreads, 1) apply_fused_kernel(const __grid_constant__ ApplyArgs a)
 {
     constexpr int kApplyEpiWarps = ApplyShape<H>::kEpiWarps;
@@ -661,7 +660,7 @@ __global__ void __launch_bounds__(ApplyShape<H>::kThreads, 1) apply_fused_kernel
                 s_unit[j] = u;
                 mbar_arrive(&ufull[j]);
                 if (u < 0) break;
-                if (u < a.n_sh) {
+                if (kFused && u < a.n_sh) {
                     // shrink unit: the live A rows of Acat tile mq (boxes of
                     // whole experts, runs of consecutive expert ids in one
                     // load where r allows) and the x chunk, per 64 columns
@@ -736,7 +735,7 @@ __global__ void __launch_bounds__(ApplyShape<H>::kThreads, 1) apply_fused_kernel
                 bool s_ready = false;
                 for (int kc = c0; kc < c1; ++kc, ++gc) {
                     const int s = (int)(gc % a.ST);
-                    if (kc >= nKb && !s_ready && !a.s_done) {
+                    if (kFused && kc >= nKb && !s_ready) {
                         // S of this linear and token tile: every 32-row slice
                         // finalized (released by the finalizing warps)
                         const int* rp = a.ready + (int64_t)tt * a.n_lin + l;
@@ -804,7 +803,7 @@ __global__ void __launch_bounds__(ApplyShape<H>::kThreads, 1) apply_fused_kernel
                 mbar_arrive(&uempty[j]);
                 if (u < 0) break;
                 int c0 = 0, c1 = 0, nKb = 0;
-                bool shrink = u < a.n_sh;
+                const bool shrink = kFused && u < a.n_sh;
                 if (shrink) {
                     const int tt = u / a.n_su;
                     ShrinkUnit su;
@@ -899,7 +898,7 @@ __global__ void __launch_bounds__(ApplyShape<H>::kThreads, 1) apply_fused_kernel
             if (!__all_sync(0xffffffffu, ok)) break;
             tc_fence_after();
             const uint32_t tacc = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)acc * a.acc_stride;
-            if (u < a.n_sh) {
+            if (kFused && u < a.n_sh) {
                 const int tt = u / a.n_su;
                 const int64_t ul = u - (int64_t)tt * a.n_su;
                 ShrinkUnit su;
@@ -1047,13 +1046,13 @@ bool encode_tile_map(CUtensorMap* m, const void* ptr, int rank, const cuuint64_t
 // the call's counters), then the fused shrink + apply kernel.  `xmaps` holds
 // the call's x maps and then the shrink-output map, `yp` is the device table
 // of output pointers and `wsb` the workspace laid out by `w`.
-template <int H>
+template <int H, bool kFused>
 int launch_apply_fused(const ApplyArgs& a, uint32_t smem, int grid, cudaStream_t s)
 {
-    if (cudaFuncSetAttribute(apply_fused_kernel<H>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+    if (cudaFuncSetAttribute(apply_fused_kernel<H, kFused>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
         cudaSuccess)
         return ADAFUSE_ERR_CUDA;
-    return launch_pdl(apply_fused_kernel<H>, dim3(grid), dim3(ApplyShape<H>::kThreads), smem, s, a);
+    return launch_pdl(apply_fused_kernel<H, kFused>, dim3(grid), dim3(ApplyShape<H>::kThreads), smem, s, a);
 }
 
 int launch_apply_kernels(Plan* p, const WsLayout& w, uint8_t* wsb, const CUtensorMap* xmaps, void* const* yp,
@@ -1152,7 +1151,6 @@ int launch_apply_kernels(Plan* p, const WsLayout& w, uint8_t* wsb, const CUtenso
     a.bcols = p->b_box_cols;
     a.stall = (p->flags & ADAFUSE_PLAN_TEST_STALL) ? 1 : 0;
     a.y_f32 = (p->flags & ADAFUSE_PLAN_Y_F32) ? 1 : 0;
-    a.s_done = w.fused ? 0 : 1;
     a.Yp = w.nsplit > 1 ? reinterpret_cast<float*>(wsb + w.off_Yp) : nullptr;
     a.cnt = w.nsplit > 1 ? reinterpret_cast<int32_t*>(wsb + w.off_cnt) : nullptr;
     a.status = p->d_status;
@@ -1169,10 +1167,14 @@ int launch_apply_kernels(Plan* p, const WsLayout& w, uint8_t* wsb, const CUtenso
     a.off_bar = (uint32_t)ST * stage_bytes;
     const int grid = (int)std::min<int64_t>(p->num_sms, n_sh + n_apply);
     p->last_launches = w.fused ? 2 : 4;
+    if (w.fused) {
+        if (H != 1) return ADAFUSE_ERR_UNSUPPORTED;     // never: fewer units than SMs imply the shortest units
+        return launch_apply_fused<1, true>(a, smem, grid, s);
+    }
     switch (H) {
-    case 1: return launch_apply_fused<1>(a, smem, grid, s);
-    case 2: return launch_apply_fused<2>(a, smem, grid, s);
-    default: return launch_apply_fused<4>(a, smem, grid, s);
+    case 1: return launch_apply_fused<1, false>(a, smem, grid, s);
+    case 2: return launch_apply_fused<2, false>(a, smem, grid, s);
+    default: return launch_apply_fused<4, false>(a, smem, grid, s);
     }
 }
 }  // namespace

@@ -954,15 +954,18 @@ int launch_merge_fused(Plan* p, const int32_t* idx0, const float* gate0, const i
         // only where they buy a W stage: at k*r = 128, G = 1 with four W
         // stages ran the 13B switch 17 % faster than G = 2 with three.
         //
-        // Above k*r = 64 (and K a multiple of 32) the Bcat of each group lives
-        // in TMEM instead (Kp / 2 columns per row block beside the two
-        // accumulators, at most 256 columns), so shared memory holds only W
-        // stages and A tiles and a group can share each A tile among up to
-        // four row blocks without giving up a W stage.
+        // From a contraction depth of 64 (K a multiple of 32) the Bcat of each
+        // group lives in TMEM instead (Kp / 2 columns per row block beside the
+        // two accumulators, at most 256 columns), so shared memory holds only
+        // W stages and A tiles and a group can share each A tile among more
+        // row blocks without giving up a W stage.  Only on long walks: at
+        // Kp = 32 the shared-memory Bcat measured faster (7B merge 4.52 vs
+        // 4.57 ms), and on a single layer the first TMA-loaded Bcat is ready
+        // sooner than one built from global loads (k*r = 128: 34.8 vs 39.7 us).
         const uint32_t at = (uint32_t)a.Kp * 256u;
-        const bool tb = a.Kp > 64 && a.Kp % 32 == 0;
-        const uint32_t bc = tb ? 0u : at;                    // smem per Bcat block
         const bool long_walk = p->merge_tiles >= 128 * (int64_t)p->num_sms;
+        const bool tb = long_walk && a.Kp >= 64 && a.Kp % 32 == 0;
+        const uint32_t bc = tb ? 0u : at;                    // smem per Bcat block
         int SW = 0, NA = 0, NAR = 0, G = 0;
         for (int g : {8, 4, 2, 1}) {
             if (g >= 4 && !long_walk) continue;

@@ -2,10 +2,9 @@
 // (token, slot) pairs, numbered p = t*k + s, stably sorted by expert index.
 //
 // One CTA.  Each thread owns a contiguous run of pairs and counts its experts;
-// an exclusive scan over (expert, thread) -- shuffles inside each warp, then
-// the eight warp totals -- gives every thread its write cursor per expert,
-// and a second pass over the same run scatters the pair ids, so the order
-// inside a segment is ascending p.  Indices outside [0, E) are left
+// an exclusive scan over (expert, thread) gives every thread its write cursor
+// per expert, and a second pass over the same run scatters the pair ids, so
+// the order inside a segment is ascending p.  Indices outside [0, E) are left
 // out and flagged.
 #include "internal.h"
 #include "ptx.cuh"
@@ -15,7 +14,6 @@ namespace af {
 namespace {
 
 constexpr int kSegThreads = 256;
-constexpr int kSegWarps = kSegThreads / 32;
 
 // zero[0 .. n_zero) is cleared as well: the counters the apply kernel of the
 // same call starts from (nothing else on the stream touches them in between).
@@ -24,9 +22,8 @@ __global__ void __launch_bounds__(kSegThreads) segments_kernel(const int32_t* id
                                                                int32_t* status, int32_t* zero, int64_t n_zero)
 {
     __shared__ int cnt[kSegThreads][kMaxE + 1];
-    __shared__ int s_wsum[kSegWarps][kMaxE + 1];
     __shared__ int s_off[kMaxE + 1];
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int tid = threadIdx.x;
     griddep_wait();
     griddep_launch_dependents();
     for (int64_t i = tid; i < n_zero; i += kSegThreads) zero[i] = 0;
@@ -40,25 +37,12 @@ __global__ void __launch_bounds__(kSegThreads) segments_kernel(const int32_t* id
         if (e < 0 || e >= E) { bad = 1; continue; }
         cnt[tid][e] += 1;
     }
-    // Exclusive prefix of cnt[.][e] over the threads, for every expert: a
-    // shuffle scan inside each warp, then the warp totals in warp order.
-    for (int e = 0; e < E; ++e) {
-        const int c = cnt[tid][e];
-        int incl = c;
-#pragma unroll
-        for (int d = 1; d < 32; d <<= 1) {
-            const int v = __shfl_up_sync(0xffffffffu, incl, d);
-            if (lane >= d) incl += v;
-        }
-        cnt[tid][e] = incl - c;                      // exclusive within the warp
-        if (lane == 31) s_wsum[warp][e] = incl;
-    }
     __syncthreads();
     if (tid < E) {
         int run = 0;
-        for (int w = 0; w < kSegWarps; ++w) {
-            const int c = s_wsum[w][tid];
-            s_wsum[w][tid] = run;
+        for (int t2 = 0; t2 < kSegThreads; ++t2) {
+            const int c = cnt[t2][tid];
+            cnt[t2][tid] = run;
             run += c;
         }
         s_off[tid + 1] = run;        // segment size for now
@@ -76,7 +60,6 @@ __global__ void __launch_bounds__(kSegThreads) segments_kernel(const int32_t* id
         for (int e = 0; e <= E; ++e) offsets[e] = s_off[e];
     }
     __syncthreads();
-    for (int e = 0; e < E; ++e) cnt[tid][e] += s_wsum[warp][e];
     for (int64_t p = p0; p < p1; ++p) {
         const int e = idx[p];
         if (e < 0 || e >= E) continue;

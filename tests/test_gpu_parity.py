@@ -499,6 +499,45 @@ def test_apply_equals_merged_weights(am, cuda_device):
         assert np.all(np.abs(y - ym) <= bound)
 
 
+def test_merge_long_walk_edge_cases(am, cuda_device):
+    """A plan just long enough for the long-walk configurations (at least 128
+    tiles per SM: row-block groups of four, the gate-scaled B rows in TMEM
+    from a contraction depth of 64): a merge at k*r = 96 with a skipped
+    out-of-range index and an expert repeated in two slots, then the in-place
+    switch to another selection at 2kr = 128 and one at 2kr = 64 (k = 1,
+    Kp = 64), each checked on two rows of every 128-row block of every linear
+    against the oracle."""
+    cfg = synth.custom([(1024, 15360)] * 20, 6, 32, 3, 1, name="longwalk")
+    m = Model(cfg, cuda_device)
+    m.W_out_flat.fill_(float("nan"))
+    sel, g = [4, 9, 4], [0.35, 0.5, 0.15]                   # 9 is out of range: skipped and flagged
+    run_merge(am, m, sel, np.array(g, np.float32), cuda_device)
+    rc, st = m.plan.status()
+    assert rc == 0 and st == am.STATUS_BAD_INDEX
+    g64 = [float(np.float32(x)) for x in g]
+    for l in range(cfg.n_lin):
+        Wl, Ol, Al, Bl = m.w.W_views[l], m.W_out[l], m.w.A_views[l], m.w.B_views[l]
+        rows = block_rows(1024, l)
+        slots = [e if 0 <= e < cfg.E else -1 for e in sel]
+        valid = [(e, gg) for e, gg in zip(slots, g64) if e >= 0]
+        assert merge_delta_bound_ok(Ol, Wl, Al, Bl, [e for e, _ in valid], [gg for _, gg in valid])
+        merge_rows_check(Ol, Wl, Al, Bl, rows, [e for e, _ in valid], [gg for _, gg in valid],
+                         f"long walk merge linear {l}")
+    d = lambda a_, t: torch.as_tensor(np.asarray(a_).astype(t)).to(cuda_device)
+    for (new_i, new_g, old_i, old_g) in (([2, 0], [0.45, 0.25], [1, 5], [0.3, 0.2]),
+                                         ([3], [0.6], [2], [0.4])):
+        # the weights hold the old selection's merge, then switch in place
+        run_merge(am, m, old_i, np.array(old_g, np.float32), cuda_device)
+        m.plan.switch(d(new_i, np.int32), d(new_g, np.float32), d(old_i, np.int32), d(old_g, np.float32))
+        torch.cuda.synchronize()
+        assert m.plan.status() == (0, 0)
+        for l in range(0, cfg.n_lin, 3):
+            Wl, Ol, Al, Bl = m.w.W_views[l], m.W_out[l], m.w.A_views[l], m.w.B_views[l]
+            merge_rows_check(Ol, Wl, Al, Bl, block_rows(1024, l + 5, per_block=1), new_i,
+                             [float(np.float32(x)) for x in new_g], f"long walk switch {len(new_i)} linear {l}",
+                             base=True, base_slots=old_i, base_gates=[float(np.float32(x)) for x in old_g])
+
+
 # ------------------------------------------------------------- full sizes
 
 ORACLE_THREADS = max(1, min(16, os.cpu_count() or 1))
