@@ -620,6 +620,7 @@ def main():
     if rc != 0 or st != 0:
         raise RuntimeError(f"device status {st} after warm-up")
     U = int(torch.unique(idxT).numel())
+    apply_launches = plan.last_launches          # 4 (segments, shrink, finalize, apply) or 2
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     t_start = torch.cuda.Event(enable_timing=True)
@@ -887,7 +888,9 @@ def main():
             "apply": {"tokens_per_s": round(apply_tps, 1), "ms": round(a_part, 4), "call_ms": round(a_call, 4),
                       "gbs": round(apply_gbs, 2), "bytes": ab, "distinct_experts": U,
                       "frac_of_peak": round(apply_gbs / peak, 4),
-                      "note": "call = segment build + fused shrink/apply kernel (2 launches)"},
+                      "launches": apply_launches,
+                      "note": ("call = segment build, shrink, finalize, fused apply" if apply_launches == 4 else
+                               "call = segment build, fused shrink + apply kernel")},
             "roofline": {"bound": "hbm", "kernel": "merge_rows_kernel", "achieved": round(kern_gbs, 2),
                          "peak": peak, "unit": "GB/s", "frac": round(kern_gbs / peak, 4),
                          "peak_source": f"{peak_kind} hbm_gbs (burst copy)",
@@ -901,7 +904,7 @@ def main():
                 "apply_fused_kernel": rec_apply.get("tensor_pipe_pct") if rec_apply else None,
                 "source": "ncu sm__pipe_tensor_cycles_active (% of peak) of a small capture of this kernel "
                           "build (2-layer merge, 4-layer apply); null when the sources changed since"},
-            "gpu_launches": 5 * args.steps,
+            "gpu_launches": (3 + apply_launches) * args.steps,
             "clocks": clocks,
             "e2e": e2e,
             "cpu_baseline": cpu,
