@@ -966,6 +966,10 @@ int launch_merge_fused(Plan* p, const int32_t* idx0, const float* gate0, const i
         const bool long_walk = p->merge_tiles >= 128 * (int64_t)p->num_sms;
         const bool tb = long_walk && a.Kp >= 64 && a.Kp % 32 == 0;
         const uint32_t bc = tb ? 0u : at;                    // smem per Bcat block
+        // Up to four W stages; a fifth in the switch (in place) with the B rows
+        // in TMEM, where it measured faster (13B switch 10.6 -> 10.2 ms, 7B
+        // switch 5.05 -> 4.90 ms) while it slowed the 13B merge (8.87 -> 9.38).
+        const int64_t sw_cap = (tb && a.mode == 1) ? 5 : 4;
         int SW = 0, NA = 0, NAR = 0, G = 0;
         for (int g : {8, 4, 2, 1}) {
             if (g >= 4 && !long_walk) continue;
@@ -973,7 +977,7 @@ int launch_merge_fused(Plan* p, const int32_t* idx0, const float* gate0, const i
                 if (tb && np * g * (a.Kp / 2) > 256) continue;
                 for (int nar : {3, 2}) {
                     const int64_t room = (int64_t)kSmemMax - 2048 - (int64_t)np * g * bc - (int64_t)nar * at;
-                    const int sw = room > 0 ? (int)std::min<int64_t>(4, room / kWTileBytes) : 0;
+                    const int sw = room > 0 ? (int)std::min<int64_t>(sw_cap, room / kWTileBytes) : 0;
                     if (sw > SW) { SW = sw; NA = np * g; NAR = nar; G = g; }
                 }
             }

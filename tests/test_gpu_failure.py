@@ -52,9 +52,11 @@ def test_stalled_merge_times_out_and_reports(am, cuda_device):
         assert_close_bf16(u16(m.W_out[l]), ref, f"after timeout, linear {l}")
 
 
-def test_stalled_apply_times_out_and_reports(am, cuda_device):
-    T = 24
-    cfg = synth.custom([(512, 384), (256, 136)], 4, 16, 2, T, name="stall-apply")
+# T = 4: the two-launch form (the other CTAs' waits for the stalled shrink
+# output run out as well); T = 24: four launches
+@pytest.mark.parametrize("T", [4, 24])
+def test_stalled_apply_times_out_and_reports(am, cuda_device, T):
+    cfg = synth.custom([(512, 384), (256, 136)], 4, 16, 2, T, name=f"stall-apply{T}")
     w = synth.make_weights(cfg, 1, device=cuda_device)
     W_out = [torch.zeros_like(t) for t in w.W_views]
     X, xs = synth.make_apply_inputs(cfg, T, 2, device=cuda_device)

@@ -416,9 +416,10 @@ def test_apply_unit_heights_unsplit(am, cuda_device, T):
     assert m.plan.status() == (0, 0)
 
 
-def test_apply_zero_gates_poison_bad_and_duplicate(am, cuda_device):
-    T = 24
-    cfg = synth.custom([(264, 392)], 6, 16, 2, T, name="aedge")
+# T = 6: the two-launch form (shrink inside the apply kernel); T = 24: four launches
+@pytest.mark.parametrize("T", [6, 24])
+def test_apply_zero_gates_poison_bad_and_duplicate(am, cuda_device, T):
+    cfg = synth.custom([(264, 392)], 6, 16, 2, T, name=f"aedge{T}")
     m, xs, xs_dev, ys, xp, yp, idx, gate, ws = apply_setup(cfg, cuda_device, T)
     idx = idx.clone()
     gate = gate.clone()
