@@ -954,7 +954,8 @@ __global__ void __launch_bounds__(ApplyShape<H>::kThreads, 1) apply_fused_kernel
                 split_range(nKb + nKe, a.nsplit, sp, kc0, kc1);
             }
             float* part = a.Yp + ((int64_t)ua * a.Npad) * kApplyRows + rin;
-            for (int c0 = 0; c0 < a.Npad; c0 += 32) {
+            const int n_tok = (int)min((int64_t)a.Npad, T - tb);     // the tile's tokens, without padding
+            for (int c0 = 0; c0 < n_tok; c0 += 32) {
                 uint32_t v[32];
                 if (kc0 == kc1) {
 #pragma unroll
@@ -965,9 +966,9 @@ __global__ void __launch_bounds__(ApplyShape<H>::kThreads, 1) apply_fused_kernel
                 if (a.nsplit > 1) {
 #pragma unroll
                     for (int i = 0; i < 32; ++i)
-                        if (c0 + i < a.Npad) part[(int64_t)(c0 + i) * kApplyRows] = __uint_as_float(v[i]);
+                        if (c0 + i < n_tok) part[(int64_t)(c0 + i) * kApplyRows] = __uint_as_float(v[i]);
                 } else if (row < d_out) {
-                    store_y_rows(y, a.y_f32, (tb + c0) * d_out + row, d_out, min(32, a.Npad - c0), T - tb - c0, v);
+                    store_y_rows(y, a.y_f32, (tb + c0) * d_out + row, d_out, n_tok - c0, n_tok - c0, v);
                 }
             }
             tc_fence_before();
@@ -984,27 +985,40 @@ __global__ void __launch_bounds__(ApplyShape<H>::kThreads, 1) apply_fused_kernel
                 if (last) {
                     __threadfence();
                     const float* p0 = a.Yp + ((int64_t)g * a.nsplit * a.Npad) * kApplyRows + rin;
-                    for (int c0 = 0; c0 < a.Npad; c0 += 32) {
-                        // 32 independent loads per split in flight; each sum
+                    for (int c0 = 0; c0 < n_tok; c0 += 16) {
+                        // 16 tokens x 4 splits of loads in flight (one L2
+                        // round trip per 4 splits, not per split); each sum
                         // still runs over the splits in order
-                        float v[32];
+                        float v[16];
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) v[i] = 0.f;
-                        for (int s2 = 0; s2 < a.nsplit; ++s2) {
-                            const float* ps = p0 + ((int64_t)s2 * a.Npad + c0) * kApplyRows;
-                            float t[32];
+                        for (int i = 0; i < 16; ++i) v[i] = 0.f;
+                        for (int s0 = 0; s0 < a.nsplit; s0 += 4) {
+                            float t[4][16];
 #pragma unroll
-                            for (int i = 0; i < 32; ++i)
-                                t[i] = (c0 + i < a.Npad) ? __ldcg(ps + (int64_t)i * kApplyRows) : 0.f;
+                            for (int j = 0; j < 4; ++j)
 #pragma unroll
-                            for (int i = 0; i < 32; ++i) v[i] += t[i];
+                                for (int i = 0; i < 16; ++i)
+                                    t[j][i] = (s0 + j < a.nsplit && c0 + i < n_tok)
+                                                  ? __ldcg(p0 + ((int64_t)(s0 + j) * a.Npad + c0 + i) * kApplyRows)
+                                                  : 0.f;
+#pragma unroll
+                            for (int j = 0; j < 4; ++j)
+                                if (s0 + j < a.nsplit) {
+#pragma unroll
+                                    for (int i = 0; i < 16; ++i) v[i] += t[j][i];
+                                }
                         }
                         if (row < d_out) {
-                            uint32_t vb[32];
+                            const int64_t off = (tb + c0) * d_out + row;
 #pragma unroll
-                            for (int i = 0; i < 32; ++i) vb[i] = __float_as_uint(v[i]);
-                            store_y_rows(y, a.y_f32, (tb + c0) * d_out + row, d_out, min(32, a.Npad - c0),
-                                         T - tb - c0, vb);
+                            for (int i = 0; i < 16; ++i) {
+                                if (c0 + i >= n_tok) break;
+                                if (a.y_f32)
+                                    static_cast<float*>(y)[off + (int64_t)i * d_out] = v[i];
+                                else
+                                    static_cast<uint16_t*>(y)[off + (int64_t)i * d_out] =
+                                        __bfloat16_as_ushort(__float2bfloat16_rn(v[i]));
+                            }
                         }
                     }
                 }
