@@ -610,8 +610,11 @@ __global__ void __launch_bounds__(ApplyShape<H>::kThreads, 1) apply_fused_kernel
     int* s_unit = reinterpret_cast<int*>(tmem_slot + 4);       // [kUnitRing]
     int* s_used = s_unit + kUnitRing;                           // [1 + kMaxE]
     int* s_loads = s_used + 1 + kMaxE;                          // [kTileM / 8]: A loads of a shrink chunk
+    int* s_first = s_loads + kTileM / 8;                        // [2]: first unit, its stages loaded early
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int total = a.n_sh + a.n_units * a.n_tt * a.nsplit;
+    const uint32_t xbytes = (uint32_t)a.Npad * 128u;
     if (threadIdx.x == 0) {
         for (int i = 0; i < a.ST; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
         for (int i = 0; i < 2; ++i) { mbar_init(&accfull[i], 1); mbar_init(&accempty[i], kApplyEpiWarps); }
@@ -619,9 +622,40 @@ __global__ void __launch_bounds__(ApplyShape<H>::kThreads, 1) apply_fused_kernel
         mbar_init(donebar, 1);
         *abort_flag = 0;
         fence_mbar_init();
+        // The CTA's first unit, and for an apply unit the W and x of its first
+        // stages, before the wait: no launch of the call writes W or x, the
+        // base chunk range does not depend on the selection, and the kernel
+        // this one follows has itself waited for every earlier launch of the
+        // stream (whose last CTA also put the work counter back to zero).
+        int u = atomicAdd(&a.sched[0], 1);
+        if (u >= total) u = -1;
+        int ne = 0;
+        if (u >= a.n_sh) {
+            const int ua = u - a.n_sh;
+            const int g = ua / a.nsplit, sp = ua - g * a.nsplit;
+            const int tt = g / a.n_units;
+            const int2 lm = a.order[g - tt * a.n_units];
+            const int nKb = (__ldg(&a.lins[lm.x].d_in) + kChunkK - 1) / kChunkK;
+            int b0, b1;
+            split_range(nKb, a.nsplit, sp, b0, b1);
+            ne = min(a.ST, b1 - b0);
+            const CUtensorMap* mW = a.maps + (size_t)lm.x * kMapsPerLinear + kMapW;
+            for (int i = 0; i < ne; ++i) {
+                if (a.stall && blockIdx.x == 0 && i == 0) continue;      // test hook (below)
+                uint8_t* dst = base + (size_t)i * a.stage_bytes;
+                mbar_arrive_expect_tx(&full[i], kAChunkBytes * H + xbytes);
+                for (int hh = 0; hh < H; ++hh)
+                    tma_load_2d(dst + hh * kAChunkBytes, mW, &full[i], (b0 + i) * kChunkK, lm.y * kApplyRows + hh * kTileM);
+                tma_load_2d(dst + kAChunkBytes * H, a.xmaps + lm.x, &full[i], (b0 + i) * kChunkK, tt * a.tile);
+            }
+        }
+        s_first[0] = u;
+        s_first[1] = ne;
     }
-    // Zero the A regions: expert chunks load only the 8-column groups they use.
-    for (int s = 0; s < a.ST; ++s)
+    __syncthreads();
+    // Zero the A regions the early loads leave alone: expert chunks load only
+    // the 8-column groups they use (a stage that held W keeps finite values).
+    for (int s = s_first[1]; s < a.ST; ++s)
         for (uint32_t o = threadIdx.x * 16; o < kAChunkBytes * H; o += kApplyThreads * 16)
             st_shared_v4(smem_u32(base + (size_t)s * a.stage_bytes + o), make_uint4(0, 0, 0, 0));
     fence_proxy_async_smem();
@@ -643,9 +677,6 @@ __global__ void __launch_bounds__(ApplyShape<H>::kThreads, 1) apply_fused_kernel
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
-    const int total = a.n_sh + a.n_units * a.n_tt * a.nsplit;
-    const uint32_t xbytes = (uint32_t)a.Npad * 128u;
-
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
@@ -655,7 +686,7 @@ __global__ void __launch_bounds__(ApplyShape<H>::kThreads, 1) apply_fused_kernel
             for (int ui = 0; !stop; ++ui) {
                 const int j = ui & (kUnitRing - 1);
                 if (!mbar_wait(&uempty[j], (uint32_t)((ui / kUnitRing) & 1) ^ 1u, abort_flag)) break;
-                int u = atomicAdd(&a.sched[0], 1);
+                int u = ui == 0 ? s_first[0] : atomicAdd(&a.sched[0], 1);
                 if (u >= total) u = -1;
                 s_unit[j] = u;
                 mbar_arrive(&ufull[j]);
@@ -723,8 +754,12 @@ __global__ void __launch_bounds__(ApplyShape<H>::kThreads, 1) apply_fused_kernel
                 const int2 lm = a.order[g - tt * a.n_units];
                 const int l = lm.x;
                 const int nKb = (__ldg(&a.lins[l].d_in) + kChunkK - 1) / kChunkK;
-                int c0, c1;
-                split_range(nKb + nKe, a.nsplit, sp, c0, c1);
+                // the split's base chunks, then its share of the expand chunks
+                int b0, b1, e0, e1;
+                split_range(nKb, a.nsplit, sp, b0, b1);
+                split_range(nKe, a.nsplit, sp, e0, e1);
+                const int nb = b1 - b0, nc = nb + (e1 - e0);
+                const int n_early = ui == 0 ? s_first[1] : 0;
                 const int m0 = lm.y * kApplyRows;
                 const int t0 = tt * a.tile;
                 const CUtensorMap* mW = a.maps + (size_t)l * kMapsPerLinear + kMapW;
@@ -733,7 +768,12 @@ __global__ void __launch_bounds__(ApplyShape<H>::kThreads, 1) apply_fused_kernel
                 const CUtensorMap* mB32 = a.maps + (size_t)l * kMapsPerLinear + kMapB32;
                 const CUtensorMap* mX = a.xmaps + l;
                 bool s_ready = false;
-                for (int kc = c0; kc < c1; ++kc, ++gc) {
+                for (int jc = 0; jc < nc; ++jc, ++gc) {
+                    const int kc = jc < nb ? b0 + jc : nKb + e0 + (jc - nb);
+                    if (jc < n_early) {                 // loaded before the wait
+                        if (!(a.stall && blockIdx.x == 0 && gc == 0)) issued = gc + 1;
+                        continue;
+                    }
                     const int s = (int)(gc % a.ST);
                     if (kFused && kc >= nKb && !s_ready) {
                         // S of this linear and token tile: every 32-row slice
@@ -802,7 +842,7 @@ __global__ void __launch_bounds__(ApplyShape<H>::kThreads, 1) apply_fused_kernel
                 const int u = s_unit[j];
                 mbar_arrive(&uempty[j]);
                 if (u < 0) break;
-                int c0 = 0, c1 = 0, nKb = 0;
+                int c0 = 0, c1 = 0, nKb = 0, b0 = 0, b1 = 0, e0 = 0, e1 = 0;
                 const bool shrink = kFused && u < a.n_sh;
                 if (shrink) {
                     const int tt = u / a.n_su;
@@ -814,13 +854,18 @@ __global__ void __launch_bounds__(ApplyShape<H>::kThreads, 1) apply_fused_kernel
                     const int g = ua / a.nsplit, sp = ua - g * a.nsplit;
                     const int l = a.order[g % a.n_units].x;
                     nKb = (__ldg(&a.lins[l].d_in) + kChunkK - 1) / kChunkK;
-                    split_range(nKb + nKe, a.nsplit, sp, c0, c1);
+                    split_range(nKb, a.nsplit, sp, b0, b1);
+                    split_range(nKe, a.nsplit, sp, e0, e1);
+                    c1 = (b1 - b0) + (e1 - e0);
                 }
                 const int acc = ui & 1;
                 if (!mbar_wait(&accempty[acc], (uint32_t)((ui >> 1) & 1) ^ 1u, abort_flag)) break;
                 tc_fence_after();
                 const uint32_t d = tmem_base + (uint32_t)acc * a.acc_stride;
-                for (int kc = c0; kc < c1; ++kc, ++gc) {
+                for (int jc = c0; jc < c1; ++jc, ++gc) {
+                    // shrink: chunk jc of the K-slice; apply: the split's base
+                    // chunks, then its expand chunks
+                    const int kc = shrink ? jc : jc < b1 - b0 ? b0 + jc : nKb + e0 + (jc - (b1 - b0));
                     const int s = (int)(gc % a.ST);
                     if (!mbar_wait(&full[s], (uint32_t)((gc / a.ST) & 1), abort_flag)) { stop = true; break; }
                     tc_fence_after();
@@ -831,7 +876,7 @@ __global__ void __launch_bounds__(ApplyShape<H>::kThreads, 1) apply_fused_kernel
                         for (int kk = 0; kk < kChunkK / 16; ++kk)
                             tc_mma_bf16(d, make_sdesc(abase + (uint32_t)kk * 32u, 16u, 1024u, kLayoutSw128),
                                         make_sdesc(baddr + (uint32_t)kk * 32u, 16u, 1024u, kLayoutSw128), idesc,
-                                        (kc != c0 || kk) ? 1u : 0u);
+                                        (jc != c0 || kk) ? 1u : 0u);
                         tc_commit(&empty[s]);
                         continue;
                     }
@@ -844,7 +889,7 @@ __global__ void __launch_bounds__(ApplyShape<H>::kThreads, 1) apply_fused_kernel
                             for (int kk = 0; kk < kChunkK / 16; ++kk)
                                 tc_mma_bf16(d_h, make_sdesc(aaddr + (uint32_t)kk * 32u, 16u, 1024u, kLayoutSw128),
                                             make_sdesc(baddr + (uint32_t)kk * 32u, 16u, 1024u, kLayoutSw128), idesc,
-                                            (kc != c0 || kk) ? 1u : 0u);
+                                            (jc != c0 || kk) ? 1u : 0u);
                         } else {
                             // K steps 0-1 of the S chunk hold the hi half, 2-3 the
                             // lo half; both multiply the same 32 Bcat columns,
@@ -860,7 +905,7 @@ __global__ void __launch_bounds__(ApplyShape<H>::kThreads, 1) apply_fused_kernel
                                     : bmode == 1 ? make_sdesc(aaddr + k2 * 4096u, 16u, 256u, kLayoutSw32)
                                                  : make_sdesc(aaddr + k2 * 32u, 16u, 512u, kLayoutSw64);
                                 tc_mma_bf16(d_h, adesc, make_sdesc(baddr + (uint32_t)kk * 32u, 16u, 1024u, kLayoutSw128),
-                                            idesc, (kc != c0 || kk) ? 1u : 0u);
+                                            idesc, (jc != c0 || kk) ? 1u : 0u);
                             }
                         }
                     }
@@ -948,10 +993,13 @@ __global__ void __launch_bounds__(ApplyShape<H>::kThreads, 1) apply_fused_kernel
             const int row = lm.y * kApplyRows + rin;
             const int64_t tb = (int64_t)tt * a.tile;
             const uint32_t tbase = tacc + (uint32_t)(hh * a.Npad);
-            int kc0 = 0, kc1 = 1;
+            int kc0 = 0, kc1 = 1;                              // chunks of the split: none means a zero share
             if (a.nsplit > 1) {
                 const int nKb = (__ldg(&a.lins[lm.x].d_in) + kChunkK - 1) / kChunkK;
-                split_range(nKb + nKe, a.nsplit, sp, kc0, kc1);
+                int b0, b1, e0, e1;
+                split_range(nKb, a.nsplit, sp, b0, b1);
+                split_range(nKe, a.nsplit, sp, e0, e1);
+                kc1 = (b1 - b0) + (e1 - e0);
             }
             float* part = a.Yp + ((int64_t)ua * a.Npad) * kApplyRows + rin;
             const int n_tok = (int)min((int64_t)a.Npad, T - tb);     // the tile's tokens, without padding
