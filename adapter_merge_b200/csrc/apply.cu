@@ -417,8 +417,17 @@ __global__ void __launch_bounds__(128) shrink_finalize_kernel(const LinDesc* lin
             if (coef != 0.f) {
                 const int mq = c / kTileM, cl = c - mq * kTileM;
                 const float* p = P + (((int64_t)tt * n_su + (int64_t)mq * total_ks + ks_base) * Npad + tl) * kTileM + cl;
+                // 8 K-slices of loads in flight; the sum still runs over them in order
                 float sum = 0.f;
-                for (int ks = 0; ks < n_ks; ++ks) sum += p[(int64_t)ks * Npad * kTileM];
+                for (int ks0 = 0; ks0 < n_ks; ks0 += 8) {
+                    float t8[8];
+#pragma unroll
+                    for (int q2 = 0; q2 < 8; ++q2)
+                        t8[q2] = ks0 + q2 < n_ks ? p[(int64_t)(ks0 + q2) * Npad * kTileM] : 0.f;
+#pragma unroll
+                    for (int q2 = 0; q2 < 8; ++q2)
+                        if (ks0 + q2 < n_ks) sum += t8[q2];
+                }
                 v = coef * sum;
             }
         }
@@ -557,13 +566,23 @@ __device__ __forceinline__ void finalize_slice(const ApplyArgs& a, const int* s_
                 for (int s = 0; s < a.k; ++s)
                     if (__ldg(&a.idx[t * a.k + s]) == e) coef[j] += __ldg(&a.gate[t * a.k + s]);
         }
-        for (int ks = 0; ks < n_ks; ++ks) {
-            float v[kTok];
+        // 8 K-slices x kTok tokens of partials in flight per L2 round trip;
+        // each sum still runs over the slices in order
+        for (int ks0 = 0; ks0 < n_ks; ks0 += 8) {
+            float v[8][kTok];
 #pragma unroll
-            for (int j = 0; j < kTok; ++j)
-                v[j] = (coef[j] != 0.f) ? __ldcg(p + (int64_t)ks * slice + (int64_t)(tl0 + j) * kTileM) : 0.f;
+            for (int q2 = 0; q2 < 8; ++q2)
 #pragma unroll
-            for (int j = 0; j < kTok; ++j) sum[j] += v[j];
+                for (int j = 0; j < kTok; ++j)
+                    v[q2][j] = (ks0 + q2 < n_ks && coef[j] != 0.f)
+                                   ? __ldcg(p + (int64_t)(ks0 + q2) * slice + (int64_t)(tl0 + j) * kTileM)
+                                   : 0.f;
+#pragma unroll
+            for (int q2 = 0; q2 < 8; ++q2)
+                if (ks0 + q2 < n_ks) {
+#pragma unroll
+                    for (int j = 0; j < kTok; ++j) sum[j] += v[q2][j];
+                }
         }
 #pragma unroll
         for (int j = 0; j < kTok; ++j) {
