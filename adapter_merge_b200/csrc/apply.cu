@@ -657,7 +657,10 @@ __global__ void __launch_bounds__(ApplyShape<H>::kThreads, 1) apply_fused_kernel
             const int nKb = (__ldg(&a.lins[lm.x].d_in) + kChunkK - 1) / kChunkK;
             int b0, b1;
             split_range(nKb, a.nsplit, sp, b0, b1);
-            ne = min(a.ST, b1 - b0);
+            // at most four stages: a whole ring from every CTA at once queues
+            // the shrink's and finalize's loads behind it (sweep T = 1: 29.7 ->
+            // 27.8 us with four, T = 16: 37.0 -> 36.0 us)
+            ne = min(min(4, a.ST), b1 - b0);
             const CUtensorMap* mW = a.maps + (size_t)lm.x * kMapsPerLinear + kMapW;
             for (int i = 0; i < ne; ++i) {
                 if (a.stall && blockIdx.x == 0 && i == 0) continue;      // test hook (below)
