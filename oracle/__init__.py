@@ -161,6 +161,23 @@ def pregate(x_bits, W_r, k, b_r=None, renorm=False, pool=False):
     return idx, gate, z
 
 
+def topk_margin(z: np.ndarray, k: int) -> np.ndarray:
+    """Per row of logits z [T, E]: z_(k) - z_(k+1), the gap between the k-th
+    and the (k+1)-th largest logit (inf when k == E).  A selection whose gap
+    is within the rounding of the logit sum depends on the summation order."""
+    zs = -np.sort(-np.asarray(z, dtype=np.float64), axis=1)
+    if k >= zs.shape[1]:
+        return np.full(zs.shape[0], np.inf)
+    return zs[:, k - 1] - zs[:, k]
+
+
+def router_scale(x_bits, W_r: np.ndarray) -> np.ndarray:
+    """Per row of x [T, H]: max over experts of sum_j |x_j| |W_r[e, j]|, the
+    scale the rounding error of a logit is proportional to."""
+    x = bf16_to_f64(_u16(x_bits))
+    return (np.abs(x) @ np.abs(np.asarray(W_r, dtype=np.float64)).T).max(axis=1)
+
+
 # ------------------------------------------------------------------ merge
 
 def merge_linear(W_bits, A_bits, B_bits, eidx: Sequence[int], gates: Sequence[float],

@@ -176,9 +176,13 @@ def make_weights(cfg: Config, seed: int = 0, device="cpu", zero_w: bool = False)
         Av.append(A[oa:oa + n].view(E, r, l.d_in)); oa += n
         n = E * l.d_out * r
         Bv.append(B[ob:ob + n].view(E, l.d_out, r)); ob += n
-    W_r = normal((E, cfg.hidden), 1.0 / math.sqrt(cfg.hidden), torch.float32, seed,
-                 f"{cfg.name}/Wr", device=device)
-    return Weights(W, A, B, Wv, Av, Bv, W_r)
+    return Weights(W, A, B, Wv, Av, Bv, make_router_weights(cfg, seed, device))
+
+
+def make_router_weights(cfg: Config, seed: int = 0, device="cpu") -> torch.Tensor:
+    """[E, H] fp32 router weights, N(0, 1/sqrt(H)) (the W_r of make_weights)."""
+    return normal((cfg.E, cfg.hidden), 1.0 / math.sqrt(cfg.hidden), torch.float32, seed,
+                  f"{cfg.name}/Wr", device=device)
 
 
 def make_router_input(cfg: Config, T: int, seed: int = 0, device="cpu", tag="xr") -> torch.Tensor:

@@ -114,3 +114,27 @@ def test_sweep_summary_groups_by_depth_and_batch():
     assert s["merge_by_kr"]["32"]["us"] == 30.0
     assert s["apply_by_T"]["16"]["points"] == 3 and s["apply_by_T"]["1"]["us"] == 23.0
     assert s["points"] == 3 and s["seconds"] == 12.3
+
+
+def test_near_tie_report_of_the_bench_router_workloads():
+    """The oracle's near-tie report over the router inputs the bench draws
+    (the request row and the decode batch of every 7B rank's seed, the 13B
+    workload): the workloads with near-tie rows are exactly the ones the GPU
+    near-tie test runs, so none is accepted without an exact-order check."""
+    import math
+    import numpy as np
+    import oracle
+    import synth
+    from helpers import NEAR_TIE_RTOL, NEAR_TIE_SEEDS_7B, u16
+    found = []
+    for cfg, seeds in ((synth.llama7b(), [1000 + r for r in range(8)]), (synth.llama13b(), [1300])):
+        for seed in seeds:
+            W_r = synth.make_router_weights(cfg, seed).numpy()
+            for tag, T in (("xreq", 1), ("xfirst", cfg.T_apply)):
+                x = u16(synth.make_router_input(cfg, T, seed, tag=tag))
+                _, _, z = oracle.pregate(x, W_r, cfg.k)
+                rel = oracle.topk_margin(z, cfg.k) / oracle.router_scale(x, W_r)
+                assert np.all(np.isfinite(rel)) and math.isfinite(float(rel.min()))
+                if (rel < NEAR_TIE_RTOL).any():
+                    found.append((cfg.name, seed, tag))
+    assert found == [("llama2-7b", s, "xfirst") for s in NEAR_TIE_SEEDS_7B]

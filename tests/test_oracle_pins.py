@@ -118,6 +118,18 @@ def test_bf16_rounding_single_step_from_double():
 
 # ----------------------------------------------------------------- router
 
+def test_topk_margin_and_router_scale_handworked():
+    """The near-tie report: z_(k) - z_(k+1) per row (inf when k = E), and the
+    scale max_e sum_j |x_j||W_r[e, j]|, on values worked by hand."""
+    z = np.array([[3.0, 1.0, 2.0, 0.0], [0.5, 0.5, -1.0, 2.0]], dtype=np.float32)
+    assert oracle.topk_margin(z, 2).tolist() == [1.0, 0.0]          # sorted 3,2,1,0 and 2,.5,.5,-1
+    assert oracle.topk_margin(z, 1).tolist() == [1.0, 1.5]
+    assert np.all(np.isinf(oracle.topk_margin(z, 4)))
+    x = np.array([[0x3F80, 0xC000]], dtype=np.uint16)                # bf16 1.0, -2.0
+    W = np.array([[0.5, 0.25], [1.0, -1.0]])
+    assert oracle.router_scale(x, W).tolist() == [3.0]               # max(0.5 + 0.5, 1 + 2)
+
+
 def test_router_handworked():
     g = _golden()
     for key in ("router", "router_tie"):
