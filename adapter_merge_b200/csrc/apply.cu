@@ -5,36 +5,40 @@
 // section 2.B); the pages print no formula for the unmerged form, so it is the
 // plain mixed-batch LoRA product above, per token with that token's top-k.
 //
-// Two launches per call, independent of the number of layers:
+// Launches per call, independent of the number of layers:
 //   1. segments  stable sort of the (token, slot) pairs by expert (segments.cu);
 //                gives the U experts the batch uses, and clears the counters
-//                that launch 2 synchronises through;
-//   2. apply     one persistent tcgen05 kernel over two kinds of work unit,
-//                taken from one queue, shrink units first:
-//      shrink    (128-row tile of Acat, K-slice of a linear, token tile):
-//                the used experts' stacked A rows times x_l^T, fp32 partial
-//                to the workspace.  The warp that completes a 32-row slice of
-//                a tile last among its K-slices adds the slices in order,
-//                applies each token's gates and stores the result as a bf16
-//                hi/lo pair S_l[T, 2 * Kext] (hi and lo interleaved by groups
-//                of 32 columns), then counts the slice as done for its linear;
-//      apply     (linear, block of 128, 256 or 512 output rows, token tile):
+//                that the later launches synchronise through;
+// then, for plans with at least one apply unit per SM or more than 8 tokens:
+//   2. shrink    (128-row tile of Acat, K-slice of a linear, token tile):
+//                the used experts' stacked A rows times x_l^T on the tensor
+//                cores, fp32 partials to the workspace;
+//   3. finalize  per (linear, token): the K-slices added in order, the
+//                token's gates applied, stored as a bf16 hi/lo pair
+//                S_l[T, 2 * Kext] (hi and lo interleaved by groups of 32
+//                columns);
+//   4. apply     (linear, block of 128, 256 or 512 output rows, token tile):
 //                D[rows x Npad] = W_block x^T (d_in/64 swizzled K chunks)
 //                then + Bcat_block S^T (the used experts' B rows, gathered by
 //                TMA, against both halves of S), all in one fp32 TMEM
-//                accumulator, then y = bf16(D^T).  The producer loads the
-//                expand chunks only once every slice of its linear's S is
-//                done (a bounded wait that, coming after all shrink units in
-//                the queue, never waits on work that has not started).  Below
-//                one unit per SM, units are split along K and the last split
-//                of each 32-row slice adds the fp32 partials in split order.
+//                accumulator, then y = bf16(D^T);
+// and for smaller plans (a layer or a few, at most 8 tokens) the shrink units
+// run inside the apply kernel instead (two launches): queued before the apply
+// units, finalized by the warp that completes a 32-row slice last among its
+// K-slices, and the apply units load their expand chunks once every slice of
+// their linear's S is done (a bounded wait that, coming after all shrink
+// units in the queue, never waits on work that has not started).  Below one
+// unit per SM, units are split along K (a range of the base chunks and a
+// range of the expand chunks each) and the last split of each 32-row slice
+// adds the fp32 partials in split order.
 // Every operand moves by TMA: W and the experts' A and B rows through the
 // plan's tensor maps, x and S through per-call maps that the host builds (and
 // caches by pointer set, T, k and workspace) before the launches.  W is streamed
-// exactly once per token tile; the x and S tiles come from L2.  Both launches
-// use programmatic dependent launch: the apply kernel sets up its shared
-// memory while the segment build runs, and waits for it before touching
-// global memory.
+// exactly once per token tile; the x and S tiles come from L2.  All launches
+// use programmatic dependent launch: each kernel sets up its shared memory
+// while the previous one runs and waits for it before touching what it wrote;
+// the apply kernel also issues its first unit's first W and x loads before
+// that wait (no launch of the call writes W or x).
 #include <cudaTypedefs.h>
 
 #include <algorithm>
@@ -658,8 +662,8 @@ __global__ void __launch_bounds__(ApplyShape<H>::kThreads, 1) apply_fused_kernel
             int b0, b1;
             split_range(nKb, a.nsplit, sp, b0, b1);
             // at most four stages: a whole ring from every CTA at once queues
-            // the shrink's and finalize's loads behind it (sweep T = 1: 29.7 ->
-            // 27.8 us with four, T = 16: 37.0 -> 36.0 us)
+            // the shrink's and finalize's loads behind it (one 4096 x 4096
+            // layer: 29.7 -> 27.8 us at T = 1, 37.0 -> 36.0 us at T = 16)
             ne = min(min(4, a.ST), b1 - b0);
             const CUtensorMap* mW = a.maps + (size_t)lm.x * kMapsPerLinear + kMapW;
             for (int i = 0; i < ne; ++i) {
