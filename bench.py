@@ -46,6 +46,7 @@ def read_peaks():
     return FALLBACK_HBM_GBS, "fallback"
 
 
+E2E_CHUNKS = 32          # chunks of layers in the end-to-end merge through host memory
 RECORDS = os.path.join(ROOT, "profiles", "records.json")
 
 
@@ -709,10 +710,12 @@ def main():
         # layers through the same public calls (one plan and one merge call
         # per chunk): the copy in of chunk c+1, the merge of chunk c and the
         # copy out of chunk c-1 overlap on three streams, so the two PCIe
-        # directions run at once.
+        # directions run at once.  Only the first chunk's copy in and the
+        # last chunk's copy out stand alone, so the chunks are small: about
+        # one layer each.
         chunks = []
         if full:
-            per = max(1, len(cfg.linears) // 8)
+            per = max(1, len(cfg.linears) // E2E_CHUNKS)
             for c0 in range(0, len(cfg.linears), per):
                 c1 = min(len(cfg.linears), c0 + per)
                 ow = sum(l.d_out * l.d_in for l in cfg.linears[:c0])
@@ -794,7 +797,7 @@ def main():
                             "h2d_bytes_per_step": x_req.numel() * 2, "d2h_bytes_per_step": 2 * cfg.k * 4,
                             "note": "weights and adapters resident; only the router input and the selection cross"},
                "note": ("merge with W, A, B in and W' out through pinned host buffers each step, pipelined "
-                        "over 8 chunks of layers (a plan and a merge call per chunk; copies in, merges and "
+                        f"over {len(chunks)} chunks of layers (a plan and a merge call per chunk; copies in, merges and "
                         "copies out overlap on three streams); apply with x in and y out (weights "
                         "resident)") if full else
                        ("host memory holds no pinned model copy per rank: merge with the router input in and "
