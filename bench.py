@@ -726,8 +726,15 @@ def main():
                 nb = sum(cfg.E * l.d_out * cfg.r for l in cfg.linears[c0:c1])
                 cplan = am.Plan(list(zip(w.W_views[c0:c1], W_out_views[c0:c1], w.A_views[c0:c1],
                                          w.B_views[c0:c1])), cfg.E, cfg.r)
-                chunks.append((cplan, slice(ow, ow + nw), slice(oa, oa + na), slice(ob, ob + nb)))
+                ox = sum(T * l.d_in for l in cfg.linears[:c0])
+                nx = sum(T * l.d_in for l in cfg.linears[c0:c1])
+                oy = sum(T * l.d_out for l in cfg.linears[:c0])
+                ny = sum(T * l.d_out for l in cfg.linears[c0:c1])
+                chunks.append((cplan, slice(ow, ow + nw), slice(oa, oa + na), slice(ob, ob + nb),
+                               slice(ox, ox + nx), slice(oy, oy + ny), am.PointerArrays(xs[c0:c1], ys[c0:c1])))
             s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+            # the chunks' applies run one after another on the stream: one workspace
+            ws_c = torch.empty(max(c[0].workspace_bytes(T, cfg.k) for c in chunks), dtype=torch.uint8, device=dev)
 
         def e2e_merge(ev, resident):
             ev[0].record(stream)
@@ -738,7 +745,7 @@ def main():
             else:
                 s_in.wait_stream(stream)
                 done_in, done_m = [], []
-                for (cplan, sw_, sa_, sb_) in chunks:
+                for (cplan, sw_, sa_, sb_, _sx, _sy, _xp) in chunks:
                     with torch.cuda.stream(s_in):
                         w.W[sw_].copy_(h_W[sw_], non_blocking=True)
                         w.A[sa_].copy_(h_A[sa_], non_blocking=True)
@@ -758,12 +765,31 @@ def main():
             ev[1].record(stream)
 
         def e2e_apply(ev):
+            # x in and y out, pipelined over the same chunks of layers as the
+            # merge (the copy in of chunk c+1, the apply of chunk c and the copy
+            # out of chunk c-1 overlap) when the chunk plans exist
             ev[0].record(stream)
             x_first.copy_(h_first, non_blocking=True)
-            X.copy_(h_X, non_blocking=True)
             idxT, gateT = am.pregate(x_first, w.W_r, cfg.k)
-            plan.apply(xp, yp, T, idxT, gateT, ws)
-            h_Y.copy_(Y, non_blocking=True)
+            if chunks:
+                s_in.wait_stream(stream)
+                for (cplan, _sw, _sa, _sb, sx_, sy_, xp_c) in chunks:
+                    with torch.cuda.stream(s_in):
+                        X[sx_].copy_(h_X[sx_], non_blocking=True)
+                        e_in = torch.cuda.Event()
+                        e_in.record(s_in)
+                    stream.wait_event(e_in)
+                    cplan.apply(xp_c, None, T, idxT, gateT, ws_c, stream=stream)
+                    e_a = torch.cuda.Event()
+                    e_a.record(stream)
+                    with torch.cuda.stream(s_out):
+                        s_out.wait_event(e_a)
+                        h_Y[sy_].copy_(Y[sy_], non_blocking=True)
+                stream.wait_stream(s_out)
+            else:
+                X.copy_(h_X, non_blocking=True)
+                plan.apply(xp, yp, T, idxT, gateT, ws)
+                h_Y.copy_(Y, non_blocking=True)
             h_sel[2].copy_(idxT[0].view(torch.float32), non_blocking=True)
             ev[1].record(stream)
 
@@ -798,14 +824,14 @@ def main():
                             "note": "weights and adapters resident; only the router input and the selection cross"},
                "note": ("merge with W, A, B in and W' out through pinned host buffers each step, pipelined "
                         f"over {len(chunks)} chunks of layers (a plan and a merge call per chunk; copies in, merges and "
-                        "copies out overlap on three streams); apply with x in and y out (weights "
-                        "resident)") if full else
+                        "copies out overlap on three streams); apply with x in and y out, pipelined over the "
+                        "same chunks (weights resident)") if full else
                        ("host memory holds no pinned model copy per rank: merge with the router input in and "
                         "the selection out (weights resident); apply with x in and y out")}
         if full:
             for (cplan, *_rest) in chunks:
                 cplan.destroy()
-            del h_W, h_A, h_B, h_Wout, chunks
+            del h_W, h_A, h_B, h_Wout, chunks, ws_c
 
     # The NEXT rows on the same plan, outside the timed region: in-place switch
     # between two selections (rank 2kr), the one-launch-per-linear merge, and
