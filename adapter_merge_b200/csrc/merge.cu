@@ -501,6 +501,35 @@ struct GroupTileIt {
     __device__ bool group_last() const { return b == nb - 1 && strip == n_strips - 1; }
 };
 
+// Gate-scales the 16-byte chunks id = tid, tid + nthr, ... of a group's raw
+// B rows in shared memory (chunk id: block, 8-column group, row; four chunks
+// per step, their loads issued together); chunks of slots without an expert
+// and of the K padding become zeros.
+__device__ __forceinline__ void scale_bcat_chunks(uint8_t* gbase, int chunks, int groups, int r, int ns,
+                                                  const int* s_e, const float* s_g, int tid, int nthr)
+{
+    for (int id0 = tid; id0 < chunks; id0 += 4 * nthr) {
+        uint4 v[4];
+        float gs[4];
+        bool live[4], slot[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int id = id0 + u * nthr;
+            const int cg = (id / kTileM) % groups;
+            const int s2 = (cg * 8) / r;
+            live[u] = id < chunks;
+            slot[u] = live[u] && s2 < ns && s_e[s2] >= 0;
+            gs[u] = slot[u] ? s_g[s2] : 0.f;
+            v[u] = slot[u] ? ld_shared_v4(smem_u32(gbase) + (uint32_t)id * 16u) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            if (live[u])    // address = block*BcBytes + cg*2048 + row*16
+                st_shared_v4(smem_u32(gbase) + (uint32_t)(id0 + u * nthr) * 16u,
+                             slot[u] ? scale_bf16x8(v[u], gs[u]) : make_uint4(0, 0, 0, 0));
+    }
+}
+
 template <bool kTB>
 __global__ void __launch_bounds__(kTB ? kMergeThreadsTB : kMergeThreads, 1)
     merge_rows_kernel(const __grid_constant__ MergeArgs a)
@@ -521,7 +550,8 @@ __global__ void __launch_bounds__(kTB ? kMergeThreadsTB : kMergeThreads, 1)
     uint64_t* accfull = bcload + NP;
     uint64_t* accempty = accfull + 2;
     uint64_t* donebar = accempty + 2;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(donebar + 1);
+    uint64_t* b0done = donebar + 1;               // (smem Bcat) the epilogue warps' share of the first group scaled
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(b0done + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     int* s_skip = reinterpret_cast<int*>(tmem_slot + 2);
     volatile int* s_bfirst = reinterpret_cast<volatile int*>(tmem_slot + 3);   // first B-row loads issued
@@ -539,6 +569,7 @@ __global__ void __launch_bounds__(kTB ? kMergeThreadsTB : kMergeThreads, 1)
         for (int i = 0; i < NP; ++i) { mbar_init(&bcfull[i], kTB ? 4 : 2); mbar_init(&bcempty[i], 1); mbar_init(&bcload[i], 1); }
         for (int i = 0; i < 2; ++i) { mbar_init(&accfull[i], 1); mbar_init(&accempty[i], kEpiWarps); }
         mbar_init(donebar, 1);
+        mbar_init(b0done, kEpiWarps);
         *abort_flag = 0;
         *s_bfirst = 0;
         fence_mbar_init();
@@ -776,29 +807,17 @@ __global__ void __launch_bounds__(kTB ? kMergeThreadsTB : kMergeThreads, 1)
                     if (!ok) break;
                     const int groups = a.Kp / 8;
                     const int chunks = it.nb * groups * kTileM;      // 16-byte chunks: (block, column group, row)
-                    // four chunks per step, their loads issued together
-                    for (int id0 = tb; id0 < chunks; id0 += 4 * 64) {
-                        uint4 v[4];
-                        float gs[4];
-                        bool live[4], slot[4];
-#pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            const int id = id0 + u * 64;
-                            const int cg = (id / kTileM) % groups;
-                            const int s2 = (cg * 8) / a.r;
-                            live[u] = id < chunks;
-                            slot[u] = live[u] && s2 < a.ns && s_e[s2] >= 0;
-                            gs[u] = slot[u] ? s_g[s2] : 0.f;
-                            v[u] = slot[u] ? ld_shared_v4(smem_u32(gbase) + (uint32_t)id * 16u) : make_uint4(0, 0, 0, 0);
-                        }
-#pragma unroll
-                        for (int u = 0; u < 4; ++u)
-                            if (live[u])    // address = block*BcBytes + cg*2048 + row*16
-                                st_shared_v4(smem_u32(gbase) + (uint32_t)(id0 + u * 64) * 16u,
-                                             slot[u] ? scale_bf16x8(v[u], gs[u]) : make_uint4(0, 0, 0, 0));
-                    }
+                    // the first group with the eight epilogue warps (which
+                    // have no accumulator to read yet), the others alone
+                    const bool first = pseq == 0;
+                    scale_bcat_chunks(gbase, chunks, groups, a.r, a.ns, s_e, s_g, tb, first ? 64 + 32 * kEpiWarps : 64);
                     fence_proxy_async_smem();
                     __syncwarp();
+                    if (first) {
+                        ok = mbar_wait(b0done, 0u, abort_flag);
+                        ok = __all_sync(0xffffffffu, ok);
+                        if (!ok) break;
+                    }
                     if (lane == 0) mbar_arrive(&bcfull[ps]);
                 }
                 if (i + 1 < count) it.next(a.lins, a.n_lin);
@@ -809,6 +828,21 @@ __global__ void __launch_bounds__(kTB ? kMergeThreadsTB : kMergeThreads, 1)
         }
     } else if (warp >= 4 && warp < 4 + kEpiWarps) {
         // ------------------------------------------------------------ epilogue
+        if (!kTB && count > 0) {
+            // help the two builder warps scale the first group's B rows
+            GroupTileIt it0;
+            it0.init(a.lins, a.n_lin, t_begin, a.G);
+            bool ok = mbar_wait(&bcload[0], 0u, abort_flag);
+            ok = __all_sync(0xffffffffu, ok);
+            if (ok) {
+                const int groups = a.Kp / 8;
+                scale_bcat_chunks(sBcat, it0.nb * groups * kTileM, groups, a.r, a.ns, s_e, s_g,
+                                  64 + (warp - 4) * 32 + lane, 64 + 32 * kEpiWarps);
+                fence_proxy_async_smem();
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(b0done);
+        }
         const int ew = warp - 4;
         const int q = warp & 3;
         const int h = ew >> 2;
