@@ -275,6 +275,23 @@ def sweep_point_arg(text):
     return pt
 
 
+def chunk_slices(cfg, T, n_chunks):
+    """Chunks of consecutive linears for the end-to-end pipelines: per chunk
+    (first linear, end linear, and the slices of the flat W, A, B, x and y
+    buffers it covers), about n_chunks of them."""
+    per = max(1, len(cfg.linears) // n_chunks)
+    out = []
+    for c0 in range(0, len(cfg.linears), per):
+        c1 = min(len(cfg.linears), c0 + per)
+        def span(size):
+            o = sum(size(l) for l in cfg.linears[:c0])
+            return slice(o, o + sum(size(l) for l in cfg.linears[c0:c1]))
+        out.append((c0, c1, span(lambda l: l.d_out * l.d_in), span(lambda l: cfg.E * cfg.r * l.d_in),
+                    span(lambda l: cfg.E * l.d_out * cfg.r), span(lambda l: T * l.d_in),
+                    span(lambda l: T * l.d_out)))
+    return out
+
+
 def measure_sweep(dev, peak, only=None, NC=8, R=5, Ts=(1, 16, 128)):
     """The single-linear 4096 x 4096 grid: E in {4, 8, 16, 32}, r in {8, 16,
     32, 64}, k in {1, 2, 4}; merge per (E, r, k) and apply per T in Ts.  A
@@ -715,23 +732,10 @@ def main():
         # one layer each.
         chunks = []
         if full:
-            per = max(1, len(cfg.linears) // E2E_CHUNKS)
-            for c0 in range(0, len(cfg.linears), per):
-                c1 = min(len(cfg.linears), c0 + per)
-                ow = sum(l.d_out * l.d_in for l in cfg.linears[:c0])
-                nw = sum(l.d_out * l.d_in for l in cfg.linears[c0:c1])
-                oa = sum(cfg.E * cfg.r * l.d_in for l in cfg.linears[:c0])
-                na = sum(cfg.E * cfg.r * l.d_in for l in cfg.linears[c0:c1])
-                ob = sum(cfg.E * l.d_out * cfg.r for l in cfg.linears[:c0])
-                nb = sum(cfg.E * l.d_out * cfg.r for l in cfg.linears[c0:c1])
+            for (c0, c1, sw_, sa_, sb_, sx_, sy_) in chunk_slices(cfg, T, E2E_CHUNKS):
                 cplan = am.Plan(list(zip(w.W_views[c0:c1], W_out_views[c0:c1], w.A_views[c0:c1],
                                          w.B_views[c0:c1])), cfg.E, cfg.r)
-                ox = sum(T * l.d_in for l in cfg.linears[:c0])
-                nx = sum(T * l.d_in for l in cfg.linears[c0:c1])
-                oy = sum(T * l.d_out for l in cfg.linears[:c0])
-                ny = sum(T * l.d_out for l in cfg.linears[c0:c1])
-                chunks.append((cplan, slice(ow, ow + nw), slice(oa, oa + na), slice(ob, ob + nb),
-                               slice(ox, ox + nx), slice(oy, oy + ny), am.PointerArrays(xs[c0:c1], ys[c0:c1])))
+                chunks.append((cplan, sw_, sa_, sb_, sx_, sy_, am.PointerArrays(xs[c0:c1], ys[c0:c1])))
             s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
             # the chunks' applies run one after another on the stream: one workspace
             ws_c = torch.empty(max(c[0].workspace_bytes(T, cfg.k) for c in chunks), dtype=torch.uint8, device=dev)

@@ -138,3 +138,26 @@ def test_near_tie_report_of_the_bench_router_workloads():
                 if (rel < NEAR_TIE_RTOL).any():
                     found.append((cfg.name, seed, tag))
     assert found == [("llama2-7b", s, "xfirst") for s in NEAR_TIE_SEEDS_7B]
+
+
+def test_chunk_slices_tile_every_flat_buffer():
+    """The end-to-end pipelines' chunks of layers cover the flat W, A, B, x and
+    y buffers exactly once, in order, and each slice matches its linears."""
+    import bench
+    import synth
+    for cfg, T in ((synth.llama7b(), 64), (synth.llama13b(), 32), (synth.tiny(), 8)):
+        for n in (1, 8, 32, 1000):
+            ch = bench.chunk_slices(cfg, T, n)
+            assert ch[0][0] == 0 and ch[-1][1] == len(cfg.linears)
+            sizes = (lambda l: l.d_out * l.d_in, lambda l: cfg.E * cfg.r * l.d_in,
+                     lambda l: cfg.E * l.d_out * cfg.r, lambda l: T * l.d_in, lambda l: T * l.d_out)
+            for b, size in enumerate(sizes):
+                end = 0
+                for c in ch:
+                    sl = c[2 + b]
+                    assert sl.start == end
+                    assert sl.stop - sl.start == sum(size(l) for l in cfg.linears[c[0]:c[1]])
+                    end = sl.stop
+                assert end == sum(size(l) for l in cfg.linears)
+            for a, b in zip(ch, ch[1:]):
+                assert a[1] == b[0]
